@@ -1,0 +1,122 @@
+// frt_common.cuh -- host error plumbing and device numeric helpers shared by
+// the library's translation units.  Everything here is this library's own;
+// nothing is shared with the CPU oracle.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/frt.h"
+
+// ------------------------------------------------------------------ host --
+
+namespace frt {
+
+// Record a reason for the calling thread (read back by frt_last_error) and
+// return `code`, so validation reads `return fail(FRT_ESHAPE, "...")`.
+int fail(int code, const char* fmt, ...);
+void clear_error();
+// Map a CUDA error from a launch to FRT_ECUDA with the call site named.
+int check_launch(const char* what);
+// Device address of the library's device-side status word for the current
+// device (bounded waits that run out record their code there).
+int* device_status_ptr();
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms();
+
+inline bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+}  // namespace frt
+
+#define FRT_REQUIRE(cond, code, ...) \
+  do { if (!(cond)) return ::frt::fail((code), __VA_ARGS__); } while (0)
+
+// ---------------------------------------------------------------- device --
+
+namespace frt {
+
+__device__ __forceinline__ float bf2f(uint16_t h) {
+  return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+// fp32 -> bf16 bits, round to nearest even (the CUDA conversion intrinsic).
+__device__ __forceinline__ uint16_t f2bf(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two fp32 -> two e4m3fn codes (lo in the low byte), round to nearest even,
+// saturating to +-448: the hardware conversion, which equals clamp-then-round.
+__device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
+  return static_cast<uint16_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+// 8 bf16 packed in a uint4 -> 8 floats.
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(const float (&f)[8]) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                    pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+}
+
+// 8 floats already divided by the scale -> 8 e4m3 codes in a uint2.
+__device__ __forceinline__ uint2 pack8_e4m3(const float (&q)[8]) {
+  uint32_t lo = pack_e4m3x2(q[0], q[1]) | (uint32_t(pack_e4m3x2(q[2], q[3])) << 16);
+  uint32_t hi = pack_e4m3x2(q[4], q[5]) | (uint32_t(pack_e4m3x2(q[6], q[7])) << 16);
+  return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// |y| max into a device float holding non-negative values: the bit patterns
+// of non-negative floats order like unsigned integers.
+__device__ __forceinline__ void atomic_max_nonneg(float* dst, float v) {
+  atomicMax(reinterpret_cast<unsigned int*>(dst), __float_as_uint(v));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// gelu_tanh(g) * u with gelu_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x +
+// 0.044715 x^3))) (the tanh form of Hendrycks & Gimpel's GELU), every step
+// an explicitly rounded fp32 operation; tanh is CUDA's tanhf.
+__device__ __forceinline__ float gelu_tanh_mul(float g, float u) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+  const float k1 = 0.044715f;
+  const float g3 = __fmul_rn(__fmul_rn(g, g), g);
+  const float inner = __fmul_rn(k0, __fadd_rn(g, __fmul_rn(k1, g3)));
+  const float gl = __fmul_rn(__fmul_rn(0.5f, g), __fadd_rn(1.0f, tanhf(inner)));
+  return __fmul_rn(gl, u);
+}
+
+}  // namespace frt

@@ -1,0 +1,62 @@
+// geglu.cu -- a5 (standalone form): merged GEGLU + static FP8 requant.
+//
+// flashrt-structures 0.2.0, impls/adarms_stack/fp8_chain.py `down_project`
+// (the merged gate/up output gu [S, 2H] becomes hid8 [S, H] in one kernel,
+// quantized with the down projection's static input scale) and the bind
+// check that the FFN activation is the tanh-approximate GELU.
+// gelu_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), the tanh
+// form of Hendrycks & Gimpel's GELU (frt::gelu_tanh_mul, shared with the
+// fused GEMM epilogue so both forms give the same codes).
+#include "frt_common.cuh"
+
+namespace frt {
+
+namespace {
+
+__global__ void geglu_kernel(int M, int H, const uint16_t* gu, long ld, const float* out_scale,
+                             uint8_t* hid8, float* amax) {
+  const int h8 = H / 8;
+  const long total = long(M) * h8;
+  const float os = __ldg(out_scale);
+  float mx = 0.0f;
+  for (long g = blockIdx.x * long(blockDim.x) + threadIdx.x; g < total;
+       g += long(gridDim.x) * blockDim.x) {
+    const long m = g / h8;
+    const int c = int(g % h8);
+    float gv[8], uv[8], q[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(gu + m * ld + 8 * c)), gv);
+    unpack8(__ldg(reinterpret_cast<const uint4*>(gu + m * ld + H + 8 * c)), uv);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float h = gelu_tanh_mul(gv[j], uv[j]);
+      mx = fmaxf(mx, fabsf(h));
+      q[j] = __fdiv_rn(h, os);
+    }
+    *reinterpret_cast<uint2*>(hid8 + m * H + 8 * c) = pack8_e4m3(q);
+  }
+  if (amax) {
+    mx = warp_max(mx);
+    if ((threadIdx.x & 31) == 0) atomic_max_nonneg(amax, mx);
+  }
+}
+
+}  // namespace
+}  // namespace frt
+
+extern "C" int frt_geglu_quant_fp8(int M, int H, const frt_bf16* gu, long ld_gu,
+                                   const float* out_scale, frt_e4m3* hid8, float* amax_out,
+                                   void* stream) {
+  using frt::aligned;
+  frt::clear_error();
+  FRT_REQUIRE(M >= 0 && H > 0 && H % 8 == 0, FRT_ESHAPE, "H must be a positive multiple of 8");
+  FRT_REQUIRE(ld_gu >= 2L * H && ld_gu % 8 == 0, FRT_ESHAPE, "ld_gu must be >= 2H and a multiple of 8");
+  FRT_REQUIRE(gu && out_scale && hid8, FRT_EINVAL, "gu, out_scale and hid8 are required");
+  FRT_REQUIRE(aligned(gu, 16) && aligned(hid8, 8), FRT_EALIGN, "gu 16-byte, hid8 8-byte aligned");
+  if (M == 0) return FRT_OK;
+  const long total = long(M) * (H / 8);
+  const long need = (total + 255) / 256;
+  const int grid = int(need < frt::num_sms() * 16L ? need : frt::num_sms() * 16L);
+  frt::geglu_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(M, H, gu, ld_gu,
+                                                                         out_scale, hid8, amax_out);
+  return frt::check_launch("frt_geglu_quant_fp8");
+}

@@ -1,0 +1,654 @@
+// gemm.cu -- a2 (+ fused a3 / a5): the packed FP8 GEMM on sm_100a tensor
+// cores (tcgen05 MMA, TMEM accumulators, TMA operand loads).
+//
+// flashrt-structures 0.2.0, impls/qkv_pack/fp8_static.py (module docstring:
+// sibling GEMMs packed into one [sum N_i, K] matrix so the small-M group pays
+// one launch; `PackedLinear._run`: out = act_scale * w_scale * (x8 @ w8^T) +
+// bias in bf16) and impls/adarms_stack/fp8_chain.py (`norm_project` feeds
+// the FP8 wire straight into the GEMM; `_quantize` folds act_scale * w_scale
+// into alpha; `down_project` consumes the merged GEGLU requant).
+//
+// Design (one CTA per SM, persistent over work units):
+//   warp 0      one lane issues TMA loads of 128-byte-wide K slices of the A
+//               and B tiles into a STAGES-deep ring (128-byte swizzle);
+//   warp 1      allocates TMEM, one lane issues tcgen05.mma (M=128, N=BN,
+//               K=32, e4m3 x e4m3 -> fp32) into one of two TMEM accumulators;
+//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter, alpha, bias,
+//               bf16 / RoPE + KV scatter / GEGLU + e4m3, stores to HBM; the
+//               double-buffered accumulator lets it overlap the next unit's
+//               main loop.
+// Large M: A = x8 (tokens on TMEM lanes), B = w8, BN = 256 (or 128).
+// Small M (<= 128): swap A and B so the packed weights fill the 128 MMA rows
+// and the few tokens are the MMA N (16..128); K is split over CTAs so the
+// weight stream is spread across the SMs, and the CTA that finishes a tile
+// last sums the fp32 partials in split order (deterministic, no atomics on
+// data, no waiting between CTAs).
+// Every wait on an mbarrier is bounded in time; a wait that runs out records
+// FRT_ETIMEOUT, the CTA drains its in-flight copies and MMAs (again bounded),
+// frees its TMEM and returns.  No TMA multicast is used anywhere.
+#include <mutex>
+
+#include "frt_common.cuh"
+#include "frt_sm100.cuh"
+
+namespace frt {
+namespace {
+
+constexpr int BM = 128;             // MMA M = TMEM lanes
+constexpr int BK = 128;             // K bytes per stage: one swizzle row
+constexpr int kThreads = 192;
+constexpr int A_BYTES = BM * BK;    // 16 KB
+constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per wait
+constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s to drain after an abort
+
+enum { EPI_BF16 = 0, EPI_GEGLU = 1, EPI_ROPE = 2 };
+
+struct GemmParams {
+  int M, N, K;
+  int a_tiles, b_tiles, k_blocks, splits, units;
+  const float* act_scale;
+  const float* w_scale;
+  const uint16_t* bias;
+  int epi;
+  void* out;
+  long ldo;
+  const float* out_scale;
+  // split + RoPE + KV epilogue
+  int Mseq, hq, hkv, hd, P, T;
+  const uint16_t* rope;
+  uint16_t* q_out;
+  uint16_t* k_cache;
+  uint16_t* v_cache;
+  // split-K
+  float* partials;
+  unsigned* counters;
+  int* status;
+};
+
+__host__ __device__ constexpr uint32_t tmem_cols_for(int n) {
+  return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512;
+}
+
+template <int BN, int STAGES>
+constexpr int smem_bytes() {
+  return STAGES * (A_BYTES + BN * BK) + 1024 /* alignment slack */ + 256 /* barriers */;
+}
+
+__device__ __forceinline__ void record_timeout(int* status) {
+  if (status) atomicExch(status, FRT_ETIMEOUT);
+}
+
+// ---------------------------------------------------------------- epilogue --
+
+// y = bf16(acc * alpha [+ bias]) as a float (the value the unfused path
+// stores and the split kernel reads back).
+__device__ __forceinline__ float scale_bias_bf16(float acc, float alpha, const uint16_t* bias,
+                                                 int n) {
+  float y = __fmul_rn(acc, alpha);
+  if (bias) y = __fadd_rn(y, bf2f(__ldg(bias + n)));
+  return bf2f(f2bf(y));
+}
+
+// Normal orientation: this thread owns token row m, columns n0 .. n0 + 31.
+__device__ __forceinline__ void epi_rows_chunk(const GemmParams& p, const float (&v)[32], int m,
+                                               int n0, float alpha) {
+  if (m >= p.M) return;
+  float y[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) y[j] = scale_bias_bf16(v[j], alpha, p.bias, n0 + j);
+  uint16_t* dst;
+  if (p.epi == EPI_BF16) {
+    dst = static_cast<uint16_t*>(p.out) + long(m) * p.ldo + n0;
+  } else {  // EPI_ROPE: the 32 columns lie inside one head (hd % 32 == 0)
+    const int b = m / p.Mseq, s = m % p.Mseq;
+    const int h = n0 / p.hd, d0 = n0 % p.hd;
+    if (h < p.hq + p.hkv) {
+      const uint16_t* rp = p.rope + long(s) * p.hd + d0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float c = bf2f(__ldg(rp + 2 * i)), sn = bf2f(__ldg(rp + 2 * i + 1));
+        const float x0 = y[2 * i], x1 = y[2 * i + 1];
+        y[2 * i] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, sn));
+        y[2 * i + 1] = __fadd_rn(__fmul_rn(x0, sn), __fmul_rn(x1, c));
+      }
+      dst = h < p.hq ? p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d0
+                     : p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d0;
+    } else {
+      const int hv = h - p.hq - p.hkv;
+      dst = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + hv) * p.hd + d0;
+    }
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = y[8 * k + j];
+    d4[k] = pack8_bf16(f);
+  }
+}
+
+// Swapped orientation: this thread (lane) owns output column n, tokens
+// m0 .. m0 + 31.  Pairs (n, n ^ 1) live in neighbouring lanes.
+__device__ __forceinline__ void epi_cols_chunk(const GemmParams& p, const float (&v)[32], int n,
+                                               int m0, float alpha, int lane) {
+  const bool col_ok = n < p.N;
+  const float bias = (p.bias && col_ok) ? bf2f(__ldg(p.bias + n)) : 0.0f;
+  if (p.epi == EPI_BF16) {
+    if (!col_ok) return;
+    uint16_t* out = static_cast<uint16_t*>(p.out);
+#pragma unroll 4
+    for (int j = 0; j < 32; ++j) {
+      const int m = m0 + j;
+      if (m < p.M) {
+        float y = __fmul_rn(v[j], alpha);
+        if (p.bias) y = __fadd_rn(y, bias);
+        out[long(m) * p.ldo + n] = f2bf(y);
+      }
+    }
+    return;
+  }
+  // EPI_ROPE: the warp's 32 columns lie inside one head
+  const int h = n / p.hd, d = n % p.hd;
+  const bool rot = h < p.hq + p.hkv;
+  const bool odd = (lane & 1) != 0;
+  for (int j = 0; j < 32; ++j) {
+    const int m = m0 + j;
+    float y = __fmul_rn(v[j], alpha);
+    if (p.bias) y = __fadd_rn(y, bias);
+    y = bf2f(f2bf(y));
+    const float other = __shfl_xor_sync(0xffffffffu, y, 1);
+    if (m >= p.M || !col_ok) continue;
+    const int b = m / p.Mseq, s = m % p.Mseq;
+    uint16_t* dst;
+    float o = y;
+    if (rot) {
+      const uint16_t* rp = p.rope + long(s) * p.hd + (d & ~1);
+      const float c = bf2f(__ldg(rp)), sn = bf2f(__ldg(rp + 1));
+      const float x0 = odd ? other : y, x1 = odd ? y : other;
+      o = odd ? __fadd_rn(__fmul_rn(x0, sn), __fmul_rn(x1, c))
+              : __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, sn));
+      dst = h < p.hq ? p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d
+                     : p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d;
+    } else {
+      const int hv = h - p.hq - p.hkv;
+      dst = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + hv) * p.hd + d;
+    }
+    *dst = f2bf(o);
+  }
+}
+
+// GEGLU (normal orientation, BN = 256): gate columns 32c.., up columns
+// 128 + 32c.. of the same tile; output column tb * 128 + 32c ...
+__device__ __forceinline__ void epi_geglu_chunk(const GemmParams& p, const float (&g)[32],
+                                                const float (&u)[32], int m, int n_gate0,
+                                                int n_up0, int out_col0, float alpha) {
+  if (m >= p.M) return;
+  const float os = __ldg(p.out_scale);
+  float q[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float gv = scale_bias_bf16(g[j], alpha, p.bias, n_gate0 + j);
+    const float uv = scale_bias_bf16(u[j], alpha, p.bias, n_up0 + j);
+    q[j] = __fdiv_rn(gelu_tanh_mul(gv, uv), os);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + long(m) * p.ldo + out_col0);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    float a[8], b[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { a[j] = q[16 * k + j]; b[j] = q[16 * k + 8 + j]; }
+    const uint2 lo = pack8_e4m3(a), hi = pack8_e4m3(b);
+    dst[k] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+  }
+}
+
+// Run the epilogue of one tile.  load(c, v) fills v with accumulator chunk c
+// (32 columns); it is called warp-uniformly.
+template <bool SWAP, int BN, class Load>
+__device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int tb, int q, int lane,
+                                              float alpha, Load load) {
+  if (!SWAP && p.epi == EPI_GEGLU) {
+    const int m = ta * BM + 32 * q + lane;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float g[32], u[32];
+      load(c, g);
+      load(c + 4, u);
+      epi_geglu_chunk(p, g, u, m, tb * BN + 32 * c, tb * BN + 128 + 32 * c, tb * 128 + 32 * c,
+                      alpha);
+    }
+    return;
+  }
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    if (!SWAP) {
+      const int n0 = tb * BN + 32 * c;
+      if (n0 >= p.N) break;
+      load(c, v);
+      epi_rows_chunk(p, v, ta * BM + 32 * q + lane, n0, alpha);
+    } else {
+      const int m0 = tb * BN + 32 * c;
+      if (m0 >= p.M) break;
+      load(c, v);
+      epi_cols_chunk(p, v, ta * BM + 32 * q + lane, m0, alpha, lane);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel --
+
+template <bool SWAP, int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const GemmParams p) {
+  constexpr int B_BYTES = BN * BK;
+  constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * BN);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* last_flag = abort_flag + 1;
+  volatile int* epi_ok = abort_flag + 2;  // [4], one per epilogue warp
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        const int tile = u / p.splits, split = u % p.splits;
+        const int ta = tile % p.a_tiles, tb = tile / p.a_tiles;
+        const int kb0 = int(long(split) * p.k_blocks / p.splits);
+        const int kb1 = int(long(split + 1) * p.k_blocks / p.splits);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitNs, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES);
+          tma_load_2d(sA + stage * A_BYTES, &tmA, &full[stage], kb * BK, ta * BM);
+          tma_load_2d(sB + stage * B_BYTES, &tmB, &full[stage], kb * BK, tb * BN);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        record_timeout(p.status);
+        *abort_flag = 1;
+        // drain: wait (bounded) for the copies still in flight, newest first
+        int st = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < issued && i < STAGES; ++i) {
+          if (--st < 0) { st = STAGES - 1; ph ^= 1u; }
+          mbar_wait_bounded(&full[st], ph, kDrainNs, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      int stage = 0, local = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++local) {
+        const int split = u % p.splits;
+        const int kb0 = int(long(split) * p.k_blocks / p.splits);
+        const int kb1 = int(long(split + 1) * p.k_blocks / p.splits);
+        const int ab = local & 1;
+        const uint32_t aph = (local >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[ab], aph ^ 1u, kWaitNs, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dcol = tmem_base + uint32_t(ab * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, kWaitNs, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = sdesc_k_sw128(a_base + stage * A_BYTES);
+          const uint64_t bd = sdesc_k_sw128(b_base + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            umma_e4m3(dcol, ad + 2 * k, bd + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[ab]);
+      }
+      if (!ok) {
+        record_timeout(p.status);
+        *abort_flag = 1;
+        umma_commit(drain);  // completes when every MMA issued so far is done
+        mbar_wait_bounded(drain, 0, kDrainNs, nullptr);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue --
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
+    int local = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++local) {
+      const int tile = u / p.splits, split = u % p.splits;
+      const int ta = tile % p.a_tiles, tb = tile / p.a_tiles;
+      const int ab = local & 1;
+      const uint32_t aph = (local >> 1) & 1;
+      // All four epilogue warps agree on whether the accumulator arrived, so
+      // none of them can be left alone at a named barrier.
+      const bool got = __all_sync(0xffffffffu,
+                                  mbar_wait_bounded(&tfull[ab], aph, kWaitNs, abort_flag));
+      if (lane == 0) epi_ok[q] = got ? 1 : 0;
+      named_bar_sync(1, 128);
+      const bool all_ok = epi_ok[0] && epi_ok[1] && epi_ok[2] && epi_ok[3];
+      named_bar_sync(1, 128);
+      if (!all_ok) {
+        if (lane == 0) record_timeout(p.status);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + uint32_t(ab * BN) + (uint32_t(32 * q) << 16);
+      if (p.splits == 1) {
+        tile_epilogue<SWAP, BN>(p, ta, tb, q, lane, alpha,
+                                [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); });
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[ab]);
+      } else {
+        // spill this split's fp32 partial: row (lane of TMEM) major
+        const int row = 32 * q + lane;
+        float* part = p.partials + (long(tile) * p.splits + split) * (BM * BN) + long(row) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(tbase + 32 * c, v);
+          float4* d4 = reinterpret_cast<float4*>(part + 32 * c);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[ab]);
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 64) {
+          const unsigned old = atomicAdd(&p.counters[tile], 1u);
+          *last_flag = (old == unsigned(p.splits - 1)) ? 1 : 0;
+        }
+        named_bar_sync(1, 128);
+        if (*last_flag) {
+          __threadfence();
+          const float* base = p.partials + long(tile) * p.splits * (BM * BN) + long(row) * BN;
+          tile_epilogue<SWAP, BN>(p, ta, tb, q, lane, alpha, [&](int c, float (&v)[32]) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+            for (int s = 0; s < p.splits; ++s) {
+              const float4* src = reinterpret_cast<const float4*>(base + long(s) * (BM * BN) + 32 * c);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const float4 f = __ldcg(src + k);
+                v[4 * k] = __fadd_rn(v[4 * k], f.x);
+                v[4 * k + 1] = __fadd_rn(v[4 * k + 1], f.y);
+                v[4 * k + 2] = __fadd_rn(v[4 * k + 2], f.z);
+                v[4 * k + 3] = __fadd_rn(v[4 * k + 3], f.w);
+              }
+            }
+          });
+          if (threadIdx.x == 64) p.counters[tile] = 0u;
+        }
+        named_bar_sync(1, 128);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// -------------------------------------------------------------------- host --
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// Row-major [rows, K] e4m3 tensor, box = 128 bytes of K x box_rows rows,
+// 128-byte swizzle, out-of-bounds elements read as zero.
+int make_map(CUtensorMap* m, const void* ptr, long rows, int K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FRT_ECUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(K)};
+  const cuuint32_t box[2] = {cuuint32_t(BK), cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FRT_ECUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return FRT_OK;
+}
+
+struct Plan {
+  bool swap;
+  int bn, a_tiles, b_tiles, k_blocks, splits, units, grid;
+  size_t counters_bytes, ws_bytes;
+};
+
+Plan make_plan(int M, int N, int K, int epi) {
+  Plan pl{};
+  pl.k_blocks = (K + BK - 1) / BK;
+  if (epi == EPI_GEGLU) { pl.swap = false; pl.bn = 256; }
+  else if (M <= 128) { pl.swap = true; pl.bn = M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+  else { pl.swap = false; pl.bn = (N % 256 == 0) ? 256 : 128; }
+  const long a_rows = pl.swap ? N : M, b_rows = pl.swap ? M : N;
+  pl.a_tiles = int((a_rows + BM - 1) / BM);
+  pl.b_tiles = int((b_rows + pl.bn - 1) / pl.bn);
+  const int tiles = pl.a_tiles * pl.b_tiles;
+  const int sms = num_sms();
+  pl.splits = 1;
+  if (tiles * 2 <= sms) {
+    pl.splits = sms / tiles;
+    if (pl.splits > pl.k_blocks) pl.splits = pl.k_blocks;
+    if (pl.splits > 16) pl.splits = 16;
+    if (pl.splits < 1) pl.splits = 1;
+  }
+  pl.units = tiles * pl.splits;
+  pl.grid = pl.units < sms ? pl.units : sms;
+  if (pl.splits > 1) {
+    pl.counters_bytes = (size_t(tiles) * sizeof(unsigned) + 255) & ~size_t(255);
+    pl.ws_bytes = pl.counters_bytes + size_t(tiles) * pl.splits * BM * pl.bn * sizeof(float);
+  }
+  return pl;
+}
+
+template <bool SWAP, int BN, int STAGES>
+int launch_t(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+             cudaStream_t s) {
+  constexpr int smem = smem_bytes<BN, STAGES>();
+  static_assert(smem <= 232448, "shared memory budget");
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(gemm_kernel<SWAP, BN, STAGES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return fail(FRT_ECUDA, "cudaFuncSetAttribute(max dynamic smem %d)", smem);
+    attr_set[dev] = true;
+  }
+  gemm_kernel<SWAP, BN, STAGES><<<pl.grid, kThreads, smem, s>>>(ta, tb, p);
+  return check_launch("gemm_kernel");
+}
+
+int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void* workspace,
+             size_t workspace_bytes, cudaStream_t s) {
+  if (pl.ws_bytes > 0) {
+    FRT_REQUIRE(workspace, FRT_EINVAL, "this shape splits K: a workspace of %zu bytes is required",
+                pl.ws_bytes);
+    FRT_REQUIRE(workspace_bytes >= pl.ws_bytes, FRT_ERANGE,
+                "workspace of %zu bytes is smaller than the %zu this shape needs", workspace_bytes,
+                pl.ws_bytes);
+    FRT_REQUIRE(aligned(workspace, 256), FRT_EALIGN, "workspace must be 256-byte aligned");
+    p.counters = static_cast<unsigned*>(workspace);
+    p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + pl.counters_bytes);
+  }
+  p.a_tiles = pl.a_tiles; p.b_tiles = pl.b_tiles; p.k_blocks = pl.k_blocks;
+  p.splits = pl.splits; p.units = pl.units;
+  p.status = device_status_ptr();
+  CUtensorMap ta, tb;
+  int rc;
+  if (!pl.swap) {
+    if ((rc = make_map(&ta, x8, p.M, p.K, BM))) return rc;
+    if ((rc = make_map(&tb, w8, p.N, p.K, pl.bn))) return rc;
+  } else {
+    if ((rc = make_map(&ta, w8, p.N, p.K, BM))) return rc;
+    if ((rc = make_map(&tb, x8, p.M, p.K, pl.bn))) return rc;
+  }
+  if (!pl.swap && pl.bn == 256) return launch_t<false, 256, 4>(pl, ta, tb, p, s);
+  if (!pl.swap) return launch_t<false, 128, 6>(pl, ta, tb, p, s);
+  if (pl.bn == 32) return launch_t<true, 32, 8>(pl, ta, tb, p, s);
+  if (pl.bn == 64) return launch_t<true, 64, 8>(pl, ta, tb, p, s);
+  return launch_t<true, 128, 6>(pl, ta, tb, p, s);
+}
+
+int validate_common(int M, int N, int K, const void* x8, const void* w8, const float* act_scale,
+                    const float* w_scale) {
+  FRT_REQUIRE(M >= 0, FRT_ESHAPE, "M must be >= 0, got %d", M);
+  FRT_REQUIRE(N > 0 && N % 32 == 0, FRT_ESHAPE, "N must be a positive multiple of 32, got %d", N);
+  FRT_REQUIRE(K > 0 && K % 16 == 0, FRT_ESHAPE, "K must be a positive multiple of 16, got %d", K);
+  FRT_REQUIRE(x8 && w8 && act_scale && w_scale, FRT_EINVAL,
+              "x8, w8, act_scale and w_scale are required");
+  FRT_REQUIRE(aligned(x8, 16) && aligned(w8, 16), FRT_EALIGN, "x8 and w8 must be 16-byte aligned");
+  return FRT_OK;
+}
+
+}  // namespace
+}  // namespace frt
+
+extern "C" size_t frt_gemm_workspace_size(int M, int N, int K, int epilogue) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return frt::make_plan(M, N, K, epilogue == FRT_EPI_GEGLU_E4M3 ? frt::EPI_GEGLU : frt::EPI_BF16)
+      .ws_bytes;
+}
+
+extern "C" int frt_packed_fp8_gemm(int M, int N, int K, const frt_e4m3* x8, const frt_e4m3* w8,
+                                   const float* act_scale, const float* w_scale,
+                                   const frt_bf16* bias, int epilogue, void* out, long ldo,
+                                   const float* out_scale, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  using frt::aligned;
+  frt::clear_error();
+  int rc = frt::validate_common(M, N, K, x8, w8, act_scale, w_scale);
+  if (rc) return rc;
+  FRT_REQUIRE(epilogue == FRT_EPI_BF16 || epilogue == FRT_EPI_GEGLU_E4M3, FRT_EINVAL,
+              "unknown epilogue %d", epilogue);
+  FRT_REQUIRE(out, FRT_EINVAL, "out is required");
+  FRT_REQUIRE(aligned(out, 16), FRT_EALIGN, "out must be 16-byte aligned");
+  if (epilogue == FRT_EPI_BF16) {
+    FRT_REQUIRE(ldo >= N && ldo % 8 == 0, FRT_EALIGN, "ldo must be >= N and a multiple of 8");
+  } else {
+    FRT_REQUIRE(N % 256 == 0, FRT_ESHAPE, "the GEGLU epilogue needs N %% 256 == 0, got %d", N);
+    FRT_REQUIRE(out_scale, FRT_EINVAL, "the GEGLU epilogue needs out_scale");
+    FRT_REQUIRE(ldo >= N / 2 && ldo % 16 == 0, FRT_EALIGN,
+                "ldo must be >= N/2 and a multiple of 16 bytes");
+  }
+  if (M == 0) return FRT_OK;
+  const int epi = epilogue == FRT_EPI_BF16 ? frt::EPI_BF16 : frt::EPI_GEGLU;
+  frt::Plan pl = frt::make_plan(M, N, K, epi);
+  frt::GemmParams p{};
+  p.M = M; p.N = N; p.K = K;
+  p.act_scale = act_scale; p.w_scale = w_scale; p.bias = bias;
+  p.epi = epi; p.out = out; p.ldo = ldo; p.out_scale = out_scale;
+  p.Mseq = 1;
+  return frt::run_gemm(pl, p, x8, w8, workspace, workspace_bytes,
+                       static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int frt_packed_fp8_gemm_rope_kvcache(
+    int B, int M, int K, int hq, int hkv, int hd, int P, int T, const frt_e4m3* x8,
+    const frt_e4m3* w8, const float* act_scale, const float* w_scale, const frt_bf16* bias,
+    const frt_bf16* rope, frt_bf16* q_out, frt_bf16* k_cache, frt_bf16* v_cache, void* workspace,
+    size_t workspace_bytes, void* stream) {
+  using frt::aligned;
+  frt::clear_error();
+  FRT_REQUIRE(B >= 0 && M >= 0 && hq >= 0 && hkv >= 1, FRT_ESHAPE, "bad B/M/heads");
+  FRT_REQUIRE(hd >= 32 && hd % 32 == 0, FRT_ESHAPE,
+              "the fused epilogue needs hd %% 32 == 0, got %d", hd);
+  FRT_REQUIRE(P >= 0 && P + M <= T, FRT_ERANGE, "P + M = %d exceeds the cache capacity T = %d",
+              P + M, T);
+  const int N = (hq + 2 * hkv) * hd;
+  const long rows = long(B) * M;
+  FRT_REQUIRE(rows <= 0x7fffffffL, FRT_ESHAPE, "B*M too large");
+  int rc = frt::validate_common(int(rows), N, K, x8, w8, act_scale, w_scale);
+  if (rc) return rc;
+  FRT_REQUIRE(rope && k_cache && v_cache && (q_out || hq == 0), FRT_EINVAL,
+              "rope, q_out, k_cache and v_cache are required");
+  FRT_REQUIRE(aligned(rope, 16) && aligned(k_cache, 16) && aligned(v_cache, 16) &&
+                  (!q_out || aligned(q_out, 16)),
+              FRT_EALIGN, "rope, q_out and the caches must be 16-byte aligned");
+  if (rows == 0) return FRT_OK;
+  frt::Plan pl = frt::make_plan(int(rows), N, K, frt::EPI_ROPE);
+  frt::GemmParams p{};
+  p.M = int(rows); p.N = N; p.K = K;
+  p.act_scale = act_scale; p.w_scale = w_scale; p.bias = bias;
+  p.epi = frt::EPI_ROPE;
+  p.Mseq = M; p.hq = hq; p.hkv = hkv; p.hd = hd; p.P = P; p.T = T;
+  p.rope = rope; p.q_out = q_out; p.k_cache = k_cache; p.v_cache = v_cache;
+  return frt::run_gemm(pl, p, x8, w8, workspace, workspace_bytes,
+                       static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,302 @@
+// producer.cu -- a1 / a1': the single-pass producer of the chain's FP8 wire.
+//
+// AdaRMS form (flashrt-structures 0.2.0, impls/adarms_stack/fp8_chain.py,
+// `norm_project`: gated residual add + AdaRMS + static quantize, and the fp32
+// tail of `_make_run` that fixes the formula and the (scale, shift, gate)
+// chunk order) and the per-token-table LayerNorm form
+// (impls/modnorm_qkv_chain/fp8_ptok_table.py, module docstring and
+// `PerTokenModChainBlock.forward`: table add + chunk selection + no-affine
+// LayerNorm + modulation + static quantize, "the six-chunk materialization
+// never exists").
+//
+// Layout: a group of G threads (G a multiple of 32) owns one row; each thread
+// holds VPT chunks of 8 bf16 (16-byte loads) in registers, so every input
+// byte is read once and every output byte written once (HBM-bound: 7*D bytes
+// per row in both forms).  G == 32 packs 4 rows per 128-thread block; larger
+// G uses one row per block and a shared-memory cross-warp reduction.
+// Arithmetic is fp32 with explicitly rounded operations (no contraction into
+// FMA), IEEE division and square root, so the only difference from a
+// sequential evaluation is the order of the row sums.
+
+#include "frt_common.cuh"
+
+namespace frt {
+namespace {
+
+struct ProducerArgs {
+  int rows, D, C, G;
+  float eps;
+  uint16_t* res;
+  const uint16_t* delta;
+  const uint16_t* gate;
+  long gate_stride;
+  const uint16_t* weight;
+  const uint16_t* style;
+  long style_stride;
+  const uint16_t* x;
+  const uint16_t* temb;
+  int chunks;
+  const float* table;
+  int shift_idx, scale_idx;
+  const float* act_scale;
+  uint8_t* x8;
+  uint16_t* gate_out;
+  float* amax;
+};
+
+__device__ __forceinline__ uint4 ldg16(const uint16_t* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Sum over the G threads of a row.  With G > 32 the block holds one row.
+__device__ __forceinline__ float row_sum(float v, int G, float* red) {
+  v = warp_sum(v);
+  if (G == 32) return v;
+  const int w = threadIdx.x >> 5, nw = G >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.0f;
+  for (int i = 0; i < nw; ++i) s = __fadd_rn(s, red[i]);
+  return s;
+}
+
+template <int VPT>
+__global__ void __launch_bounds__(512) adarms_kernel(ProducerArgs a) {
+  __shared__ float red[16];
+  const int G = a.G;
+  const int rpb = blockDim.x / G;
+  const int t = threadIdx.x % G;
+  const long r = long(blockIdx.x) * rpb + threadIdx.x / G;
+  if (G == 32 && r >= a.rows) return;          // warp-uniform, no block sync
+  const bool ok = r < a.rows;                  // G > 32: whole block uniform
+  const int D = a.D, C = a.C;
+
+  float hr[VPT][8];
+  float ss = 0.0f;
+  if (ok) {
+    uint16_t* rr = a.res + r * D;
+    const uint16_t* dd = a.delta + r * D;
+    const uint16_t* gg = a.gate + r * a.gate_stride;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = t + i * G;
+      if (c < C) {
+        float rv[8], dv[8], gv[8];
+        unpack8(*reinterpret_cast<const uint4*>(rr + 8 * c), rv);
+        unpack8(ldg16(dd + 8 * c), dv);
+        unpack8(ldg16(gg + 8 * c), gv);
+        float h[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) h[j] = __fadd_rn(rv[j], __fmul_rn(gv[j], dv[j]));
+        const uint4 hb = pack8_bf16(h);
+        *reinterpret_cast<uint4*>(rr + 8 * c) = hb;
+        unpack8(hb, hr[i]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss = __fadd_rn(ss, __fmul_rn(hr[i][j], hr[i][j]));
+      }
+    }
+  }
+  ss = row_sum(ss, G, red);
+  if (!ok) return;
+  const float ms = __fdiv_rn(ss, float(D));
+  const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
+  const float as = __ldg(a.act_scale);
+  const uint16_t* st = a.style + r * a.style_stride;
+  float mx = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int c = t + i * G;
+    if (c < C) {
+      float wv[8], sc[8], sh[8];
+      if (a.weight) unpack8(ldg16(a.weight + 8 * c), wv);
+      else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) wv[j] = 1.0f;
+      }
+      unpack8(ldg16(st + 8 * c), sc);
+      unpack8(ldg16(st + D + 8 * c), sh);
+      float q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float v = __fmul_rn(hr[i][j], inv);
+        v = __fmul_rn(v, wv[j]);
+        v = __fmul_rn(v, __fadd_rn(1.0f, sc[j]));
+        const float y = __fadd_rn(v, sh[j]);
+        mx = fmaxf(mx, fabsf(y));
+        q[j] = __fdiv_rn(y, as);
+      }
+      *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
+      if (a.gate_out)
+        *reinterpret_cast<uint4*>(a.gate_out + r * D + 8 * c) = ldg16(st + 2 * D + 8 * c);
+    }
+  }
+  if (a.amax) {
+    mx = warp_max(mx);
+    if ((threadIdx.x & 31) == 0) atomic_max_nonneg(a.amax, mx);
+  }
+}
+
+template <int VPT>
+__global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
+  __shared__ float red[16];
+  const int G = a.G;
+  const int rpb = blockDim.x / G;
+  const int t = threadIdx.x % G;
+  const long r = long(blockIdx.x) * rpb + threadIdx.x / G;
+  if (G == 32 && r >= a.rows) return;
+  const bool ok = r < a.rows;
+  const int D = a.D, C = a.C;
+
+  float xv[VPT][8];
+  float sum = 0.0f;
+  if (ok) {
+    const uint16_t* xr = a.x + r * D;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = t + i * G;
+      if (c < C) {
+        unpack8(ldg16(xr + 8 * c), xv[i]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sum = __fadd_rn(sum, xv[i][j]);
+      }
+    }
+  }
+  sum = row_sum(sum, G, red);
+  const float mu = __fdiv_rn(sum, float(D));
+  float sq = 0.0f;
+  if (ok) {
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = t + i * G;
+      if (c < C) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float d = __fsub_rn(xv[i][j], mu);
+          sq = __fadd_rn(sq, __fmul_rn(d, d));
+        }
+      }
+    }
+  }
+  sq = row_sum(sq, G, red);
+  if (!ok) return;
+  const float var = __fdiv_rn(sq, float(D));
+  const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
+  const float as = __ldg(a.act_scale);
+  const uint16_t* tr = a.temb + r * long(a.chunks) * D;
+  const uint16_t* tsh = tr + long(a.shift_idx) * D;
+  const uint16_t* tsc = tr + long(a.scale_idx) * D;
+  const float* bsh = a.table + long(a.shift_idx) * D;
+  const float* bsc = a.table + long(a.scale_idx) * D;
+  float mx = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int c = t + i * G;
+    if (c < C) {
+      float esh[8], esc[8];
+      unpack8(ldg16(tsh + 8 * c), esh);
+      unpack8(ldg16(tsc + 8 * c), esc);
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(bsh + 8 * c));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(bsh + 8 * c + 4));
+      const float4 c0 = __ldg(reinterpret_cast<const float4*>(bsc + 8 * c));
+      const float4 c1 = __ldg(reinterpret_cast<const float4*>(bsc + 8 * c + 4));
+      const float tsh8[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      const float tsc8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      float q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float shift = __fadd_rn(tsh8[j], esh[j]);
+        const float scale = __fadd_rn(tsc8[j], esc[j]);
+        float v = __fmul_rn(__fsub_rn(xv[i][j], mu), inv);
+        v = __fmul_rn(v, __fadd_rn(1.0f, scale));
+        const float y = __fadd_rn(v, shift);
+        mx = fmaxf(mx, fabsf(y));
+        q[j] = __fdiv_rn(y, as);
+      }
+      *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
+    }
+  }
+  if (a.amax) {
+    mx = warp_max(mx);
+    if ((threadIdx.x & 31) == 0) atomic_max_nonneg(a.amax, mx);
+  }
+}
+
+}  // namespace
+}  // namespace frt
+
+using frt::ProducerArgs;
+
+extern "C" int frt_ada_norm_quant_fp8(
+    int mode, int rows, int D, float eps, frt_bf16* res, const frt_bf16* delta,
+    const frt_bf16* prev_gate, long gate_row_stride, const frt_bf16* weight,
+    const frt_bf16* style, long style_row_stride, const frt_bf16* x,
+    const frt_bf16* temb, int chunks, const float* table, int shift_idx,
+    int scale_idx, const float* act_scale, frt_e4m3* x8_out, frt_bf16* gate_out,
+    float* amax_out, void* stream) {
+  using frt::aligned;
+  frt::clear_error();
+  FRT_REQUIRE(mode == FRT_NORM_ADARMS || mode == FRT_NORM_LAYERNORM_TABLE,
+              FRT_EINVAL, "mode %d is not FRT_NORM_ADARMS or FRT_NORM_LAYERNORM_TABLE", mode);
+  FRT_REQUIRE(rows >= 0, FRT_ESHAPE, "rows must be >= 0, got %d", rows);
+  FRT_REQUIRE(D >= 8 && D <= 16384 && D % 8 == 0, FRT_ESHAPE,
+              "D must be a multiple of 8 in [8, 16384], got %d", D);
+  FRT_REQUIRE(eps >= 0.0f, FRT_EINVAL, "eps must be >= 0");
+  FRT_REQUIRE(act_scale && x8_out, FRT_EINVAL, "act_scale and x8_out are required");
+  FRT_REQUIRE(aligned(x8_out, 8), FRT_EALIGN, "x8_out must be 8-byte aligned");
+  FRT_REQUIRE(aligned(act_scale, 4), FRT_EALIGN, "act_scale must be 4-byte aligned");
+  if (mode == FRT_NORM_ADARMS) {
+    FRT_REQUIRE(res && delta && prev_gate && style, FRT_EINVAL,
+                "AdaRMS needs res, delta, prev_gate and style");
+    FRT_REQUIRE(aligned(res, 16) && aligned(delta, 16) && aligned(prev_gate, 16) &&
+                    aligned(style, 16) && (!weight || aligned(weight, 16)) &&
+                    (!gate_out || aligned(gate_out, 16)),
+                FRT_EALIGN, "bf16 tensors must be 16-byte aligned");
+    FRT_REQUIRE(gate_row_stride >= 0 && gate_row_stride % 8 == 0 &&
+                    style_row_stride >= 0 && style_row_stride % 8 == 0,
+                FRT_EALIGN, "row strides must be non-negative multiples of 8");
+    FRT_REQUIRE(gate_row_stride == 0 || gate_row_stride >= D, FRT_ESHAPE,
+                "gate_row_stride must be 0 or >= D");
+    FRT_REQUIRE(style_row_stride == 0 || style_row_stride >= 3L * D, FRT_ESHAPE,
+                "style_row_stride must be 0 or >= 3*D");
+  } else {
+    FRT_REQUIRE(x && temb && table, FRT_EINVAL, "LayerNorm-table needs x, temb and table");
+    FRT_REQUIRE(chunks >= 1 && shift_idx >= 0 && shift_idx < chunks && scale_idx >= 0 &&
+                    scale_idx < chunks,
+                FRT_EINVAL, "chunk indices (%d, %d) outside [0, %d)", shift_idx, scale_idx, chunks);
+    FRT_REQUIRE(aligned(x, 16) && aligned(temb, 16) && aligned(table, 16), FRT_EALIGN,
+                "x, temb and table must be 16-byte aligned");
+  }
+  FRT_REQUIRE(!amax_out || aligned(amax_out, 4), FRT_EALIGN, "amax_out must be 4-byte aligned");
+  if (rows == 0) return FRT_OK;
+
+  ProducerArgs a{};
+  a.rows = rows; a.D = D; a.C = D / 8; a.eps = eps;
+  a.res = res; a.delta = delta; a.gate = prev_gate; a.gate_stride = gate_row_stride;
+  a.weight = weight; a.style = style; a.style_stride = style_row_stride;
+  a.x = x; a.temb = temb; a.chunks = chunks; a.table = table;
+  a.shift_idx = shift_idx; a.scale_idx = scale_idx;
+  a.act_scale = act_scale; a.x8 = x8_out; a.gate_out = gate_out; a.amax = amax_out;
+  int vpt;
+  if (a.C <= 128) { a.G = 32; vpt = (a.C + 31) / 32; }
+  else { vpt = 4; a.G = ((a.C + 127) / 128) * 32; }
+  const int rpb = a.G == 32 ? 4 : 1;
+  const dim3 block(a.G * rpb), grid((rows + rpb - 1) / rpb);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (mode == FRT_NORM_ADARMS) {
+    switch (vpt) {
+      case 1: frt::adarms_kernel<1><<<grid, block, 0, s>>>(a); break;
+      case 2: frt::adarms_kernel<2><<<grid, block, 0, s>>>(a); break;
+      case 3: frt::adarms_kernel<3><<<grid, block, 0, s>>>(a); break;
+      default: frt::adarms_kernel<4><<<grid, block, 0, s>>>(a); break;
+    }
+  } else {
+    switch (vpt) {
+      case 1: frt::ln_table_kernel<1><<<grid, block, 0, s>>>(a); break;
+      case 2: frt::ln_table_kernel<2><<<grid, block, 0, s>>>(a); break;
+      case 3: frt::ln_table_kernel<3><<<grid, block, 0, s>>>(a); break;
+      default: frt::ln_table_kernel<4><<<grid, block, 0, s>>>(a); break;
+    }
+  }
+  return frt::check_launch("frt_ada_norm_quant_fp8");
+}

@@ -1,0 +1,317 @@
+/*
+ * frt.h -- C ABI of libfrt, the sm_100a (B200) fused static-FP8
+ * attention-input chain.
+ *
+ * The chain (flashrt-structures 0.2.0, impls/adarms_stack/fp8_chain.py,
+ * module docstring and `_make_run`; impls/modnorm_qkv_chain/fp8_ptok_table.py,
+ * `PerTokenModChainBlock.forward`):
+ *   1. producer: gated residual add + adaptive RMS or LayerNorm with
+ *      shift/scale(/gate) modulation + static-scale e4m3 quantize, one pass;
+ *   2. one FP8 GEMM over sibling weights packed into one [sum N_i, K] matrix
+ *      with one joint per-tensor scale (impls/qkv_pack/fp8_static.py,
+ *      module docstring and `_pack_weights`), plus bias;
+ *   3. split + adjacent-pair RoPE + KV-cache write behind a copied prefix.
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers unless marked "host".  The caller
+ *     owns all memory; the library allocates nothing.  Tensors are dense,
+ *     row-major, with the shapes given.  bf16 tensors are passed as
+ *     frt_bf16 (the 16-bit pattern), e4m3fn tensors as frt_e4m3 (the code).
+ *   - Scales (act_scale, w_scale, out_scale) are device fp32 [1] tensors,
+ *     never host floats, so calls can be captured into CUDA graphs.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work
+ *     is enqueued asynchronously; nothing synchronises with the host.
+ *   - Arguments are validated on the host before any launch.  A rejected
+ *     call launches nothing and returns a negative FRT_E* code; the reason
+ *     is available from frt_last_error() on the calling thread.  FRT_ECUDA
+ *     reports a CUDA error seen at launch.
+ *   - Device-side waits (mbarrier pipelines) are bounded in time.  A wait
+ *     that runs out records FRT_ETIMEOUT in the library's device status
+ *     word, makes the kernel drain and return, and frt_device_status()
+ *     reports it later.
+ */
+#ifndef FRT_H_
+#define FRT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t frt_bf16; /* bfloat16 bit pattern */
+typedef uint8_t frt_e4m3;  /* float8 e4m3fn code   */
+
+enum {
+  FRT_OK = 0,
+  FRT_EINVAL = -1,   /* null pointer, bad enum, bad scalar                 */
+  FRT_ESHAPE = -2,   /* dimension outside what the kernel supports         */
+  FRT_EALIGN = -3,   /* pointer or stride not aligned as required          */
+  FRT_ERANGE = -4,   /* P + M > T, workspace too small, row capacity       */
+  FRT_ECUDA = -5,    /* CUDA reported an error at launch                   */
+  FRT_ETIMEOUT = -6  /* a bounded device-side wait ran out                 */
+};
+
+/* Reason for the last failing call on this thread ("" if none). */
+const char* frt_last_error(void);
+
+/* ABI version of this header (major * 100 + minor). */
+int frt_version(void);
+
+/* Read (and with reset != 0, clear) the device status word of the current
+ * device.  Synchronises `stream` first.  Returns FRT_OK, FRT_ETIMEOUT (some
+ * bounded wait ran out since the last reset) or FRT_ECUDA. */
+int frt_device_status(int reset, void* stream);
+
+/* ----------------------------------------------------------------------- */
+/* a1 / a1'  Producer.                                                      */
+/* ----------------------------------------------------------------------- */
+enum { FRT_NORM_ADARMS = 0, FRT_NORM_LAYERNORM_TABLE = 1 };
+
+/*
+ * frt_ada_norm_quant_fp8 -- one pass over `rows` rows of width D.
+ *
+ * mode FRT_NORM_ADARMS (fp8_chain.py, `norm_project` -> the norm kernel's
+ * call, and the fp32 tail of `_make_run`, which fixes the formula):
+ *   h = res + prev_gate * delta;  res <- bf16(h)            (in place)
+ *   y = bf16(h) / sqrt(mean(bf16(h)^2) + eps) * w * (1 + scale) + shift
+ *   x8 = e4m3(clamp(y / act_scale, +-448));  gate_out = gate
+ *   res, delta: [rows, D].  prev_gate: [1 or rows, D], row stride
+ *   gate_row_stride elements (0 = one row broadcast).  weight: [D] or NULL
+ *   (= ones).  style: [1 or rows, 3D] = (scale, shift, gate) chunks, row
+ *   stride style_row_stride (0 = broadcast).  gate_out: [rows, D] or NULL.
+ *   x, temb, table, chunks, shift_idx, scale_idx are ignored.
+ *
+ * mode FRT_NORM_LAYERNORM_TABLE (fp8_ptok_table.py, module docstring and
+ * `PerTokenModChainBlock.forward`: table add + chunk selection + no-affine
+ * LayerNorm + modulation + static quantize):
+ *   shift = table[shift_idx] + temb[r, shift_idx];  scale likewise
+ *   y = (x - mean(x)) / sqrt(var(x) + eps) * (1 + scale) + shift  (biased var)
+ *   x: [rows, D]; temb: [rows, chunks, D] bf16; table: [chunks, D] fp32.
+ *   res, delta, prev_gate, weight, style, gate_out are ignored.
+ *
+ * act_scale: device fp32 [1].  x8_out: [rows, D] e4m3.  amax_out: NULL or a
+ * device fp32 [1] the caller zeroed; the kernel raises it to max |y| (the
+ * static calibration of fp8_chain.py `bind_adarms_fp8_chain`).
+ * Requires 8 <= D <= 16384, D % 8 == 0, 16-byte aligned bf16 pointers and
+ * row strides that are multiples of 8, x8_out 8-byte aligned.  rows == 0 is
+ * a no-op.  All arithmetic fp32; divisions and square roots IEEE-rounded.
+ */
+int frt_ada_norm_quant_fp8(int mode, int rows, int D, float eps,
+                           frt_bf16* res, const frt_bf16* delta,
+                           const frt_bf16* prev_gate, long gate_row_stride,
+                           const frt_bf16* weight, const frt_bf16* style,
+                           long style_row_stride, const frt_bf16* x,
+                           const frt_bf16* temb, int chunks,
+                           const float* table, int shift_idx, int scale_idx,
+                           const float* act_scale, frt_e4m3* x8_out,
+                           frt_bf16* gate_out, float* amax_out, void* stream);
+
+/* ----------------------------------------------------------------------- */
+/* a0  Joint per-tensor weight pack (bind time).                            */
+/* ----------------------------------------------------------------------- */
+enum {
+  FRT_PACK_CONCAT = 0,     /* rows in sibling order (torch.cat along N)    */
+  FRT_PACK_QK_INTERLEAVE = 1, /* siblings (q, k, v): in each q and k head,
+                                 row i -> 2i, row hd/2+i -> 2i+1; v as is   */
+  FRT_PACK_GATE_UP_BLOCKS = 2 /* siblings (gate, up), equal n, n % 128 == 0:
+                                 128-row gate block then the matching up
+                                 block, repeated (for the fused GEGLU)      */
+};
+
+/*
+ * frt_pack_weights_fp8 (qkv_pack/fp8_static.py `_pack_weights`;
+ * fp8_chain.py `_quantize` with `_interleave_rows`):
+ *   w_scale = max(amax(|w_all|) / 448, 1e-8);  w8 = e4m3(clamp(w / w_scale))
+ * w: HOST array of n_siblings DEVICE pointers, sibling i is [n_rows[i], K]
+ * bf16 (n_rows is a HOST array).  bias: NULL or a HOST array of device
+ * pointers, entries NULL for siblings without bias (zeros are packed).
+ * w8_out: [N, K] e4m3, N = sum n_rows.  w_scale_out: device fp32 [1].
+ * bias_out: [N] bf16 or NULL.  layout: FRT_PACK_*; hd is the head size for
+ * FRT_PACK_QK_INTERLEAVE.  1 <= n_siblings <= 4, K % 16 == 0.
+ * Bit-exact: true fp32 division, round to nearest even.
+ */
+int frt_pack_weights_fp8(int n_siblings, const frt_bf16* const* w,
+                         const int* n_rows, int K, const frt_bf16* const* bias,
+                         int layout, int hd, frt_e4m3* w8_out,
+                         float* w_scale_out, frt_bf16* bias_out, void* stream);
+
+/* ----------------------------------------------------------------------- */
+/* a2 (+ a5)  Packed FP8 GEMM on tcgen05 tensor cores.                      */
+/* ----------------------------------------------------------------------- */
+enum { FRT_EPI_BF16 = 0, FRT_EPI_GEGLU_E4M3 = 1 };
+
+/*
+ * Bytes of workspace frt_packed_fp8_gemm / _rope_kvcache need for this
+ * shape (0 if the chosen schedule does not split K).  The workspace must be
+ * zero-filled once before its first use; every completed call leaves its
+ * counters at zero again.  Calls that share a workspace must not overlap.
+ */
+size_t frt_gemm_workspace_size(int M, int N, int K, int epilogue);
+
+/*
+ * frt_packed_fp8_gemm (qkv_pack/fp8_static.py `PackedLinear._run`;
+ * fp8_chain.py `norm_project` / `down_project`):
+ *   acc[m, n] = sum_k x8[m, k] * w8[n, k]            (fp32 accumulate)
+ *   FRT_EPI_BF16:  out[m, n] = bf16(acc * (act_scale * w_scale) + bias[n])
+ *                  out: [M, ldo] bf16, ldo >= N.
+ *   FRT_EPI_GEGLU_E4M3 (fp8_chain.py `down_project`, the merged GEGLU +
+ *   requant kernel): w8 packed with FRT_PACK_GATE_UP_BLOCKS; with
+ *   g, u = bf16(acc * alpha + bias) of matching gate/up columns,
+ *                  out[m, j] = e4m3(gelu_tanh(g) * u / out_scale)
+ *                  out: [M, ldo] e4m3, ldo >= N / 2; N % 256 == 0.
+ * x8: [M, K] e4m3; w8: [N, K] e4m3; bias: [N] bf16 or NULL.
+ * Requires K % 16 == 0, N % 32 == 0, 16-byte aligned x8/w8/out, ldo % 16 == 0
+ * (bytes of a row).  M == 0 is a no-op.  workspace: see
+ * frt_gemm_workspace_size (may be NULL when that is 0).
+ */
+int frt_packed_fp8_gemm(int M, int N, int K, const frt_e4m3* x8,
+                        const frt_e4m3* w8, const float* act_scale,
+                        const float* w_scale, const frt_bf16* bias,
+                        int epilogue, void* out, long ldo,
+                        const float* out_scale, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
+ * frt_packed_fp8_gemm_rope_kvcache -- the packed q/k/v GEMM with the split +
+ * RoPE + KV write fused into its epilogue (qkv_pack/fp8_static.py joint
+ * slots: q and k are one contiguous run consumed together; attention_core
+ * `alias_suffix`: the producer writes the suffix in place).  Same result,
+ * bit for bit, as frt_packed_fp8_gemm (bf16) followed by
+ * frt_split_rope_kvcache on the bf16 output.  N = (hq + 2*hkv) * hd; rows
+ * are b * M + s for b < B; see frt_split_rope_kvcache for the outputs.
+ * hd % 32 == 0.  The prefix is not copied here (frt_prefix_copy_kv).
+ */
+int frt_packed_fp8_gemm_rope_kvcache(
+    int B, int M, int K, int hq, int hkv, int hd, int P, int T,
+    const frt_e4m3* x8, const frt_e4m3* w8, const float* act_scale,
+    const float* w_scale, const frt_bf16* bias, const frt_bf16* rope,
+    frt_bf16* q_out, frt_bf16* k_cache, frt_bf16* v_cache, void* workspace,
+    size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------------------- */
+/* a3 / a4  RoPE table, split + RoPE + KV write, prefix copy.               */
+/* ----------------------------------------------------------------------- */
+
+/*
+ * frt_build_rope_table (fp8_chain.py `_build_rope`): for s < M, i < hd/2,
+ *   rope[s, 2i] = bf16(cos((P + s) * theta^(-2i/hd))), rope[s, 2i+1] = sin
+ * evaluated in fp64 and rounded once to bf16.  rope_out: [M, hd] bf16.
+ */
+int frt_build_rope_table(int M, int hd, int P, double theta,
+                         frt_bf16* rope_out, void* stream);
+
+/*
+ * frt_split_rope_kvcache (fp8_chain.py `_make_run`, the split kernel call;
+ * buffers as in `_alloc`): qkv [B*M, (hq + 2*hkv)*hd] bf16, row b*M + s.
+ * For q and k heads every adjacent pair (x0, x1) with c = rope[s, 2i],
+ * sn = rope[s, 2i+1] becomes (x0*c - x1*sn, x0*sn + x1*c) (fp32, rounded to
+ * bf16).  q_out: [B, M, hq, hd]; k_cache, v_cache: [B, T, hkv, hd], written
+ * at rows P + s (v copied).  If prefix_k is non-NULL the same launch also
+ * copies the prefix (see frt_prefix_copy_kv).  Requires P + M <= T,
+ * hd % 8 == 0, 16-byte aligned pointers.
+ */
+int frt_split_rope_kvcache(int B, int M, int hq, int hkv, int hd, int P,
+                           int T, const frt_bf16* qkv, const frt_bf16* rope,
+                           frt_bf16* q_out, frt_bf16* k_cache,
+                           frt_bf16* v_cache, const frt_bf16* prefix_k,
+                           const frt_bf16* prefix_v, int prefix_T_src,
+                           int prefix_interleave, void* stream);
+
+/*
+ * frt_prefix_copy_kv (fp8_chain.py `_make_run`, the `ad:prefix` range):
+ * prefix_k, prefix_v: host-cache layout [B, hkv, T_src, hd] bf16 (device
+ * memory).  Rows p < P go to k_cache / v_cache [B, T, hkv, hd].  With
+ * interleave != 0 the key's head dimension is gathered through
+ * kperm[2i] = i, kperm[2i+1] = hd/2 + i (rotate-half -> adjacent pairs);
+ * v is copied as is.  Bit-exact copy.  P <= T_src, P <= T, hd % 8 == 0.
+ */
+int frt_prefix_copy_kv(int B, int hkv, int hd, int P, int T, int T_src,
+                       const frt_bf16* prefix_k, const frt_bf16* prefix_v,
+                       int interleave, frt_bf16* k_cache, frt_bf16* v_cache,
+                       void* stream);
+
+/* ----------------------------------------------------------------------- */
+/* a5  GEGLU + static requant (standalone form).                            */
+/* ----------------------------------------------------------------------- */
+
+/*
+ * frt_geglu_quant_fp8 (fp8_chain.py `down_project`; tanh-GELU required by
+ * `bind_adarms_fp8_chain`): gu [M, 2H] bf16 (gate in columns [0, H), up in
+ * [H, 2H)), row stride ld_gu elements;
+ *   hid8[m, j] = e4m3(gelu_tanh(g) * u / out_scale),
+ *   gelu_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
+ * hid8: [M, H].  amax_out: NULL or zeroed device fp32 [1] raised to
+ * max |gelu_tanh(g) * u| (calibration).  H % 8 == 0.
+ */
+int frt_geglu_quant_fp8(int M, int H, const frt_bf16* gu, long ld_gu,
+                        const float* out_scale, frt_e4m3* hid8,
+                        float* amax_out, void* stream);
+
+/* ----------------------------------------------------------------------- */
+/* The attention-input chain layer: producer -> packed GEMM (+ RoPE + KV).  */
+/* ----------------------------------------------------------------------- */
+enum {
+  FRT_CHAIN_FUSED_ROPE = 0, /* GEMM epilogue does split + RoPE + KV write */
+  FRT_CHAIN_UNFUSED = 1     /* GEMM -> qkv (bf16) -> split kernel          */
+};
+
+typedef struct frt_chain_desc {
+  int B, M, D;            /* rows = B * M, model width D = K of the GEMM   */
+  int hq, hkv, hd;        /* heads; N = (hq + 2*hkv) * hd                  */
+  int P, T;               /* prefix rows already in the cache; capacity    */
+  float eps;
+  int norm_mode;          /* FRT_NORM_*                                    */
+  int flags;              /* FRT_CHAIN_*                                   */
+  /* producer, FRT_NORM_ADARMS */
+  frt_bf16* res; const frt_bf16* delta; const frt_bf16* prev_gate;
+  long gate_row_stride; const frt_bf16* norm_weight; const frt_bf16* style;
+  long style_row_stride; frt_bf16* gate_out;
+  /* producer, FRT_NORM_LAYERNORM_TABLE */
+  const frt_bf16* x; const frt_bf16* temb; int chunks; const float* table;
+  int shift_idx, scale_idx;
+  const float* act_scale; /* device [1] */
+  frt_e4m3* x8;           /* [B*M, D] caller-owned staging of the wire     */
+  /* packed projection */
+  const frt_e4m3* w8; const float* w_scale; const frt_bf16* bias;
+  /* RoPE + cache */
+  const frt_bf16* rope;   /* [M, hd] */
+  frt_bf16* q_out; frt_bf16* k_cache; frt_bf16* v_cache;
+  /* optional prefix copy (NULL prefix_k = none) */
+  const frt_bf16* prefix_k; const frt_bf16* prefix_v; int prefix_T_src;
+  int prefix_interleave;
+  frt_bf16* qkv;          /* [B*M, N], needed only with FRT_CHAIN_UNFUSED  */
+  void* workspace; size_t workspace_bytes;
+} frt_chain_desc;
+
+/* Workspace bytes frt_chain_layer needs for this descriptor. */
+size_t frt_chain_workspace_size(const frt_chain_desc* d);
+
+/*
+ * frt_chain_layer (fp8_chain.py `_make_run`, one layer's attention half:
+ * norm_project(slot 2l, "qkv") then the split kernel; fp8_ptok_table.py:
+ * producer then the Q/K/V wire projections): launches the producer, then
+ * the packed GEMM with the fused split + RoPE + KV epilogue (or, with
+ * FRT_CHAIN_UNFUSED, the GEMM into d->qkv and the split kernel), plus the
+ * prefix copy when d->prefix_k is set.  All launches on `stream`.
+ */
+int frt_chain_layer(const frt_chain_desc* d, void* stream);
+
+/* ----------------------------------------------------------------------- */
+/* Self-test of the bounded device wait.                                    */
+/* ----------------------------------------------------------------------- */
+
+/*
+ * Launches one CTA that waits on an mbarrier nobody arrives on, bounded by
+ * `timeout_us` microseconds, then returns.  Synchronises `stream` and
+ * returns FRT_ETIMEOUT when the bound ran out (the expected outcome), so a
+ * test can check that bounded waits end and report.  Clears the status.
+ */
+int frt_selftest_bounded_wait(int timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FRT_H_ */

@@ -1,0 +1,60 @@
+"""Comparison helpers for the GPU-vs-oracle parity tests.
+
+Tolerances are the chain's stated bar:
+  * indices, copies, caches: bit-exact;
+  * e4m3 activation codes: >= 99.99 % identical, every other code exactly one
+    step away (adjacent magnitude with the same sign, or +-0 against the
+    smallest subnormal, or +0 against -0);
+  * GEMM / RoPE outputs: max |err| <= 2e-2 * rms(ref), fp32 accumulation.
+"""
+
+import numpy as np
+
+from fp8_transformer_block_b200.synth import bf16_value
+
+CODE_MATCH = 0.9999
+RMS_TOL = 2e-2
+
+
+def e4m3_step_distance(a, b):
+    a = np.asarray(a, np.uint8).astype(np.int32)
+    b = np.asarray(b, np.uint8).astype(np.int32)
+    ma, mb = a & 0x7F, b & 0x7F
+    sa, sb = a >> 7, b >> 7
+    same = a == b
+    adjacent = (sa == sb) & (np.abs(ma - mb) == 1)
+    zero_cross = ((ma == 0) & (mb <= 1)) | ((mb == 0) & (ma <= 1))
+    dist = np.where(same, 0, np.where(adjacent | zero_cross, 1, 2))
+    return dist
+
+
+def assert_codes(got, ref, match=CODE_MATCH, what="codes"):
+    d = e4m3_step_distance(got, ref)
+    frac = float((d == 0).mean()) if d.size else 1.0
+    bad = int((d > 1).sum())
+    assert bad == 0, f"{what}: {bad} codes differ by more than one step"
+    assert frac >= match, f"{what}: only {frac:.6f} identical (< {match})"
+    return frac
+
+
+def rel_rms_err(got_bf16, ref_bf16):
+    g = bf16_value(got_bf16).astype(np.float64)
+    r = bf16_value(ref_bf16).astype(np.float64)
+    rms = np.sqrt((r ** 2).mean()) if r.size else 1.0
+    return float(np.abs(g - r).max() / rms) if r.size else 0.0
+
+
+def assert_rms(got_bf16, ref_bf16, tol=RMS_TOL, what="values"):
+    e = rel_rms_err(got_bf16, ref_bf16)
+    assert e <= tol, f"{what}: max|err| = {e:.3e} * rms(ref) > {tol}"
+    return e
+
+
+def bf16_ulps(got_bf16, ref_bf16):
+    """Distance in bf16 units of the last place (same-sign values)."""
+    g = np.asarray(got_bf16, np.uint16).astype(np.int32)
+    r = np.asarray(ref_bf16, np.uint16).astype(np.int32)
+    # map sign-magnitude to a monotone integer line
+    g = np.where(g & 0x8000, -(g & 0x7FFF), g)
+    r = np.where(r & 0x8000, -(r & 0x7FFF), r)
+    return np.abs(g - r)

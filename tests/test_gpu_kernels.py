@@ -1,0 +1,377 @@
+"""GPU parity of every kernel against the CPU oracle, through the C ABI.
+
+Each test draws seeded inputs, runs the oracle and the CUDA path on the same
+bytes and applies the stated bar (see tests/parity.py).  Output buffers and
+caches are pre-filled with a NaN sentinel so stray writes are caught.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from fp8_transformer_block_b200 import synth
+from fp8_transformer_block_b200.synth import bf16_bits, normal_bf16
+from parity import assert_codes, assert_rms, bf16_ulps
+from chain_cases import SENTINEL, calibrate_adarms, calibrate_dit
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rt():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from fp8_transformer_block_b200 import build
+    build.build()
+    from fp8_transformer_block_b200 import frt, runtime
+    return frt, runtime, torch
+
+
+def _sync(torch):
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------ bounded wait --
+
+def test_bounded_wait_reports_timeout(rt):
+    frt, runtime, torch = rt
+    rc = frt.frt_selftest_bounded_wait(20000)
+    assert rc == frt.FRT_ETIMEOUT
+    assert frt.frt_device_status(True) == frt.FRT_OK
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0            # the context is still usable
+
+
+# ---------------------------------------------------------------- producer --
+
+def _gpu_adarms(rt, inp, act_scale, eps=1e-6, weight=None, amax=False):
+    frt, runtime, torch = rt
+    res = runtime.bf16_dev(inp["res"])
+    delta = runtime.bf16_dev(inp["delta"])
+    gate = runtime.bf16_dev(inp["prev_gate"])
+    style = runtime.bf16_dev(inp["style"])
+    rows, D = inp["res"].shape
+    x8 = runtime.empty_u8(rows, D)
+    gate_out = runtime.empty_bf16(rows, D)
+    sc = runtime.scale_dev(act_scale)
+    am = torch.zeros(1, dtype=torch.float32, device="cuda") if amax else None
+    w = None if weight is None else runtime.bf16_dev(weight)
+    frt.frt_ada_norm_quant_fp8(
+        frt.FRT_NORM_ADARMS, rows, D, eps, res, delta, gate,
+        0 if inp["prev_gate"].shape[0] == 1 else D, w, style,
+        0 if inp["style"].shape[0] == 1 else 3 * D, None, None, 0, None, 0, 0,
+        sc, x8, gate_out, am)
+    _sync(torch)
+    return {"res": runtime.bf16_host(res), "x8": runtime.u8_host(x8),
+            "gate_out": runtime.bf16_host(gate_out),
+            "amax": None if am is None else float(am.item())}
+
+
+@pytest.mark.parametrize("rows,D,outliers,per_row", [
+    (64, 512, False, False),      # tiny AdaRMS layer
+    (50, 2048, True, False),      # VLA action expert, 1 % outlier rows x20
+    (37, 776, False, True),       # ragged: D = 97 chunks, per-row style/gate
+    (5, 16384, False, False),     # widest D
+    (3, 8, False, False),         # narrowest D
+    (1024, 2048, True, True),     # gate/up MLP producer site
+])
+def test_producer_adarms_parity(rt, rows, D, outliers, per_row):
+    inp = synth.adarms_inputs(rows, D, 4242 + D, outliers=outliers)
+    if per_row:
+        rng = np.random.default_rng(D)
+        inp["prev_gate"] = normal_bf16(rng, (rows, D))
+        inp["style"] = normal_bf16(rng, (rows, 3 * D), 0.5)
+    ref1 = oracle.ada_rms_norm_quant(inp["res"], inp["delta"],
+                                     inp["prev_gate"], inp["style"], 1.0)
+    a = ref1["amax"] / 448.0
+    ref = oracle.ada_rms_norm_quant(inp["res"], inp["delta"],
+                                    inp["prev_gate"], inp["style"], a)
+    got = _gpu_adarms(rt, inp, a, amax=True)
+    assert np.array_equal(got["res"], ref["res"]), "residual update"
+    assert np.array_equal(got["gate_out"], ref["gate_out"]), "gate_out"
+    assert_codes(got["x8"], ref["x8"], what="x8")
+    assert abs(got["amax"] - ref1["amax"]) <= 1e-5 * ref1["amax"]
+
+
+@pytest.mark.parametrize("rows,D,chunks,sidx,cidx", [
+    (256, 3072, 6, 0, 1),         # video-DiT attention site
+    (33, 1000, 6, 3, 4),          # ragged, FFN-site chunks
+    (2, 16384, 6, 0, 1),
+])
+def test_producer_layernorm_parity(rt, rows, D, chunks, sidx, cidx):
+    frt, runtime, torch = rt
+    inp = synth.dit_inputs(rows, D, 777 + D, chunks)
+    a = oracle.ada_layer_norm_quant_table(inp["x"], inp["temb"], inp["table"],
+                                          sidx, cidx, 1.0)["amax"] / 448.0
+    ref = oracle.ada_layer_norm_quant_table(inp["x"], inp["temb"],
+                                            inp["table"], sidx, cidx, a)
+    x8 = runtime.empty_u8(rows, D)
+    am = torch.zeros(1, dtype=torch.float32, device="cuda")
+    frt.frt_ada_norm_quant_fp8(
+        frt.FRT_NORM_LAYERNORM_TABLE, rows, D, 1e-6, None, None, None, 0,
+        None, None, 0, runtime.bf16_dev(inp["x"]),
+        runtime.bf16_dev(inp["temb"]), chunks, runtime.f32_dev(inp["table"]),
+        sidx, cidx, runtime.scale_dev(a), x8, None, am)
+    _sync(torch)
+    assert_codes(runtime.u8_host(x8), ref["x8"], what="x8")
+    assert abs(float(am.item()) - a * 448.0) <= 1e-5 * a * 448.0
+
+
+def test_producer_layernorm_full_dit(rt):
+    frt, runtime, torch = rt
+    w = synth.WORKLOADS["video_dit"]
+    inp = synth.dit_inputs(w.rows, w.D, w.seed)
+    a = calibrate_dit(w, inp["table"])
+    ref = oracle.ada_layer_norm_quant_table(inp["x"], inp["temb"],
+                                            inp["table"], 0, 1, a)
+    x8 = runtime.empty_u8(w.rows, w.D)
+    frt.frt_ada_norm_quant_fp8(
+        frt.FRT_NORM_LAYERNORM_TABLE, w.rows, w.D, w.eps, None, None, None,
+        0, None, None, 0, runtime.bf16_dev(inp["x"]),
+        runtime.bf16_dev(inp["temb"]), 6, runtime.f32_dev(inp["table"]), 0,
+        1, runtime.scale_dev(a), x8, None, None)
+    _sync(torch)
+    assert_codes(runtime.u8_host(x8), ref["x8"], what="video-DiT x8")
+
+
+# -------------------------------------------------------------------- pack --
+
+@pytest.mark.parametrize("case", ["qk_interleave", "bias_concat",
+                                  "gate_up_blocks"])
+def test_pack_bit_exact(rt, case):
+    frt, runtime, torch = rt
+    if case == "qk_interleave":
+        ws, bs = synth.qkv_weights(8, 1, 64, 512, 11)
+        layout, hd = frt.FRT_PACK_QK_INTERLEAVE, 64
+    elif case == "bias_concat":
+        ws, bs = synth.qkv_weights(4, 4, 128, 1024, 12, bias=True)
+        bs[1] = None
+        layout, hd = frt.FRT_PACK_CONCAT, 0
+    else:
+        mw = synth.mlp_weights(512, 2048, 13)
+        ws, bs = [mw["gate"], mw["up"]], None
+        layout, hd = frt.FRT_PACK_GATE_UP_BLOCKS, 0
+    ref = oracle.pack_weights_fp8(ws, bs, layout=layout, hd=hd)
+    pk = runtime.pack(ws, bs, layout=layout, hd=hd)
+    _sync(torch)
+    assert float(pk.w_scale.item()) == ref["w_scale"]
+    assert np.array_equal(runtime.u8_host(pk.w8), ref["w8"])
+    if pk.bias is not None:
+        assert np.array_equal(runtime.bf16_host(pk.bias), ref["bias"])
+
+
+# -------------------------------------------------------------------- GEMM --
+
+def _x8_codes(rows, K, seed):
+    inp = synth.adarms_inputs(rows, K, seed)
+    return oracle.ada_rms_norm_quant(inp["res"], inp["delta"],
+                                     inp["prev_gate"], inp["style"],
+                                     0.02)["x8"]
+
+
+GEMM_CASES = [
+    # M, N, K, bias   (M <= 128 runs the swapped, split-K schedule)
+    (1, 640, 512, False),
+    (16, 640, 512, False),
+    (50, 2560, 2048, False),
+    (64, 640, 512, True),
+    (100, 672, 528, True),         # ragged N tile, K tail (528 = 4*128 + 16)
+    (128, 2560, 2048, False),
+    (129, 640, 512, False),        # first normal-orientation size
+    (300, 672, 528, True),         # ragged everywhere, BN = 128
+    (1000, 2560, 2048, True),      # BN = 256, persistent
+    (256, 9216, 3072, True),       # video-DiT projection width
+]
+
+
+@pytest.mark.parametrize("M,N,K,bias", GEMM_CASES)
+def test_gemm_parity(rt, M, N, K, bias):
+    frt, runtime, torch = rt
+    rng = np.random.default_rng(M * 7 + N)
+    x8 = _x8_codes(M, K, 100 + M)
+    w = normal_bf16(rng, (N, K), 0.02)
+    b = normal_bf16(rng, (N,), 0.5) if bias else None
+    pk_ref = oracle.pack_weights_fp8([w], [b])
+    a = 0.0173
+    ref = oracle.fp8_gemm(x8, pk_ref["w8"], a, pk_ref["w_scale"],
+                          pk_ref["bias"] if bias else None)
+    w8 = runtime.u8_dev(pk_ref["w8"])
+    ws = runtime.scale_dev(pk_ref["w_scale"])
+    bd = runtime.bf16_dev(pk_ref["bias"]) if bias else None
+    out = torch.full((M, N), float("nan"), dtype=torch.bfloat16,
+                     device="cuda")
+    wsb = frt.frt_gemm_workspace_size(M, N, K)
+    wsp = runtime.workspace(wsb)
+    for _ in range(2):   # a second call reuses the zeroed split counters
+        frt.frt_packed_fp8_gemm(M, N, K, runtime.u8_dev(x8), w8,
+                                runtime.scale_dev(a), ws, bd, frt.FRT_EPI_BF16,
+                                out, N, None, wsp, wsb)
+    _sync(torch)
+    got = runtime.bf16_host(out)
+    assert_rms(got, ref, what=f"GEMM {M}x{N}x{K}")
+    assert np.percentile(bf16_ulps(got, ref), 99.9) <= 1
+    if wsp is not None:
+        assert not wsp[:256].any().item(), "split counters left non-zero"
+
+
+def test_gemm_zero_input_gives_bias(rt):
+    frt, runtime, torch = rt
+    for M in (7, 200):
+        N, K = 640, 512
+        rng = np.random.default_rng(M)
+        b = normal_bf16(rng, (N,), 1.0)
+        w8 = runtime.u8_dev(rng.integers(0, 0x7E, (N, K), dtype=np.uint8))
+        out = runtime.empty_bf16(M, N)
+        wsb = frt.frt_gemm_workspace_size(M, N, K)
+        frt.frt_packed_fp8_gemm(M, N, K, runtime.empty_u8(M, K).zero_(), w8,
+                                runtime.scale_dev(0.5), runtime.scale_dev(0.01),
+                                runtime.bf16_dev(b), frt.FRT_EPI_BF16, out, N,
+                                None, runtime.workspace(wsb), wsb)
+        _sync(torch)
+        assert np.array_equal(runtime.bf16_host(out), np.tile(b, (M, 1)))
+
+
+# ------------------------------------------------- rope table / split / KV --
+
+@pytest.mark.parametrize("M,hd,P", [(50, 256, 816), (4096, 128, 0), (64, 64, 0)])
+def test_rope_table(rt, M, hd, P):
+    frt, runtime, torch = rt
+    t = runtime.empty_bf16(M, hd)
+    frt.frt_build_rope_table(M, hd, P, 10000.0, t)
+    _sync(torch)
+    ref = oracle.rope_table(M, hd, P)
+    got = runtime.bf16_host(t)
+    d = bf16_ulps(got, ref)
+    assert d.max() <= 1 and (d == 0).mean() >= 0.9999
+
+
+def _caches(runtime, torch, B, T, hkv, hd):
+    kc = torch.full((B, T, hkv, hd), 0, dtype=torch.int16, device="cuda")
+    kc.fill_(np.int16(np.uint16(SENTINEL).view(np.int16)).item())
+    vc = kc.clone()
+    return kc.view(torch.bfloat16), vc.view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("B,M,hq,hkv,hd,P,T,bias,prefix", [
+    (1, 64, 8, 1, 64, 0, 64, False, False),      # tiny AdaRMS
+    (1, 50, 8, 1, 256, 816, 1024, False, True),  # VLA action expert
+    (2, 200, 4, 4, 128, 0, 256, True, False),    # DiT-shaped, normal tiles
+    (1, 1, 8, 1, 64, 816, 817, False, True),     # one token
+])
+def test_split_rope_fused_and_unfused(rt, B, M, hq, hkv, hd, P, T, bias,
+                                      prefix):
+    frt, runtime, torch = rt
+    K = 512
+    N = (hq + 2 * hkv) * hd
+    rows = B * M
+    x8 = _x8_codes(rows, K, 500 + M)
+    ws_, bs_ = synth.qkv_weights(hq, hkv, hd, K, 900 + M, bias=bias)
+    pk_ref = oracle.pack_weights_fp8(ws_, bs_, layout=1, hd=hd)
+    pk = runtime.pack(ws_, bs_, layout=frt.FRT_PACK_QK_INTERLEAVE, hd=hd)
+    a = 0.02
+    sc = runtime.scale_dev(a)
+    x8d = runtime.u8_dev(x8)
+    rope = runtime.empty_bf16(M, hd)
+    frt.frt_build_rope_table(M, hd, P, 10000.0, rope)
+    pkh = pvh = None
+    if prefix:
+        pkh, pvh = synth.prefix_cache(B, hkv, P + 8, hd, 31)
+    wsb = frt.frt_gemm_workspace_size(rows, N, K)
+    wsp = runtime.workspace(wsb)
+    # unfused: GEMM -> qkv -> split (+ prefix in the same launch)
+    qkv = runtime.empty_bf16(rows, N)
+    frt.frt_packed_fp8_gemm(rows, N, K, x8d, pk.w8, sc, pk.w_scale, pk.bias,
+                            frt.FRT_EPI_BF16, qkv, N, None, wsp, wsb)
+    q1 = runtime.empty_bf16(B, M, hq, hd)
+    k1, v1 = _caches(runtime, torch, B, T, hkv, hd)
+    pkd = runtime.bf16_dev(pkh) if prefix else None
+    pvd = runtime.bf16_dev(pvh) if prefix else None
+    frt.frt_split_rope_kvcache(B, M, hq, hkv, hd, P, T, qkv, rope, q1, k1, v1,
+                               pkd, pvd, P + 8 if prefix else 0, 1)
+    # fused: GEMM epilogue does split + RoPE + KV; prefix copied separately
+    q2 = runtime.empty_bf16(B, M, hq, hd)
+    k2, v2 = _caches(runtime, torch, B, T, hkv, hd)
+    if prefix:
+        frt.frt_prefix_copy_kv(B, hkv, hd, P, T, P + 8, pkd, pvd, 1, k2, v2)
+    frt.frt_packed_fp8_gemm_rope_kvcache(B, M, K, hq, hkv, hd, P, T, x8d,
+                                         pk.w8, sc, pk.w_scale, pk.bias, rope,
+                                         q2, k2, v2, wsp, wsb)
+    _sync(torch)
+    h = runtime.bf16_host
+    assert np.array_equal(h(q1), h(q2)), "fused q differs from unfused"
+    assert np.array_equal(h(k1), h(k2)), "fused k cache differs"
+    assert np.array_equal(h(v1), h(v2)), "fused v cache differs"
+    # unfused split vs the oracle split on the GPU's own qkv: bit-exact
+    kc0 = np.full((B, T, hkv, hd), SENTINEL, np.uint16)
+    if prefix:
+        kc0a, vc0a = oracle.prefix_copy(pkh, pvh, P, kc0, kc0, True)
+    else:
+        kc0a, vc0a = kc0, kc0
+    qo, ko, vo = oracle.split_rope_kvcache(h(qkv), oracle.rope_table(M, hd, P),
+                                           B, M, hq, hkv, hd, P, kc0a, vc0a)
+    assert np.array_equal(h(q1), qo)
+    assert np.array_equal(h(k1), ko)
+    assert np.array_equal(h(v1), vo)
+    # GEMM vs oracle GEMM on the same codes, then end to end
+    ref_qkv = oracle.fp8_gemm(x8, pk_ref["w8"], a, pk_ref["w_scale"],
+                              pk_ref["bias"] if bias else None)
+    assert_rms(h(qkv), ref_qkv, what="qkv")
+    qr, kr, vr = oracle.split_rope_kvcache(ref_qkv, oracle.rope_table(M, hd, P),
+                                           B, M, hq, hkv, hd, P, kc0a, vc0a)
+    assert_rms(h(q2), qr, what="q_out")
+    sl = slice(P, P + M)
+    assert_rms(h(k2)[:, sl], kr[:, sl], what="k rows")
+    assert np.array_equal(h(k2)[:, P + M:], kr[:, P + M:])   # untouched
+    assert np.array_equal(h(k2)[:, :P], kr[:, :P])           # prefix
+
+
+# ------------------------------------------------------------------- GEGLU --
+
+def test_geglu_standalone_parity(rt):
+    frt, runtime, torch = rt
+    rng = np.random.default_rng(5)
+    M, H = 96, 1024
+    gu = bf16_bits(np.concatenate([rng.standard_normal((M, H)) * 2,
+                                   rng.standard_normal((M, H))], 1))
+    _, amax = oracle.geglu_quant(gu, 1.0)
+    a = amax / 448.0
+    ref, _ = oracle.geglu_quant(gu, a)
+    hid = runtime.empty_u8(M, H)
+    am = torch.zeros(1, dtype=torch.float32, device="cuda")
+    frt.frt_geglu_quant_fp8(M, H, runtime.bf16_dev(gu), 2 * H,
+                            runtime.scale_dev(a), hid, am)
+    _sync(torch)
+    assert_codes(runtime.u8_host(hid), ref, what="hid8")
+    assert abs(float(am.item()) - amax) <= 1e-5 * amax
+
+
+@pytest.mark.parametrize("M", [64, 300])
+def test_geglu_fused_epilogue(rt, M):
+    frt, runtime, torch = rt
+    D, H = 512, 1024
+    mw = synth.mlp_weights(D, H, 21)
+    x8 = runtime.u8_dev(_x8_codes(M, D, 77))
+    sc = runtime.scale_dev(0.02)
+    cat = runtime.pack([mw["gate"], mw["up"]])
+    blk = runtime.pack([mw["gate"], mw["up"]],
+                       layout=frt.FRT_PACK_GATE_UP_BLOCKS)
+    gu = runtime.empty_bf16(M, 2 * H)
+    wsb = frt.frt_gemm_workspace_size(M, 2 * H, D)
+    wsp = runtime.workspace(wsb)
+    frt.frt_packed_fp8_gemm(M, 2 * H, D, x8, cat.w8, sc, cat.w_scale, None,
+                            frt.FRT_EPI_BF16, gu, 2 * H, None, wsp, wsb)
+    out_scale = runtime.scale_dev(0.01)
+    h1 = runtime.empty_u8(M, H)
+    frt.frt_geglu_quant_fp8(M, H, gu, 2 * H, out_scale, h1)
+    h2 = runtime.empty_u8(M, H)
+    wsb2 = frt.frt_gemm_workspace_size(M, 2 * H, D, frt.FRT_EPI_GEGLU_E4M3)
+    frt.frt_packed_fp8_gemm(M, 2 * H, D, x8, blk.w8, sc, blk.w_scale, None,
+                            frt.FRT_EPI_GEGLU_E4M3, h2, H, out_scale,
+                            runtime.workspace(wsb2), wsb2)
+    _sync(torch)
+    # the fused codes equal the unfused GPU path's; that path equals the
+    # oracle's GEGLU on the same gu
+    assert_codes(runtime.u8_host(h2), runtime.u8_host(h1), match=0.9999,
+                 what="fused vs unfused")
+    ref, _ = oracle.geglu_quant(runtime.bf16_host(gu), 0.01)
+    assert_codes(runtime.u8_host(h1), ref, what="unfused vs oracle")
