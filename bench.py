@@ -1,0 +1,880 @@
+"""Benchmark of the fused static-FP8 attention-input chain on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl reference]
+
+One step = one pass of the chain over one batch of the workload, all inputs
+resident in HBM: for the default workload (the VLA action-expert layer: 50
+tokens behind an 816-token prefix, D=2048, 8 q heads + 1 kv head of 256,
+packed N=2560) that is the prefix copy into the layer's caches, the AdaRMS
+producer and the packed FP8 q/k/v GEMM with the split + RoPE + KV write in
+its epilogue: the three launches frt_chain_layer makes.  Other workloads
+(--config): tiny_adarms, video_dit, gateup_mlp, adarms_stack18[:M].
+
+Timing: W untimed warm-up steps, then K timed steps.  Before every timed step
+the L2 is flushed (a 256 MB write) and the GPU is held by a short spin so the
+host has enqueued the whole step before its first event; each kernel is
+bracketed by CUDA events on the launching stream.  The JSON line reports the
+device time; `e2e` repeats the step through frt_chain_layer with pinned host
+inputs copied in and the outputs copied back inside the timed region.
+With N > 1 (torchrun) every rank runs an independent replica on its own
+batch (no data-path collective); value = all ranks' tokens / max rank time.
+
+--impl reference times the CPU oracle (the reference arm: plain C, OpenMP
+over rows) on the host cores on the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("chain tokens/s & µs/layer; GEMM % FP8 tensor peak, "
+          "producer % HBM GB/s")
+DEFAULT_CONFIG = "vla_action_expert"
+FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_PER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+# DRAM bytes per launch of the dominant kernel from the committed ncu capture
+# (profiles/), keyed by workload; valid only while the kernel's source hash
+# matches the one the counters were taken on.
+NCU_TRAFFIC = {}
+
+
+def _src_hash():
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "producer.cu", "rope.cu", "frt_sm100.cuh",
+              "frt_common.cuh"):
+        with open(os.path.join(ROOT, "fp8_transformer_block_b200", "csrc", f),
+                  "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "measured")
+    except (OSError, KeyError, ValueError):
+        return (FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback")
+
+
+# ---------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while the
+    timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", f"frt_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu_id], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- runners ----
+
+class Kern:
+    """One kind of launch in a step, with its algorithmic work per launch."""
+
+    def __init__(self, name, bound, algo_bytes=0.0, flops=0.0, per_step=1):
+        self.name, self.bound = name, bound
+        self.algo_bytes, self.flops = float(algo_bytes), float(flops)
+        self.per_step = per_step
+
+
+class ChainRunner:
+    """Attention-input chain layers: prefix copy, producer (AdaRMS or
+    per-token-table LayerNorm), packed q/k/v GEMM with the fused split +
+    RoPE + KV epilogue.  With layers > 1 the residual is carried and layer
+    l+1 takes layer l's q_out (viewed [rows, D]) as delta and its gate_out
+    as gate; layer 0 sees delta = gate = 0."""
+
+    def __init__(self, w, torch, frt, rt, synth):
+        self.w, self.torch, self.frt, self.rt = w, torch, frt, rt
+        self.dit = w.kind == "dit"
+        self.L = w.layers
+        B, M, D = w.B, w.M, w.D
+        self.rows = rows = B * M
+        N = w.N
+        self.layers = []
+        for l in range(self.L):
+            if self.L > 1:
+                li = synth.stack_layer_inputs(w, l)
+                ws, bs, style = li["w"], li["b"], li["style"]
+                pkh, pvh = li["prefix_k"], li["prefix_v"]
+            else:
+                ws, bs = synth.qkv_weights(w.hq, w.hkv, w.hd, D, w.seed,
+                                           bias=w.bias)
+                style, pkh, pvh = None, None, None
+                if w.P > 0:
+                    pkh, pvh = synth.prefix_cache(B, w.hkv, max(1024, w.P),
+                                                  w.hd, w.seed)
+            layout = (frt.FRT_PACK_CONCAT if self.dit
+                      else frt.FRT_PACK_QK_INTERLEAVE)
+            pk = rt.pack(ws, bs if w.bias else None, layout=layout, hd=w.hd)
+            self.layers.append({
+                "pk": pk,
+                "kc": torch.zeros(B, w.T, w.hkv, w.hd, dtype=torch.bfloat16,
+                                  device="cuda"),
+                "vc": torch.zeros(B, w.T, w.hkv, w.hd, dtype=torch.bfloat16,
+                                  device="cuda"),
+                "style": None if style is None else rt.bf16_dev(style),
+                "pk_host": pkh, "pv_host": pvh,
+                "pkd": None if pkh is None else rt.bf16_dev(pkh),
+                "pvd": None if pvh is None else rt.bf16_dev(pvh),
+                "T_src": 0 if pkh is None else int(pkh.shape[2])})
+        self.rope = rt.empty_bf16(M, w.hd)
+        frt.frt_build_rope_table(M, w.hd, w.P, w.theta, self.rope)
+        if self.dit:
+            inp = synth.dit_inputs(rows, D, w.seed)
+            self.x = rt.bf16_dev(inp["x"])
+            self.temb = rt.bf16_dev(inp["temb"])
+            self.table = rt.f32_dev(inp["table"])
+            self.host_in = {"x": inp["x"], "temb": inp["temb"]}
+        else:
+            inp = synth.adarms_inputs(rows, D, w.seed, outliers=w.outliers)
+            self.res0 = rt.bf16_dev(inp["res"])
+            self.res = self.res0.clone()
+            self.delta = rt.bf16_dev(inp["delta"])
+            self.gate = rt.bf16_dev(inp["prev_gate"])
+            self.style1 = rt.bf16_dev(inp["style"])
+            self.zero = torch.zeros(rows, D, dtype=torch.bfloat16, device="cuda")
+            self.gate_out = [rt.empty_bf16(rows, D) for _ in range(2)]
+            self.host_in = {k: inp[k] for k in
+                            ("res", "delta", "prev_gate", "style")}
+        self.x8 = rt.empty_u8(rows, D)
+        self.q = [rt.empty_bf16(B, M, w.hq, w.hd) for _ in range(2)]
+        self.ws_bytes = frt.frt_gemm_workspace_size(rows, N, D)
+        self.ws = rt.workspace(self.ws_bytes)
+        self.calibrate(synth)
+        ks = []
+        if self.layers[0]["pkd"] is not None:
+            ks.append(Kern("prefix_copy", "hbm",
+                           4.0 * B * w.P * w.hkv * w.hd * 2, per_step=self.L))
+        prod = (rows * D * (2 + 2 * 2 + 1) if self.dit
+                else rows * D * (4 + 2 + 1 + 2) + 4 * D * 2)
+        ks.append(Kern("producer", "hbm", prod, per_step=self.L))
+        gbytes = (N * D + rows * D + M * w.hd * 2 + rows * N * 2
+                  + (N * 2 if w.bias else 0))
+        gflops = 2.0 * rows * N * D
+        ks.append(Kern("gemm_rope_kv",
+                       "tensor" if gflops / gbytes > 560 else "hbm",
+                       gbytes, gflops, per_step=self.L))
+        self.kerns = ks
+        self.tokens = rows
+        self.launches = sum(k.per_step for k in ks)
+
+    # ----------------------------------------------------------------------
+    def _inputs(self, l):
+        """(delta, gate, gate_stride, style) of layer l."""
+        if self.L == 1:
+            return self.delta, self.gate, 0, self.style1
+        if l == 0:
+            return self.zero, self.zero, 0, self.layers[0]["style"]
+        return (self.q[(l - 1) % 2], self.gate_out[(l - 1) % 2], self.w.D,
+                self.layers[l]["style"])
+
+    def _producer(self, l, scale, amax=None):
+        frt, w = self.frt, self.w
+        if self.dit:
+            frt.frt_ada_norm_quant_fp8(
+                frt.FRT_NORM_LAYERNORM_TABLE, self.rows, w.D, w.eps, None,
+                None, None, 0, None, None, 0, self.x, self.temb, 6,
+                self.table, 0, 1, scale, self.x8, None, amax)
+        else:
+            d, g, gs, st = self._inputs(l)
+            frt.frt_ada_norm_quant_fp8(
+                frt.FRT_NORM_ADARMS, self.rows, w.D, w.eps, self.res, d, g,
+                gs, None, st, 0, None, None, 0, None, 0, 0, scale, self.x8,
+                self.gate_out[l % 2], amax)
+
+    def _gemm(self, l, scale):
+        w, lay = self.w, self.layers[l]
+        self.frt.frt_packed_fp8_gemm_rope_kvcache(
+            w.B, w.M, w.D, w.hq, w.hkv, w.hd, w.P, w.T, self.x8,
+            lay["pk"].w8, scale, lay["pk"].w_scale, lay["pk"].bias,
+            self.rope, self.q[l % 2], lay["kc"], lay["vc"], self.ws,
+            self.ws_bytes)
+
+    def _prefix(self, l):
+        w, lay = self.w, self.layers[l]
+        if lay["pkd"] is not None:
+            self.frt.frt_prefix_copy_kv(w.B, w.hkv, w.hd, w.P, w.T,
+                                        lay["T_src"], lay["pkd"], lay["pvd"],
+                                        1, lay["kc"], lay["vc"])
+
+    def calibrate(self, synth):
+        """Static activation scale per layer = amax / 448 of the producer's
+        output on the calibration batch (seed + 500), from the GPU
+        producer's amax output; stacked layers are calibrated in order, each
+        on the output of the already-calibrated layers before it."""
+        torch, frt, rt, w = self.torch, self.frt, self.rt, self.w
+        am = torch.zeros(1, dtype=torch.float32, device="cuda")
+        one = rt.scale_dev(1.0)
+        self.act = []
+        if self.dit:
+            cal = synth.dit_inputs(w.cal_rows, w.D, w.seed + synth.CAL_OFFSET,
+                                   with_table=False)
+            x8 = rt.empty_u8(w.cal_rows, w.D)
+            frt.frt_ada_norm_quant_fp8(
+                frt.FRT_NORM_LAYERNORM_TABLE, w.cal_rows, w.D, w.eps, None,
+                None, None, 0, None, None, 0, rt.bf16_dev(cal["x"]),
+                rt.bf16_dev(cal["temb"]), 6, self.table, 0, 1, one, x8, None,
+                am)
+            self.act = [rt.scale_dev(float(am.item()) / 448.0)]
+            return
+        if self.L == 1:
+            cal = synth.adarms_inputs(w.cal_rows, w.D,
+                                      w.seed + synth.CAL_OFFSET,
+                                      outliers=w.outliers)
+            x8 = rt.empty_u8(w.cal_rows, w.D)
+            frt.frt_ada_norm_quant_fp8(
+                frt.FRT_NORM_ADARMS, w.cal_rows, w.D, w.eps,
+                rt.bf16_dev(cal["res"]), rt.bf16_dev(cal["delta"]),
+                rt.bf16_dev(cal["prev_gate"]), 0, None,
+                rt.bf16_dev(cal["style"]), 0, None, None, 0, None, 0, 0, one,
+                x8, None, am)
+            self.act = [rt.scale_dev(float(am.item()) / 448.0)]
+            return
+        cal = synth.adarms_inputs(self.rows, w.D, w.seed + synth.CAL_OFFSET)
+        self.res.copy_(rt.bf16_dev(cal["res"]))
+        snap = torch.empty_like(self.res)
+        for l in range(self.L):
+            snap.copy_(self.res)
+            am.zero_()
+            self._producer(l, one, am)
+            a = rt.scale_dev(max(float(am.item()), 1e-30) / 448.0)
+            self.act.append(a)
+            self.res.copy_(snap)
+            self._producer(l, a)
+            self._gemm(l, a)
+        self.res.copy_(self.res0)
+
+    # ----------------------------------------------------------------------
+    def reset(self):
+        """Restore the state a step mutates (the residual); untimed."""
+        if not self.dit:
+            self.res.copy_(self.res0)
+
+    def step(self, ev=None):
+        """Issue one step; ev[k][l] = (start, end) events per kernel kind k
+        and layer l, or None."""
+        for l in range(self.L):
+            k = 0
+            if self.layers[l]["pkd"] is not None:
+                if ev: ev[k][l][0].record()
+                self._prefix(l)
+                if ev: ev[k][l][1].record()
+                k += 1
+            if ev: ev[k][l][0].record()
+            self._producer(l, self.act[l if not self.dit else 0])
+            if ev: ev[k][l][1].record()
+            k += 1
+            if ev: ev[k][l][0].record()
+            self._gemm(l, self.act[l if not self.dit else 0])
+            if ev: ev[k][l][1].record()
+
+    # ---------------------------------------------------------------- e2e --
+    def e2e_setup(self):
+        torch = self.torch
+        self.pin_in = {k: torch.from_numpy(v.view(np.int16)).pin_memory()
+                       for k, v in self.host_in.items()}
+        self.dev_in = ({"x": self.x, "temb": self.temb} if self.dit else
+                       {"res": self.res, "delta": self.delta,
+                        "prev_gate": self.gate, "style": self.style1})
+        for l, lay in enumerate(self.layers):
+            if lay["pk_host"] is not None:
+                self.pin_in[f"pk{l}"] = torch.from_numpy(
+                    lay["pk_host"].view(np.int16)).pin_memory()
+                self.pin_in[f"pv{l}"] = torch.from_numpy(
+                    lay["pv_host"].view(np.int16)).pin_memory()
+                self.dev_in[f"pk{l}"] = lay["pkd"]
+                self.dev_in[f"pv{l}"] = lay["pvd"]
+        w = self.w
+        outs = {"q": self.q[(self.L - 1) % 2]}
+        for l, lay in enumerate(self.layers):
+            outs[f"k{l}"] = lay["kc"][:, w.P:w.P + w.M]
+            outs[f"v{l}"] = lay["vc"][:, w.P:w.P + w.M]
+        if not self.dit:
+            outs["res"] = self.res
+            outs["gate"] = self.gate_out[(self.L - 1) % 2]
+        self.dev_out = outs
+        self.pin_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory()
+                        for k, v in outs.items()}
+        self.h2d_bytes = sum(t.numel() * t.element_size()
+                             for t in self.pin_in.values())
+        self.d2h_bytes = sum(t.numel() * t.element_size()
+                             for t in self.pin_out.values())
+        self.descs = []
+        frt, rt = self.frt, self.rt
+        for l, lay in enumerate(self.layers):
+            d, g, gs, st = self._inputs(l) if not self.dit else (None,) * 4
+            self.descs.append(rt.chain_desc(
+                B=w.B, M=w.M, D=w.D, hq=w.hq, hkv=w.hkv, hd=w.hd, P=w.P,
+                T=w.T, eps=w.eps,
+                norm_mode=(frt.FRT_NORM_LAYERNORM_TABLE if self.dit
+                           else frt.FRT_NORM_ADARMS),
+                flags=frt.FRT_CHAIN_FUSED_ROPE,
+                res=None if self.dit else self.res, delta=d, prev_gate=g,
+                gate_row_stride=gs or 0, style=st, style_row_stride=0,
+                gate_out=None if self.dit else self.gate_out[l % 2],
+                x=self.x if self.dit else None,
+                temb=self.temb if self.dit else None,
+                chunks=6 if self.dit else 0,
+                table=self.table if self.dit else None, shift_idx=0,
+                scale_idx=1, act_scale=self.act[l if not self.dit else 0],
+                x8=self.x8, w8=lay["pk"].w8, w_scale=lay["pk"].w_scale,
+                bias=lay["pk"].bias, rope=self.rope, q_out=self.q[l % 2],
+                k_cache=lay["kc"], v_cache=lay["vc"], prefix_k=lay["pkd"],
+                prefix_v=lay["pvd"], prefix_T_src=lay["T_src"],
+                prefix_interleave=1, workspace=self.ws,
+                workspace_bytes=self.ws_bytes))
+
+    def e2e_step(self):
+        for k, t in self.pin_in.items():
+            d = self.dev_in[k]
+            d.view(self.torch.int16).copy_(t.view(d.shape), non_blocking=True)
+        for d in self.descs:
+            self.frt.frt_chain_layer(d)
+        for k, t in self.pin_out.items():
+            t.copy_(self.dev_out[k], non_blocking=True)
+
+
+class MlpRunner:
+    """Gate/up sibling MLP: AdaRMS producer -> packed gate/up FP8 GEMM with
+    the GEGLU + static requant epilogue -> down-projection FP8 GEMM."""
+
+    def __init__(self, w, torch, frt, rt, synth):
+        self.w, self.torch, self.frt, self.rt = w, torch, frt, rt
+        M, D, H = w.M, w.D, w.H
+        self.rows = M
+        mw = synth.mlp_weights(D, H, w.seed)
+        self.gu = rt.pack([mw["gate"], mw["up"]],
+                          layout=frt.FRT_PACK_GATE_UP_BLOCKS)
+        self.dn = rt.pack([mw["down"]])
+        inp = synth.adarms_inputs(M, D, w.seed)
+        self.host_in = {k: inp[k] for k in ("res", "delta", "prev_gate", "style")}
+        self.res0 = rt.bf16_dev(inp["res"])
+        self.res = self.res0.clone()
+        self.delta = rt.bf16_dev(inp["delta"])
+        self.gate = rt.bf16_dev(inp["prev_gate"])
+        self.style = rt.bf16_dev(inp["style"])
+        self.gate_out = rt.empty_bf16(M, D)
+        self.x8 = rt.empty_u8(M, D)
+        self.hid8 = rt.empty_u8(M, H)
+        self.out = rt.empty_bf16(M, D)
+        self.ws1 = frt.frt_gemm_workspace_size(M, 2 * H, D, frt.FRT_EPI_GEGLU_E4M3)
+        self.ws2 = frt.frt_gemm_workspace_size(M, D, H)
+        self.wsp1, self.wsp2 = rt.workspace(self.ws1), rt.workspace(self.ws2)
+        self.calibrate(synth, mw)
+        self.kerns = [
+            Kern("producer", "hbm", M * D * 9 + 4 * D * 2),
+            Kern("gemm_gateup_geglu", "tensor", 2 * H * D + M * D + M * H,
+                 2.0 * M * 2 * H * D),
+            Kern("gemm_down", "tensor", D * H + M * H + M * D * 2,
+                 2.0 * M * D * H),
+        ]
+        self.tokens = M
+        self.launches = 3
+
+    def calibrate(self, synth, mw):
+        torch, frt, rt, w = self.torch, self.frt, self.rt, self.w
+        C, D, H = w.cal_rows, w.D, w.H
+        cal = synth.adarms_inputs(C, D, w.seed + synth.CAL_OFFSET)
+        am = torch.zeros(1, dtype=torch.float32, device="cuda")
+        x8 = rt.empty_u8(C, D)
+        res = rt.bf16_dev(cal["res"])
+        frt.frt_ada_norm_quant_fp8(
+            frt.FRT_NORM_ADARMS, C, D, w.eps, res, rt.bf16_dev(cal["delta"]),
+            rt.bf16_dev(cal["prev_gate"]), 0, None, rt.bf16_dev(cal["style"]),
+            0, None, None, 0, None, 0, 0, rt.scale_dev(1.0), x8, None, am)
+        self.a_gu = rt.scale_dev(float(am.item()) / 448.0)
+        res = rt.bf16_dev(cal["res"])
+        frt.frt_ada_norm_quant_fp8(
+            frt.FRT_NORM_ADARMS, C, D, w.eps, res, rt.bf16_dev(cal["delta"]),
+            rt.bf16_dev(cal["prev_gate"]), 0, None, rt.bf16_dev(cal["style"]),
+            0, None, None, 0, None, 0, 0, self.a_gu, x8, None, None)
+        cat = rt.pack([mw["gate"], mw["up"]])
+        gu = rt.empty_bf16(C, 2 * H)
+        wsb = frt.frt_gemm_workspace_size(C, 2 * H, D)
+        frt.frt_packed_fp8_gemm(C, 2 * H, D, x8, cat.w8, self.a_gu,
+                                cat.w_scale, None, frt.FRT_EPI_BF16, gu,
+                                2 * H, None, rt.workspace(wsb), wsb)
+        am.zero_()
+        hid = rt.empty_u8(C, H)
+        frt.frt_geglu_quant_fp8(C, H, gu, 2 * H, rt.scale_dev(1.0), hid, am)
+        self.a_dn = rt.scale_dev(float(am.item()) / 448.0)
+        del cat, gu
+
+    def reset(self):
+        self.res.copy_(self.res0)
+
+    def step(self, ev=None):
+        frt, w = self.frt, self.w
+        M, D, H = w.M, w.D, w.H
+        if ev: ev[0][0][0].record()
+        frt.frt_ada_norm_quant_fp8(
+            frt.FRT_NORM_ADARMS, M, D, w.eps, self.res, self.delta, self.gate,
+            0, None, self.style, 0, None, None, 0, None, 0, 0, self.a_gu,
+            self.x8, self.gate_out, None)
+        if ev: ev[0][0][1].record()
+        if ev: ev[1][0][0].record()
+        frt.frt_packed_fp8_gemm(M, 2 * H, D, self.x8, self.gu.w8, self.a_gu,
+                                self.gu.w_scale, None, frt.FRT_EPI_GEGLU_E4M3,
+                                self.hid8, H, self.a_dn, self.wsp1, self.ws1)
+        if ev: ev[1][0][1].record()
+        if ev: ev[2][0][0].record()
+        frt.frt_packed_fp8_gemm(M, D, H, self.hid8, self.dn.w8, self.a_dn,
+                                self.dn.w_scale, None, frt.FRT_EPI_BF16,
+                                self.out, D, None, self.wsp2, self.ws2)
+        if ev: ev[2][0][1].record()
+
+    def e2e_setup(self):
+        torch = self.torch
+        self.pin_in = {k: torch.from_numpy(v.view(np.int16)).pin_memory()
+                       for k, v in self.host_in.items()}
+        self.dev_in = {"res": self.res, "delta": self.delta,
+                       "prev_gate": self.gate, "style": self.style}
+        self.dev_out = {"out": self.out, "res": self.res,
+                        "gate": self.gate_out}
+        self.pin_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory()
+                        for k, v in self.dev_out.items()}
+        self.h2d_bytes = sum(t.numel() * 2 for t in self.pin_in.values())
+        self.d2h_bytes = sum(t.numel() * 2 for t in self.pin_out.values())
+
+    def e2e_step(self):
+        for k, t in self.pin_in.items():
+            d = self.dev_in[k]
+            d.view(self.torch.int16).copy_(t.view(d.shape), non_blocking=True)
+        self.step()
+        for k, t in self.pin_out.items():
+            t.copy_(self.dev_out[k], non_blocking=True)
+
+
+def make_runner(name, torch, frt, rt, synth):
+    base, _, m = name.partition(":")
+    w = synth.WORKLOADS[base]
+    if m:
+        w = w.with_M(int(m))
+    if w.kind == "mlp":
+        return MlpRunner(w, torch, frt, rt, synth)
+    return ChainRunner(w, torch, frt, rt, synth)
+
+
+def workload_text(w):
+    if w.kind == "mlp":
+        return (f"{w.name}: M={w.M} D={w.D} gate/up {w.H} each (packed "
+                f"N={2 * w.H}) + GEGLU requant + down [{w.D},{w.H}]")
+    s = (f"{w.name}: B={w.B} M={w.M} D={w.D} Hq={w.hq}x{w.hd} "
+         f"Hkv={w.hkv}x{w.hd} N={w.N} P={w.P} T={w.T}")
+    if w.layers > 1:
+        s += f", {w.layers} layers, residual carried"
+    return s + (" bias" if w.bias else "")
+
+
+# ------------------------------------------------------- CPU oracle arm ----
+
+def oracle_sampler(name, synth, rows_cap=None):
+    """Closure running the CPU oracle on a bounded sample of the workload:
+    all tokens when that is cheap, else a seeded subset of rows (rows are
+    independent through the whole chain).  Returns (fn, tokens, text)."""
+    import oracle
+    base, _, m = name.partition(":")
+    w = synth.WORKLOADS[base]
+    if m:
+        w = w.with_M(int(m))
+    rng = np.random.default_rng(7)
+    if w.kind == "mlp":
+        n = rows_cap or 32
+        sel = np.sort(rng.choice(w.M, size=min(n, w.M), replace=False))
+        mw = synth.mlp_weights(w.D, w.H, w.seed)
+        gu_p = oracle.pack_weights_fp8([mw["gate"], mw["up"]])
+        dn_p = oracle.pack_weights_fp8([mw["down"]])
+        inp = synth.adarms_inputs(w.M, w.D, w.seed)
+        sub = {k: (v[sel] if v.shape[0] == w.M else v) for k, v in inp.items()}
+
+        def fn():
+            pr = oracle.ada_rms_norm_quant(sub["res"], sub["delta"],
+                                           sub["prev_gate"], sub["style"],
+                                           0.01, eps=w.eps)
+            gu = oracle.fp8_gemm(pr["x8"], gu_p["w8"], 0.01, gu_p["w_scale"])
+            hid, _ = oracle.geglu_quant(gu, 0.05)
+            oracle.fp8_gemm(hid, dn_p["w8"], 0.05, dn_p["w_scale"])
+        return fn, len(sel), f"{len(sel)} of {w.M} rows, full MLP per row"
+
+    L = w.layers
+    rows = w.rows
+    n = rows if rows_cap is None else min(rows, rows_cap)
+    if rows > 256 and rows_cap is None:
+        n = 64 if w.kind == "dit" else 256
+    sel = np.sort(rng.choice(rows, size=n, replace=False)) if n < rows \
+        else np.arange(rows)
+    layers = []
+    for l in range(L):
+        if L > 1:
+            li = synth.stack_layer_inputs(w, l)
+            ws, bs, style = li["w"], li["b"], li["style"]
+            pkh, pvh = li["prefix_k"], li["prefix_v"]
+        else:
+            ws, bs = synth.qkv_weights(w.hq, w.hkv, w.hd, w.D, w.seed,
+                                       bias=w.bias)
+            style, pkh, pvh = None, None, None
+            if w.P > 0:
+                pkh, pvh = synth.prefix_cache(w.B, w.hkv, max(1024, w.P),
+                                              w.hd, w.seed)
+        pk = oracle.pack_weights_fp8(ws, bs, layout=0 if w.kind == "dit" else 1,
+                                     hd=w.hd)
+        layers.append((pk, style, pkh, pvh))
+    rope = oracle.rope_table(w.M, w.hd, w.P, w.theta)
+    kc0 = np.zeros((w.B, w.T, w.hkv, w.hd), np.uint16)
+    if w.kind == "dit":
+        inp = synth.dit_inputs(rows, w.D, w.seed)
+        x, temb, table = inp["x"][sel], inp["temb"][sel], inp["table"]
+    else:
+        inp = synth.adarms_inputs(rows, w.D, w.seed, outliers=w.outliers)
+        sub = {k: (v[sel] if v.shape[0] == rows else v) for k, v in inp.items()}
+    s_of = sel % w.M
+
+    def fn():
+        res = None if w.kind == "dit" else sub["res"]
+        delta = gate = None
+        for l, (pk, style, pkh, pvh) in enumerate(layers):
+            if pkh is not None:
+                oracle.prefix_copy(pkh, pvh, w.P, kc0, kc0, interleave=True)
+            if w.kind == "dit":
+                x8 = oracle.ada_layer_norm_quant_table(x, temb, table, 0, 1,
+                                                       0.01, eps=w.eps)["x8"]
+            else:
+                if L == 1:
+                    d, g, st = sub["delta"], sub["prev_gate"], sub["style"]
+                elif l == 0:
+                    d = np.zeros_like(res)
+                    g, st = np.zeros((1, w.D), np.uint16), style
+                else:
+                    d, g, st = delta, gate, style
+                pr = oracle.ada_rms_norm_quant(res, d, g, st, 0.01, eps=w.eps)
+                res, x8, gate = pr["res"], pr["x8"], pr["gate_out"]
+            qkv = oracle.fp8_gemm(x8, pk["w8"], 0.01, pk["w_scale"],
+                                  pk["bias"] if w.bias else None)
+            # split + RoPE row by row (each sampled row has its own position)
+            qs = []
+            for i in range(len(sel)):
+                s = int(s_of[i])
+                kk = np.zeros((1, 1, w.hkv, w.hd), np.uint16)
+                q, _, _ = oracle.split_rope_kvcache(
+                    qkv[i:i + 1], rope[s:s + 1], 1, 1, w.hq, w.hkv, w.hd, 0,
+                    kk, kk)
+                qs.append(q.reshape(-1))
+            delta = np.stack(qs) if w.hq * w.hd == w.D else None
+    return fn, len(sel) * 1, (f"{len(sel)} of {rows} rows, {L} layer(s) "
+                              "of prefix copy + producer + GEMM + split/RoPE")
+
+
+def cpu_baseline(name, synth, seconds=12.0):
+    import oracle
+    fn, tokens, text = oracle_sampler(name, synth)
+    fn()  # warm
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or n >= 2000:
+            break
+    return {"value": tokens * n / el, "unit": "tokens/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{text}; {n} repetitions in {el:.1f} s"}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from fp8_transformer_block_b200 import synth
+    import oracle
+    fn, tokens, text = oracle_sampler(args.config, synth)
+    t0 = time.perf_counter()
+    fn()
+    t1 = time.perf_counter() - t0
+    cap = None
+    if args.steps * t1 > 150.0:   # keep the whole run within a few minutes
+        base, _, m = args.config.partition(":")
+        w = synth.WORKLOADS[base]
+        full = w.M if w.kind == "mlp" else w.rows
+        cap = max(1, int(full * 150.0 / (args.steps * t1) * 0.5))
+        fn, tokens, text = oracle_sampler(args.config, synth, rows_cap=cap)
+    for _ in range(args.warmup):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fn()
+    el = time.perf_counter() - t0
+    v = tokens * args.steps / el
+    base, _, m = args.config.partition(":")
+    w = synth.WORKLOADS[base].with_M(int(m)) if m else synth.WORKLOADS[base]
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3/fp32",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload_text(w),
+                       "sample_per_step": text},
+            "cpu_baseline": {"value": v, "unit": "tokens/s",
+                             "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": text},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU arm --
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+    from fp8_transformer_block_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    from fp8_transformer_block_b200 import frt, synth
+    from fp8_transformer_block_b200 import runtime as rt
+
+    runner = make_runner(args.config, torch, frt, rt, synth)
+    w = runner.w
+    kinds = runner.kerns
+    L = getattr(runner, "L", 1)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    sleep_cycles = max(1_000_000, 300_000 * runner.launches)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        runner.reset()
+        runner.step()
+    torch.cuda.synchronize()
+    assert frt.frt_device_status(True) == frt.FRT_OK
+
+    K = args.steps
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    s_ev = [(mk(), mk()) for _ in range(K)]
+    k_ev = [[[(mk(), mk()) for _ in range(L if k.per_step > 1 else 1)]
+             for k in kinds] for _ in range(K)]
+    gpu_id = str(local)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # noqa: BLE001
+        pass
+    clocks = ClockSampler(gpu_id)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_wall = time.perf_counter()
+    for i in range(K):
+        runner.reset()
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(sleep_cycles)
+        s_ev[i][0].record()
+        runner.step(k_ev[i])
+        s_ev[i][1].record()
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - t_wall
+    clk = clocks.stop()
+    assert frt.frt_device_status(True) == frt.FRT_OK
+
+    step_ms = [a.elapsed_time(b) for a, b in s_ev]
+    total_ms = sum(step_ms)
+    kern_ms = []
+    for kk, kd in enumerate(kinds):
+        tot = sum(a.elapsed_time(b) for i in range(K) for a, b in k_ev[i][kk])
+        kern_ms.append(tot / (K * len(k_ev[0][kk])))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_total_ms = float(t.item())
+    ms_per_step = max_total_ms / K
+    value = world * runner.tokens * K / (max_total_ms / 1e3)
+
+    # ---- e2e through the public entry points with host buffers
+    runner.e2e_setup()
+    for _ in range(3):
+        runner.e2e_step()
+    torch.cuda.synchronize()
+    KE = min(K, 200)
+    e_ev = [(mk(), mk()) for _ in range(KE)]
+    barrier()
+    for i in range(KE):
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(sleep_cycles)
+        e_ev[i][0].record()
+        runner.e2e_step()
+        e_ev[i][1].record()
+    torch.cuda.synchronize()
+    e_ms = sum(a.elapsed_time(b) for a, b in e_ev)
+    te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * runner.tokens * KE / (float(te.item()) / 1e3)
+
+    # ---- roofline of the dominant kernel
+    hbm, bf16_burst, bf16_sust, src = _peaks()
+    shares = [ms * k.per_step for ms, k in zip(kern_ms, kinds)]
+    dom = int(np.argmax(shares))
+    kd = kinds[dom]
+    if kd.bound == "tensor":
+        achieved = kd.flops / (kern_ms[dom] * 1e-3) / 1e12
+        peak = bf16_burst * FP8_PER_BF16
+        unit = "TFLOP/s"
+    else:
+        achieved = kd.algo_bytes / (kern_ms[dom] * 1e-3) / 1e9
+        peak = hbm
+        unit = "GB/s"
+    tr = NCU_TRAFFIC.get((args.config, kd.name))
+    traffic = tr[0] if tr and tr[1] == _src_hash() else None
+    kern_list = []
+    for ms, k in zip(kern_ms, kinds):
+        e = {"kernel": k.name, "us": round(ms * 1e3, 3),
+             "launches_per_step": k.per_step, "bound": k.bound,
+             "algo_bytes": int(k.algo_bytes),
+             "GB_s": round(k.algo_bytes / (ms * 1e-3) / 1e9, 1),
+             "hbm_frac": round(k.algo_bytes / (ms * 1e-3) / 1e9 / hbm, 4)}
+        if k.flops:
+            e["TFLOP_s"] = round(k.flops / (ms * 1e-3) / 1e12, 2)
+            e["fp8_frac"] = round(k.flops / (ms * 1e-3) / 1e12 /
+                                  (bf16_burst * FP8_PER_BF16), 4)
+        kern_list.append(e)
+
+    if rank != 0:
+        return 0
+    cpu = None
+    if world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(args.config, synth, seconds=args.cpu_seconds)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "us_per_layer": 1e3 * ms_per_step / L,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3/fp32", "data": "synthetic",
+        "config": {"workload": workload_text(w),
+                   "l2": "flushed before every timed step (256 MB write)",
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "timing": "CUDA events per step on the launching stream"},
+        "roofline": {"bound": kd.bound, "kernel": kd.name,
+                     "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{src} "
+                     + ("(bf16 burst x 2, nominal fp8/bf16 ratio)"
+                        if unit == "TFLOP/s" else "(HBM copy)"),
+                     "algo_per_launch": kd.flops if unit == "TFLOP/s"
+                     else kd.algo_bytes},
+        "kernels": kern_list,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(runner.h2d_bytes),
+                "d2h_bytes_per_step": int(runner.d2h_bytes)},
+        "gpu_launches": runner.launches * K,
+        "clocks": clk,
+        "wall_s_timed_loop": round(wall, 3),
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", default="frt", choices=["frt", "reference"])
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
