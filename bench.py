@@ -224,7 +224,8 @@ class ChainRunner:
                        gbytes, gflops, per_step=self.L))
         self.kerns = ks
         self.tokens = rows
-        self.launches = sum(k.per_step for k in ks)
+        self.launches = 2 * self.L   # frt_chain_layer: producer(+prefix), GEMM
+        self._build_descs()
 
     # ----------------------------------------------------------------------
     def _inputs(self, l):
@@ -313,28 +314,53 @@ class ChainRunner:
         self.res.copy_(self.res0)
 
     # ----------------------------------------------------------------------
+    def _build_descs(self):
+        frt, rt, w = self.frt, self.rt, self.w
+        self.descs = []
+        for l, lay in enumerate(self.layers):
+            d, g, gs, st = self._inputs(l) if not self.dit else (None,) * 4
+            self.descs.append(rt.chain_desc(
+                B=w.B, M=w.M, D=w.D, hq=w.hq, hkv=w.hkv, hd=w.hd, P=w.P,
+                T=w.T, eps=w.eps,
+                norm_mode=(frt.FRT_NORM_LAYERNORM_TABLE if self.dit
+                           else frt.FRT_NORM_ADARMS),
+                flags=frt.FRT_CHAIN_FUSED_ROPE,
+                res=None if self.dit else self.res, delta=d, prev_gate=g,
+                gate_row_stride=gs or 0, style=st, style_row_stride=0,
+                gate_out=None if self.dit else self.gate_out[l % 2],
+                x=self.x if self.dit else None,
+                temb=self.temb if self.dit else None,
+                chunks=6 if self.dit else 0,
+                table=self.table if self.dit else None, shift_idx=0,
+                scale_idx=1, act_scale=self.act[l if not self.dit else 0],
+                x8=self.x8, w8=lay["pk"].w8, w_scale=lay["pk"].w_scale,
+                bias=lay["pk"].bias, rope=self.rope, q_out=self.q[l % 2],
+                k_cache=lay["kc"], v_cache=lay["vc"], prefix_k=lay["pkd"],
+                prefix_v=lay["pvd"], prefix_T_src=lay["T_src"],
+                prefix_interleave=1, workspace=self.ws,
+                workspace_bytes=self.ws_bytes))
+
     def reset(self):
         """Restore the state a step mutates (the residual); untimed."""
         if not self.dit:
             self.res.copy_(self.res0)
 
-    def step(self, ev=None):
-        """Issue one step; ev[k][l] = (start, end) events per kernel kind k
-        and layer l, or None."""
-        for l in range(self.L):
-            k = 0
-            if self.layers[l]["pkd"] is not None:
-                if ev: ev[k][l][0].record()
-                self._prefix(l)
-                if ev: ev[k][l][1].record()
-                k += 1
-            if ev: ev[k][l][0].record()
-            self._producer(l, self.act[l if not self.dit else 0])
-            if ev: ev[k][l][1].record()
-            k += 1
-            if ev: ev[k][l][0].record()
-            self._gemm(l, self.act[l if not self.dit else 0])
-            if ev: ev[k][l][1].record()
+    def step(self):
+        """One step through the public entry point: frt_chain_layer per
+        layer (producer + prefix in one launch, then the fused GEMM)."""
+        for d in self.descs:
+            self.frt.frt_chain_layer(d)
+
+    def kernel_calls(self):
+        """(Kern, call) pairs timing each kernel alone through the C ABI."""
+        kc = []
+        by = {k.name: k for k in self.kerns}
+        if "prefix_copy" in by:
+            kc.append((by["prefix_copy"], lambda: self._prefix(0)))
+        kc.append((by["producer"],
+                   lambda: self._producer(0, self.act[0])))
+        kc.append((by["gemm_rope_kv"], lambda: self._gemm(0, self.act[0])))
+        return kc
 
     # ---------------------------------------------------------------- e2e --
     def e2e_setup(self):
@@ -367,37 +393,12 @@ class ChainRunner:
                              for t in self.pin_in.values())
         self.d2h_bytes = sum(t.numel() * t.element_size()
                              for t in self.pin_out.values())
-        self.descs = []
-        frt, rt = self.frt, self.rt
-        for l, lay in enumerate(self.layers):
-            d, g, gs, st = self._inputs(l) if not self.dit else (None,) * 4
-            self.descs.append(rt.chain_desc(
-                B=w.B, M=w.M, D=w.D, hq=w.hq, hkv=w.hkv, hd=w.hd, P=w.P,
-                T=w.T, eps=w.eps,
-                norm_mode=(frt.FRT_NORM_LAYERNORM_TABLE if self.dit
-                           else frt.FRT_NORM_ADARMS),
-                flags=frt.FRT_CHAIN_FUSED_ROPE,
-                res=None if self.dit else self.res, delta=d, prev_gate=g,
-                gate_row_stride=gs or 0, style=st, style_row_stride=0,
-                gate_out=None if self.dit else self.gate_out[l % 2],
-                x=self.x if self.dit else None,
-                temb=self.temb if self.dit else None,
-                chunks=6 if self.dit else 0,
-                table=self.table if self.dit else None, shift_idx=0,
-                scale_idx=1, act_scale=self.act[l if not self.dit else 0],
-                x8=self.x8, w8=lay["pk"].w8, w_scale=lay["pk"].w_scale,
-                bias=lay["pk"].bias, rope=self.rope, q_out=self.q[l % 2],
-                k_cache=lay["kc"], v_cache=lay["vc"], prefix_k=lay["pkd"],
-                prefix_v=lay["pvd"], prefix_T_src=lay["T_src"],
-                prefix_interleave=1, workspace=self.ws,
-                workspace_bytes=self.ws_bytes))
 
     def e2e_step(self):
         for k, t in self.pin_in.items():
             d = self.dev_in[k]
             d.view(self.torch.int16).copy_(t.view(d.shape), non_blocking=True)
-        for d in self.descs:
-            self.frt.frt_chain_layer(d)
+        self.step()
         for k, t in self.pin_out.items():
             t.copy_(self.dev_out[k], non_blocking=True)
 
@@ -471,25 +472,35 @@ class MlpRunner:
     def reset(self):
         self.res.copy_(self.res0)
 
-    def step(self, ev=None):
+    def _producer(self):
         frt, w = self.frt, self.w
-        M, D, H = w.M, w.D, w.H
-        if ev: ev[0][0][0].record()
         frt.frt_ada_norm_quant_fp8(
-            frt.FRT_NORM_ADARMS, M, D, w.eps, self.res, self.delta, self.gate,
-            0, None, self.style, 0, None, None, 0, None, 0, 0, self.a_gu,
-            self.x8, self.gate_out, None)
-        if ev: ev[0][0][1].record()
-        if ev: ev[1][0][0].record()
-        frt.frt_packed_fp8_gemm(M, 2 * H, D, self.x8, self.gu.w8, self.a_gu,
-                                self.gu.w_scale, None, frt.FRT_EPI_GEGLU_E4M3,
-                                self.hid8, H, self.a_dn, self.wsp1, self.ws1)
-        if ev: ev[1][0][1].record()
-        if ev: ev[2][0][0].record()
-        frt.frt_packed_fp8_gemm(M, D, H, self.hid8, self.dn.w8, self.a_dn,
-                                self.dn.w_scale, None, frt.FRT_EPI_BF16,
-                                self.out, D, None, self.wsp2, self.ws2)
-        if ev: ev[2][0][1].record()
+            frt.FRT_NORM_ADARMS, w.M, w.D, w.eps, self.res, self.delta,
+            self.gate, 0, None, self.style, 0, None, None, 0, None, 0, 0,
+            self.a_gu, self.x8, self.gate_out, None)
+
+    def _gateup(self):
+        frt, w = self.frt, self.w
+        frt.frt_packed_fp8_gemm(w.M, 2 * w.H, w.D, self.x8, self.gu.w8,
+                                self.a_gu, self.gu.w_scale, None,
+                                frt.FRT_EPI_GEGLU_E4M3, self.hid8, w.H,
+                                self.a_dn, self.wsp1, self.ws1)
+
+    def _down(self):
+        frt, w = self.frt, self.w
+        frt.frt_packed_fp8_gemm(w.M, w.D, w.H, self.hid8, self.dn.w8,
+                                self.a_dn, self.dn.w_scale, None,
+                                frt.FRT_EPI_BF16, self.out, w.D, None,
+                                self.wsp2, self.ws2)
+
+    def step(self):
+        self._producer()
+        self._gateup()
+        self._down()
+
+    def kernel_calls(self):
+        return list(zip(self.kerns, (self._producer, self._gateup,
+                                     self._down)))
 
     def e2e_setup(self):
         torch = self.torch
@@ -716,7 +727,6 @@ def run_gpu(args):
 
     runner = make_runner(args.config, torch, frt, rt, synth)
     w = runner.w
-    kinds = runner.kerns
     L = getattr(runner, "L", 1)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     sleep_cycles = max(1_000_000, 300_000 * runner.launches)
@@ -734,8 +744,6 @@ def run_gpu(args):
     K = args.steps
     mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     s_ev = [(mk(), mk()) for _ in range(K)]
-    k_ev = [[[(mk(), mk()) for _ in range(L if k.per_step > 1 else 1)]
-             for k in kinds] for _ in range(K)]
     gpu_id = str(local)
     try:
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -751,7 +759,7 @@ def run_gpu(args):
         flush.fill_(i & 0xFF)
         torch.cuda._sleep(sleep_cycles)
         s_ev[i][0].record()
-        runner.step(k_ev[i])
+        runner.step()
         s_ev[i][1].record()
     torch.cuda.synchronize()
     barrier()
@@ -761,16 +769,28 @@ def run_gpu(args):
 
     step_ms = [a.elapsed_time(b) for a, b in s_ev]
     total_ms = sum(step_ms)
-    kern_ms = []
-    for kk, kd in enumerate(kinds):
-        tot = sum(a.elapsed_time(b) for i in range(K) for a, b in k_ev[i][kk])
-        kern_ms.append(tot / (K * len(k_ev[0][kk])))
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     max_total_ms = float(t.item())
     ms_per_step = max_total_ms / K
     value = world * runner.tokens * K / (max_total_ms / 1e3)
+
+    # ---- each kernel alone (cold L2, GPU held until the launch is queued)
+    KK = max(20, min(K, 200))
+    kern_ms = []
+    for kd, call in runner.kernel_calls():
+        evs = [(mk(), mk()) for _ in range(KK)]
+        for i in range(KK):
+            runner.reset()
+            flush.fill_(i & 0xFF)
+            torch.cuda._sleep(1_000_000)
+            evs[i][0].record()
+            call()
+            evs[i][1].record()
+        torch.cuda.synchronize()
+        kern_ms.append(sum(a.elapsed_time(b) for a, b in evs) / KK)
+    kinds = [kd for kd, _ in runner.kernel_calls()]
 
     # ---- e2e through the public entry points with host buffers
     runner.e2e_setup()
@@ -793,7 +813,7 @@ def run_gpu(args):
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     e2e_value = world * runner.tokens * KE / (float(te.item()) / 1e3)
 
-    # ---- roofline of the dominant kernel
+    # ---- roofline of the dominant kernel (largest share of a step)
     hbm, bf16_burst, bf16_sust, src = _peaks()
     shares = [ms * k.per_step for ms, k in zip(kern_ms, kinds)]
     dom = int(np.argmax(shares))
@@ -835,7 +855,8 @@ def run_gpu(args):
         "config": {"workload": workload_text(w),
                    "l2": "flushed before every timed step (256 MB write)",
                    "parallelism": "replicas" if world > 1 else "single",
-                   "timing": "CUDA events per step on the launching stream"},
+                   "timing": "CUDA events per step on the launching stream; "
+                             "kernels timed alone the same way"},
         "roofline": {"bound": kd.bound, "kernel": kd.name,
                      "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic,

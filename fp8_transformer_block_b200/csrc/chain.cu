@@ -7,11 +7,13 @@
 // `ad:prefix` range; impls/modnorm_qkv_chain/fp8_ptok_table.py: the
 // per-token-table producer feeding the Q/K/V wire projections.
 //
-// Launch sequence on one stream, no host synchronisation:
-//   [prefix copy] -> producer -> packed GEMM with the split + RoPE + KV write
-//   in its epilogue (FRT_CHAIN_FUSED_ROPE), or packed GEMM -> qkv -> split
-//   kernel carrying the prefix copy too (FRT_CHAIN_UNFUSED).
-#include "frt_common.cuh"
+// Launch sequence on one stream, no host synchronisation, every kernel with
+// programmatic dependent launch (each starts while its predecessor drains):
+//   FRT_CHAIN_FUSED_ROPE: producer (its extra blocks copy the prefix) ->
+//     packed GEMM with the split + RoPE + KV write in its epilogue;
+//   FRT_CHAIN_UNFUSED: producer -> packed GEMM -> qkv -> split kernel that
+//     also copies the prefix.
+#include "frt_internal.cuh"
 
 extern "C" size_t frt_chain_workspace_size(const frt_chain_desc* d) {
   if (!d) return 0;
@@ -35,15 +37,18 @@ extern "C" int frt_chain_layer(const frt_chain_desc* d, void* stream) {
   FRT_REQUIRE(d->P >= 0 && d->P + d->M <= d->T, FRT_ERANGE,
               "P + M = %d exceeds the cache capacity T = %d", d->P + d->M, d->T);
   int rc;
-  if (d->flags == FRT_CHAIN_FUSED_ROPE && d->prefix_k) {
-    rc = frt_prefix_copy_kv(d->B, d->hkv, d->hd, d->P, d->T, d->prefix_T_src, d->prefix_k,
-                            d->prefix_v, d->prefix_interleave, d->k_cache, d->v_cache, stream);
+  frt::PrefixArgs pre{};
+  const bool fuse_prefix = d->flags == FRT_CHAIN_FUSED_ROPE && d->prefix_k;
+  if (fuse_prefix) {
+    rc = frt::prefix_args(d->B, d->hkv, d->hd, d->P, d->T, d->prefix_T_src, d->prefix_k,
+                          d->prefix_v, d->prefix_interleave, d->k_cache, d->v_cache, &pre);
     if (rc) return rc;
   }
-  rc = frt_ada_norm_quant_fp8(d->norm_mode, rows, d->D, d->eps, d->res, d->delta, d->prev_gate,
-                              d->gate_row_stride, d->norm_weight, d->style, d->style_row_stride,
-                              d->x, d->temb, d->chunks, d->table, d->shift_idx, d->scale_idx,
-                              d->act_scale, d->x8, d->gate_out, nullptr, stream);
+  rc = frt::producer_call(d->norm_mode, rows, d->D, d->eps, d->res, d->delta, d->prev_gate,
+                          d->gate_row_stride, d->norm_weight, d->style, d->style_row_stride, d->x,
+                          d->temb, d->chunks, d->table, d->shift_idx, d->scale_idx, d->act_scale,
+                          d->x8, d->gate_out, nullptr, fuse_prefix ? &pre : nullptr,
+                          static_cast<cudaStream_t>(stream));
   if (rc) return rc;
   if (d->flags == FRT_CHAIN_FUSED_ROPE) {
     return frt_packed_fp8_gemm_rope_kvcache(d->B, d->M, d->D, d->hq, d->hkv, d->hd, d->P, d->T,

@@ -36,6 +36,35 @@ inline bool aligned(const void* p, size_t a) {
 #define FRT_REQUIRE(cond, code, ...) \
   do { if (!(cond)) return ::frt::fail((code), __VA_ARGS__); } while (0)
 
+namespace frt {
+
+// Launch with programmatic dependent launch allowed: the kernel may begin
+// (prologue, loads of data no earlier kernel writes) while its predecessor in
+// the stream finishes.  Every kernel launched this way executes pdl_wait()
+// before it touches memory an earlier kernel may read or write.
+template <typename... KArgs, typename... Args>
+int launch_pdl(const char* what, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+               cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FRT_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+  }
+  return FRT_OK;
+}
+
+}  // namespace frt
+
 // ---------------------------------------------------------------- device --
 
 namespace frt {
@@ -99,6 +128,15 @@ __device__ __forceinline__ float warp_max(float v) {
 // of non-negative floats order like unsigned integers.
 __device__ __forceinline__ void atomic_max_nonneg(float* dst, float v) {
   atomicMax(reinterpret_cast<unsigned int*>(dst), __float_as_uint(v));
+}
+
+// Programmatic dependent launch: wait for the preceding kernel's completion
+// (and the visibility of its writes); allow the next kernel to start early.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

@@ -17,6 +17,8 @@ __global__ void geglu_kernel(int M, int H, const uint16_t* gu, long ld, const fl
                              uint8_t* hid8, float* amax) {
   const int h8 = H / 8;
   const long total = long(M) * h8;
+  pdl_trigger();
+  pdl_wait();
   const float os = __ldg(out_scale);
   float mx = 0.0f;
   for (long g = blockIdx.x * long(blockDim.x) + threadIdx.x; g < total;
@@ -56,7 +58,7 @@ extern "C" int frt_geglu_quant_fp8(int M, int H, const frt_bf16* gu, long ld_gu,
   const long total = long(M) * (H / 8);
   const long need = (total + 255) / 256;
   const int grid = int(need < frt::num_sms() * 16L ? need : frt::num_sms() * 16L);
-  frt::geglu_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(M, H, gu, ld_gu,
-                                                                         out_scale, hid8, amax_out);
-  return frt::check_launch("frt_geglu_quant_fp8");
+  return frt::launch_pdl("geglu_kernel", frt::geglu_kernel, dim3(grid), dim3(256), 0,
+                         static_cast<cudaStream_t>(stream), M, H, gu, ld_gu, out_scale, hid8,
+                         amax_out);
 }

@@ -69,11 +69,6 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(int n) {
   return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512;
 }
 
-template <int BN, int STAGES>
-constexpr int smem_bytes() {
-  return STAGES * (A_BYTES + BN * BK) + 1024 /* alignment slack */ + 256 /* barriers */;
-}
-
 __device__ __forceinline__ void record_timeout(int* status) {
   if (status) atomicExch(status, FRT_ETIMEOUT);
 }
@@ -89,13 +84,33 @@ __device__ __forceinline__ float scale_bias_bf16(float acc, float alpha, const u
   return bf2f(f2bf(y));
 }
 
-// Normal orientation: this thread owns token row m, columns n0 .. n0 + 31.
+// 32 consecutive bf16 starting at a 64-byte aligned address -> floats.
+__device__ __forceinline__ void load32_bf16(const uint16_t* src, float (&f)[32]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float t[8];
+    unpack8(__ldg(s4 + k), t);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[8 * k + j] = t[j];
+  }
+}
+
+// This thread owns token row m, output columns n0 .. n0 + 31 (the normal
+// orientation, and the swapped one after the shared-memory transpose).
 __device__ __forceinline__ void epi_rows_chunk(const GemmParams& p, const float (&v)[32], int m,
                                                int n0, float alpha) {
   if (m >= p.M) return;
   float y[32];
+  if (p.bias) {
+    float b[32];
+    load32_bf16(p.bias + n0, b);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) y[j] = scale_bias_bf16(v[j], alpha, p.bias, n0 + j);
+    for (int j = 0; j < 32; ++j) y[j] = bf2f(f2bf(__fadd_rn(__fmul_rn(v[j], alpha), b[j])));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) y[j] = bf2f(f2bf(__fmul_rn(v[j], alpha)));
+  }
   uint16_t* dst;
   if (p.epi == EPI_BF16) {
     dst = static_cast<uint16_t*>(p.out) + long(m) * p.ldo + n0;
@@ -103,10 +118,11 @@ __device__ __forceinline__ void epi_rows_chunk(const GemmParams& p, const float 
     const int b = m / p.Mseq, s = m % p.Mseq;
     const int h = n0 / p.hd, d0 = n0 % p.hd;
     if (h < p.hq + p.hkv) {
-      const uint16_t* rp = p.rope + long(s) * p.hd + d0;
+      float r[32];
+      load32_bf16(p.rope + long(s) * p.hd + d0, r);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float c = bf2f(__ldg(rp + 2 * i)), sn = bf2f(__ldg(rp + 2 * i + 1));
+        const float c = r[2 * i], sn = r[2 * i + 1];
         const float x0 = y[2 * i], x1 = y[2 * i + 1];
         y[2 * i] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, sn));
         y[2 * i + 1] = __fadd_rn(__fmul_rn(x0, sn), __fmul_rn(x1, c));
@@ -125,56 +141,6 @@ __device__ __forceinline__ void epi_rows_chunk(const GemmParams& p, const float 
 #pragma unroll
     for (int j = 0; j < 8; ++j) f[j] = y[8 * k + j];
     d4[k] = pack8_bf16(f);
-  }
-}
-
-// Swapped orientation: this thread (lane) owns output column n, tokens
-// m0 .. m0 + 31.  Pairs (n, n ^ 1) live in neighbouring lanes.
-__device__ __forceinline__ void epi_cols_chunk(const GemmParams& p, const float (&v)[32], int n,
-                                               int m0, float alpha, int lane) {
-  const bool col_ok = n < p.N;
-  const float bias = (p.bias && col_ok) ? bf2f(__ldg(p.bias + n)) : 0.0f;
-  if (p.epi == EPI_BF16) {
-    if (!col_ok) return;
-    uint16_t* out = static_cast<uint16_t*>(p.out);
-#pragma unroll 4
-    for (int j = 0; j < 32; ++j) {
-      const int m = m0 + j;
-      if (m < p.M) {
-        float y = __fmul_rn(v[j], alpha);
-        if (p.bias) y = __fadd_rn(y, bias);
-        out[long(m) * p.ldo + n] = f2bf(y);
-      }
-    }
-    return;
-  }
-  // EPI_ROPE: the warp's 32 columns lie inside one head
-  const int h = n / p.hd, d = n % p.hd;
-  const bool rot = h < p.hq + p.hkv;
-  const bool odd = (lane & 1) != 0;
-  for (int j = 0; j < 32; ++j) {
-    const int m = m0 + j;
-    float y = __fmul_rn(v[j], alpha);
-    if (p.bias) y = __fadd_rn(y, bias);
-    y = bf2f(f2bf(y));
-    const float other = __shfl_xor_sync(0xffffffffu, y, 1);
-    if (m >= p.M || !col_ok) continue;
-    const int b = m / p.Mseq, s = m % p.Mseq;
-    uint16_t* dst;
-    float o = y;
-    if (rot) {
-      const uint16_t* rp = p.rope + long(s) * p.hd + (d & ~1);
-      const float c = bf2f(__ldg(rp)), sn = bf2f(__ldg(rp + 1));
-      const float x0 = odd ? other : y, x1 = odd ? y : other;
-      o = odd ? __fadd_rn(__fmul_rn(x0, sn), __fmul_rn(x1, c))
-              : __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, sn));
-      dst = h < p.hq ? p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d
-                     : p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d;
-    } else {
-      const int hv = h - p.hq - p.hkv;
-      dst = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + hv) * p.hd + d;
-    }
-    *dst = f2bf(o);
   }
 }
 
@@ -204,10 +170,16 @@ __device__ __forceinline__ void epi_geglu_chunk(const GemmParams& p, const float
 }
 
 // Run the epilogue of one tile.  load(c, v) fills v with accumulator chunk c
-// (32 columns); it is called warp-uniformly.
-template <bool SWAP, int BN, class Load>
+// (32 columns of this thread's TMEM lane); it is called warp-uniformly.
+// done() runs once every chunk has been loaded (it releases the TMEM
+// accumulator when the chunks come from TMEM).
+// Swapped orientation: the chunks are staged in the shared-memory tile T
+// (fp32 [128 output columns][BN tokens], row stride BN + 4) and read back
+// transposed, so each thread then owns one token row with 32 contiguous
+// output columns and the row epilogue applies unchanged.
+template <bool SWAP, int BN, class Load, class Done>
 __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int tb, int q, int lane,
-                                              float alpha, Load load) {
+                                              float alpha, float* T, Load load, Done done) {
   if (!SWAP && p.epi == EPI_GEGLU) {
     const int m = ta * BM + 32 * q + lane;
 #pragma unroll 1
@@ -215,29 +187,66 @@ __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int t
       float g[32], u[32];
       load(c, g);
       load(c + 4, u);
+      if (c == 3) done();
       epi_geglu_chunk(p, g, u, m, tb * BN + 32 * c, tb * BN + 128 + 32 * c, tb * 128 + 32 * c,
                       alpha);
     }
     return;
   }
+  if (!SWAP) {
+    const int m = ta * BM + 32 * q + lane;
+    int c_last = BN / 32 - 1;
+    while (c_last > 0 && tb * BN + 32 * c_last >= p.N) --c_last;
+#pragma unroll 1
+    for (int c = 0; c <= c_last; ++c) {
+      float v[32];
+      load(c, v);
+      if (c == c_last) done();
+      epi_rows_chunk(p, v, m, tb * BN + 32 * c, alpha);
+    }
+    return;
+  }
+  constexpr int TS = BN + 4;
+  const int row = 32 * q + lane;
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     float v[32];
-    if (!SWAP) {
-      const int n0 = tb * BN + 32 * c;
-      if (n0 >= p.N) break;
-      load(c, v);
-      epi_rows_chunk(p, v, ta * BM + 32 * q + lane, n0, alpha);
-    } else {
-      const int m0 = tb * BN + 32 * c;
-      if (m0 >= p.M) break;
-      load(c, v);
-      epi_cols_chunk(p, v, ta * BM + 32 * q + lane, m0, alpha, lane);
-    }
+    load(c, v);
+    float4* d4 = reinterpret_cast<float4*>(T + row * TS + 32 * c);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
   }
+  done();
+  named_bar_sync(2, 128);
+  constexpr int COLS = BM * BN / 128;   // output columns per thread (BN for BN <= 128)
+  const int t = int(threadIdx.x) - 64;  // 0 .. 127 over the four epilogue warps
+  const int m_local = t % BN, g = t / BN;
+  const int m = tb * BN + m_local;
+#pragma unroll 1
+  for (int cc = 0; cc < COLS / 32; ++cc) {
+    const int nl0 = g * COLS + 32 * cc;
+    const int n0 = ta * BM + nl0;
+    if (n0 >= p.N) break;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = T[(nl0 + j) * TS + m_local];
+    epi_rows_chunk(p, v, m, n0, alpha);
+  }
+  named_bar_sync(2, 128);
 }
 
 // ------------------------------------------------------------------ kernel --
+
+template <bool SWAP, int BN>
+__host__ __device__ constexpr int t_tile_bytes() {
+  return SWAP ? BM * (BN + 4) * 4 : 0;
+}
+
+template <bool SWAP, int BN, int STAGES>
+__host__ __device__ constexpr int smem_total() {
+  return STAGES * (A_BYTES + BN * BK) + t_tile_bytes<SWAP, BN>() + 1024 + 256;
+}
 
 template <bool SWAP, int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -250,7 +259,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  float* T = reinterpret_cast<float*>(sB + STAGES * B_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES + t_tile_bytes<SWAP, BN>());
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -261,6 +271,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   volatile int* epi_ok = abort_flag + 2;  // [4], one per epilogue warp
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the next kernel in the stream may start its prologue now; it waits for
+  // this grid's completion before touching memory
+  pdl_trigger();
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -290,22 +303,47 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
+      // The packed weights are never written by an earlier kernel: the first
+      // unit's weight slices are requested before waiting on the producer
+      // kernel of the activations, so they stream in while it finishes.
+      const CUtensorMap* wmap = SWAP ? &tmA : &tmB;
+      const CUtensorMap* xmap = SWAP ? &tmB : &tmA;
+      const int u0 = blockIdx.x;
+      int n_pre = 0;
+      if (u0 < p.units) {
+        const int tile = u0 / p.splits, split = u0 % p.splits;
+        const int ta = tile % p.a_tiles, tb = tile / p.a_tiles;
+        const int kb0 = int(long(split) * p.k_blocks / p.splits);
+        const int kb1 = int(long(split + 1) * p.k_blocks / p.splits);
+        n_pre = kb1 - kb0 < STAGES ? kb1 - kb0 : STAGES;
+        for (int i = 0; i < n_pre; ++i) {
+          mbar_arrive_expect_tx(&full[i], A_BYTES + B_BYTES);
+          if (SWAP) tma_load_2d(sA + i * A_BYTES, wmap, &full[i], (kb0 + i) * BK, ta * BM);
+          else tma_load_2d(sB + i * B_BYTES, wmap, &full[i], (kb0 + i) * BK, tb * BN);
+        }
+      }
+      pdl_wait();
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+      for (int u = u0; u < p.units && ok; u += gridDim.x) {
         const int tile = u / p.splits, split = u % p.splits;
         const int ta = tile % p.a_tiles, tb = tile / p.a_tiles;
         const int kb0 = int(long(split) * p.k_blocks / p.splits);
         const int kb1 = int(long(split + 1) * p.k_blocks / p.splits);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitNs, abort_flag)) {
-            ok = false;
-            break;
+          const bool pre = (u == u0) && (kb - kb0 < n_pre);
+          if (!pre) {
+            if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitNs, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES);
+            if (SWAP) tma_load_2d(sA + stage * A_BYTES, wmap, &full[stage], kb * BK, ta * BM);
+            else tma_load_2d(sB + stage * B_BYTES, wmap, &full[stage], kb * BK, tb * BN);
           }
-          mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES);
-          tma_load_2d(sA + stage * A_BYTES, &tmA, &full[stage], kb * BK, ta * BM);
-          tma_load_2d(sB + stage * B_BYTES, &tmB, &full[stage], kb * BK, tb * BN);
+          if (SWAP) tma_load_2d(sB + stage * B_BYTES, xmap, &full[stage], kb * BK, tb * BN);
+          else tma_load_2d(sA + stage * A_BYTES, xmap, &full[stage], kb * BK, ta * BM);
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -362,6 +400,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     }
   } else {
     // ----------------------------------------------------------- epilogue --
+    pdl_wait();
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
     int local = 0;
@@ -385,12 +424,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + uint32_t(ab * BN) + (uint32_t(32 * q) << 16);
-      if (p.splits == 1) {
-        tile_epilogue<SWAP, BN>(p, ta, tb, q, lane, alpha,
-                                [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); });
+      auto release_tmem = [&]() {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[ab]);
+      };
+      if (p.splits == 1) {
+        tile_epilogue<SWAP, BN>(
+            p, ta, tb, q, lane, alpha, T,
+            [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); }, release_tmem);
       } else {
         // spill this split's fp32 partial: row (lane of TMEM) major
         const int row = 32 * q + lane;
@@ -404,9 +446,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           for (int k = 0; k < 8; ++k)
             d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[ab]);
+        release_tmem();
         __threadfence();
         named_bar_sync(1, 128);
         if (threadIdx.x == 64) {
@@ -417,21 +457,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         if (*last_flag) {
           __threadfence();
           const float* base = p.partials + long(tile) * p.splits * (BM * BN) + long(row) * BN;
-          tile_epilogue<SWAP, BN>(p, ta, tb, q, lane, alpha, [&](int c, float (&v)[32]) {
+          tile_epilogue<SWAP, BN>(
+              p, ta, tb, q, lane, alpha, T,
+              [&](int c, float (&v)[32]) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-            for (int s = 0; s < p.splits; ++s) {
-              const float4* src = reinterpret_cast<const float4*>(base + long(s) * (BM * BN) + 32 * c);
+                for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+                for (int s = 0; s < p.splits; ++s) {
+                  const float4* src =
+                      reinterpret_cast<const float4*>(base + long(s) * (BM * BN) + 32 * c);
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const float4 f = __ldcg(src + k);
-                v[4 * k] = __fadd_rn(v[4 * k], f.x);
-                v[4 * k + 1] = __fadd_rn(v[4 * k + 1], f.y);
-                v[4 * k + 2] = __fadd_rn(v[4 * k + 2], f.z);
-                v[4 * k + 3] = __fadd_rn(v[4 * k + 3], f.w);
-              }
-            }
-          });
+                  for (int k = 0; k < 8; ++k) {
+                    const float4 f = __ldcg(src + k);
+                    v[4 * k] = __fadd_rn(v[4 * k], f.x);
+                    v[4 * k + 1] = __fadd_rn(v[4 * k + 1], f.y);
+                    v[4 * k + 2] = __fadd_rn(v[4 * k + 2], f.z);
+                    v[4 * k + 3] = __fadd_rn(v[4 * k + 3], f.w);
+                  }
+                }
+              },
+              [] {});
           if (threadIdx.x == 64) p.counters[tile] = 0u;
         }
         named_bar_sync(1, 128);
@@ -520,7 +564,7 @@ Plan make_plan(int M, int N, int K, int epi) {
 template <bool SWAP, int BN, int STAGES>
 int launch_t(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
              cudaStream_t s) {
-  constexpr int smem = smem_bytes<BN, STAGES>();
+  constexpr int smem = smem_total<SWAP, BN, STAGES>();
   static_assert(smem <= 232448, "shared memory budget");
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -531,8 +575,8 @@ int launch_t(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const
       return fail(FRT_ECUDA, "cudaFuncSetAttribute(max dynamic smem %d)", smem);
     attr_set[dev] = true;
   }
-  gemm_kernel<SWAP, BN, STAGES><<<pl.grid, kThreads, smem, s>>>(ta, tb, p);
-  return check_launch("gemm_kernel");
+  return launch_pdl("gemm_kernel", gemm_kernel<SWAP, BN, STAGES>, dim3(pl.grid), dim3(kThreads),
+                    size_t(smem), s, ta, tb, p);
 }
 
 int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void* workspace,
@@ -562,8 +606,8 @@ int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void
   if (!pl.swap && pl.bn == 256) return launch_t<false, 256, 4>(pl, ta, tb, p, s);
   if (!pl.swap) return launch_t<false, 128, 6>(pl, ta, tb, p, s);
   if (pl.bn == 32) return launch_t<true, 32, 8>(pl, ta, tb, p, s);
-  if (pl.bn == 64) return launch_t<true, 64, 8>(pl, ta, tb, p, s);
-  return launch_t<true, 128, 6>(pl, ta, tb, p, s);
+  if (pl.bn == 64) return launch_t<true, 64, 7>(pl, ta, tb, p, s);
+  return launch_t<true, 128, 4>(pl, ta, tb, p, s);
 }
 
 int validate_common(int M, int N, int K, const void* x8, const void* w8, const float* act_scale,
@@ -598,6 +642,7 @@ extern "C" int frt_packed_fp8_gemm(int M, int N, int K, const frt_e4m3* x8, cons
   FRT_REQUIRE(epilogue == FRT_EPI_BF16 || epilogue == FRT_EPI_GEGLU_E4M3, FRT_EINVAL,
               "unknown epilogue %d", epilogue);
   FRT_REQUIRE(out, FRT_EINVAL, "out is required");
+  FRT_REQUIRE(!bias || aligned(bias, 16), FRT_EALIGN, "bias must be 16-byte aligned");
   FRT_REQUIRE(aligned(out, 16), FRT_EALIGN, "out must be 16-byte aligned");
   if (epilogue == FRT_EPI_BF16) {
     FRT_REQUIRE(ldo >= N && ldo % 8 == 0, FRT_EALIGN, "ldo must be >= N and a multiple of 8");
@@ -638,6 +683,7 @@ extern "C" int frt_packed_fp8_gemm_rope_kvcache(
   if (rc) return rc;
   FRT_REQUIRE(rope && k_cache && v_cache && (q_out || hq == 0), FRT_EINVAL,
               "rope, q_out, k_cache and v_cache are required");
+  FRT_REQUIRE(!bias || aligned(bias, 16), FRT_EALIGN, "bias must be 16-byte aligned");
   FRT_REQUIRE(aligned(rope, 16) && aligned(k_cache, 16) && aligned(v_cache, 16) &&
                   (!q_out || aligned(q_out, 16)),
               FRT_EALIGN, "rope, q_out and the caches must be 16-byte aligned");

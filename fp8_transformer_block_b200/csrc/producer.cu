@@ -12,19 +12,24 @@
 // Layout: a group of G threads (G a multiple of 32) owns one row; each thread
 // holds VPT chunks of 8 bf16 (16-byte loads) in registers, so every input
 // byte is read once and every output byte written once (HBM-bound: 7*D bytes
-// per row in both forms).  G == 32 packs 4 rows per 128-thread block; larger
-// G uses one row per block and a shared-memory cross-warp reduction.
+// per row for the table form, 9*D with the gate output for AdaRMS).  All of a
+// row's streamed inputs are loaded before the row reduction so they are in
+// flight together.  Few rows (the latency regime) spread a row over more
+// threads (VPT = 1); many rows use VPT = 4.  G == 32 packs 4 rows per block;
+// larger G uses one row per block and a shared-memory cross-warp reduction.
 // Arithmetic is fp32 with explicitly rounded operations (no contraction into
 // FMA), IEEE division and square root, so the only difference from a
 // sequential evaluation is the order of the row sums.
+// Launched with programmatic dependent launch; blocks past the row blocks
+// (when the chain passes a prefix) copy the cache prefix in the same grid.
 
-#include "frt_common.cuh"
+#include "frt_internal.cuh"
 
 namespace frt {
 namespace {
 
 struct ProducerArgs {
-  int rows, D, C, G;
+  int rows, D, C, G, row_blocks;
   float eps;
   uint16_t* res;
   const uint16_t* delta;
@@ -42,6 +47,7 @@ struct ProducerArgs {
   uint8_t* x8;
   uint16_t* gate_out;
   float* amax;
+  PrefixArgs pre;  // pre.units == 0: no prefix blocks
 };
 
 __device__ __forceinline__ uint4 ldg16(const uint16_t* p) {
@@ -61,9 +67,22 @@ __device__ __forceinline__ float row_sum(float v, int G, float* red) {
   return s;
 }
 
+// Blocks past the row blocks copy the prefix (grid-stride over its units).
+__device__ __forceinline__ bool prefix_block(const ProducerArgs& a) {
+  if (int(blockIdx.x) < a.row_blocks) return false;
+  const long nb = long(gridDim.x) - a.row_blocks;
+  for (long u = (long(blockIdx.x) - a.row_blocks) * blockDim.x + threadIdx.x; u < a.pre.units;
+       u += nb * blockDim.x)
+    prefix_unit(a.pre, u);
+  return true;
+}
+
 template <int VPT>
 __global__ void __launch_bounds__(512) adarms_kernel(ProducerArgs a) {
   __shared__ float red[16];
+  pdl_trigger();
+  pdl_wait();
+  if (prefix_block(a)) return;
   const int G = a.G;
   const int rpb = blockDim.x / G;
   const int t = threadIdx.x % G;
@@ -78,15 +97,24 @@ __global__ void __launch_bounds__(512) adarms_kernel(ProducerArgs a) {
     uint16_t* rr = a.res + r * D;
     const uint16_t* dd = a.delta + r * D;
     const uint16_t* gg = a.gate + r * a.gate_stride;
+    uint4 rv4[VPT], dv4[VPT], gv4[VPT];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int c = t + i * G;
       if (c < C) {
-        float rv[8], dv[8], gv[8];
-        unpack8(*reinterpret_cast<const uint4*>(rr + 8 * c), rv);
-        unpack8(ldg16(dd + 8 * c), dv);
-        unpack8(ldg16(gg + 8 * c), gv);
-        float h[8];
+        rv4[i] = *reinterpret_cast<const uint4*>(rr + 8 * c);
+        dv4[i] = ldg16(dd + 8 * c);
+        gv4[i] = ldg16(gg + 8 * c);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = t + i * G;
+      if (c < C) {
+        float rv[8], dv[8], gv[8], h[8];
+        unpack8(rv4[i], rv);
+        unpack8(dv4[i], dv);
+        unpack8(gv4[i], gv);
 #pragma unroll
         for (int j = 0; j < 8; ++j) h[j] = __fadd_rn(rv[j], __fmul_rn(gv[j], dv[j]));
         const uint4 hb = pack8_bf16(h);
@@ -140,6 +168,9 @@ __global__ void __launch_bounds__(512) adarms_kernel(ProducerArgs a) {
 template <int VPT>
 __global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
   __shared__ float red[16];
+  pdl_trigger();
+  pdl_wait();
+  if (prefix_block(a)) return;
   const int G = a.G;
   const int rpb = blockDim.x / G;
   const int t = threadIdx.x % G;
@@ -149,14 +180,28 @@ __global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
   const int D = a.D, C = a.C;
 
   float xv[VPT][8];
+  uint4 esh4[VPT], esc4[VPT];
   float sum = 0.0f;
   if (ok) {
     const uint16_t* xr = a.x + r * D;
+    const uint16_t* tr = a.temb + r * long(a.chunks) * D;
+    const uint16_t* tsh = tr + long(a.shift_idx) * D;
+    const uint16_t* tsc = tr + long(a.scale_idx) * D;
+    uint4 xv4[VPT];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int c = t + i * G;
       if (c < C) {
-        unpack8(ldg16(xr + 8 * c), xv[i]);
+        xv4[i] = ldg16(xr + 8 * c);
+        esh4[i] = ldg16(tsh + 8 * c);
+        esc4[i] = ldg16(tsc + 8 * c);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = t + i * G;
+      if (c < C) {
+        unpack8(xv4[i], xv[i]);
 #pragma unroll
         for (int j = 0; j < 8; ++j) sum = __fadd_rn(sum, xv[i][j]);
       }
@@ -183,9 +228,6 @@ __global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
   const float var = __fdiv_rn(sq, float(D));
   const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
   const float as = __ldg(a.act_scale);
-  const uint16_t* tr = a.temb + r * long(a.chunks) * D;
-  const uint16_t* tsh = tr + long(a.shift_idx) * D;
-  const uint16_t* tsc = tr + long(a.scale_idx) * D;
   const float* bsh = a.table + long(a.shift_idx) * D;
   const float* bsc = a.table + long(a.scale_idx) * D;
   float mx = 0.0f;
@@ -194,8 +236,8 @@ __global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
     const int c = t + i * G;
     if (c < C) {
       float esh[8], esc[8];
-      unpack8(ldg16(tsh + 8 * c), esh);
-      unpack8(ldg16(tsc + 8 * c), esc);
+      unpack8(esh4[i], esh);
+      unpack8(esc4[i], esc);
       const float4 s0 = __ldg(reinterpret_cast<const float4*>(bsh + 8 * c));
       const float4 s1 = __ldg(reinterpret_cast<const float4*>(bsh + 8 * c + 4));
       const float4 c0 = __ldg(reinterpret_cast<const float4*>(bsc + 8 * c));
@@ -223,21 +265,15 @@ __global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
 }
 
 }  // namespace
-}  // namespace frt
 
-using frt::ProducerArgs;
-
-extern "C" int frt_ada_norm_quant_fp8(
-    int mode, int rows, int D, float eps, frt_bf16* res, const frt_bf16* delta,
-    const frt_bf16* prev_gate, long gate_row_stride, const frt_bf16* weight,
-    const frt_bf16* style, long style_row_stride, const frt_bf16* x,
-    const frt_bf16* temb, int chunks, const float* table, int shift_idx,
-    int scale_idx, const float* act_scale, frt_e4m3* x8_out, frt_bf16* gate_out,
-    float* amax_out, void* stream) {
-  using frt::aligned;
-  frt::clear_error();
-  FRT_REQUIRE(mode == FRT_NORM_ADARMS || mode == FRT_NORM_LAYERNORM_TABLE,
-              FRT_EINVAL, "mode %d is not FRT_NORM_ADARMS or FRT_NORM_LAYERNORM_TABLE", mode);
+int producer_call(int mode, int rows, int D, float eps, uint16_t* res, const uint16_t* delta,
+                  const uint16_t* prev_gate, long gate_row_stride, const uint16_t* weight,
+                  const uint16_t* style, long style_row_stride, const uint16_t* x,
+                  const uint16_t* temb, int chunks, const float* table, int shift_idx,
+                  int scale_idx, const float* act_scale, uint8_t* x8_out, uint16_t* gate_out,
+                  float* amax_out, const PrefixArgs* pre, cudaStream_t s) {
+  FRT_REQUIRE(mode == FRT_NORM_ADARMS || mode == FRT_NORM_LAYERNORM_TABLE, FRT_EINVAL,
+              "mode %d is not FRT_NORM_ADARMS or FRT_NORM_LAYERNORM_TABLE", mode);
   FRT_REQUIRE(rows >= 0, FRT_ESHAPE, "rows must be >= 0, got %d", rows);
   FRT_REQUIRE(D >= 8 && D <= 16384 && D % 8 == 0, FRT_ESHAPE,
               "D must be a multiple of 8 in [8, 16384], got %d", D);
@@ -252,8 +288,8 @@ extern "C" int frt_ada_norm_quant_fp8(
                     aligned(style, 16) && (!weight || aligned(weight, 16)) &&
                     (!gate_out || aligned(gate_out, 16)),
                 FRT_EALIGN, "bf16 tensors must be 16-byte aligned");
-    FRT_REQUIRE(gate_row_stride >= 0 && gate_row_stride % 8 == 0 &&
-                    style_row_stride >= 0 && style_row_stride % 8 == 0,
+    FRT_REQUIRE(gate_row_stride >= 0 && gate_row_stride % 8 == 0 && style_row_stride >= 0 &&
+                    style_row_stride % 8 == 0,
                 FRT_EALIGN, "row strides must be non-negative multiples of 8");
     FRT_REQUIRE(gate_row_stride == 0 || gate_row_stride >= D, FRT_ESHAPE,
                 "gate_row_stride must be 0 or >= D");
@@ -268,7 +304,8 @@ extern "C" int frt_ada_norm_quant_fp8(
                 "x, temb and table must be 16-byte aligned");
   }
   FRT_REQUIRE(!amax_out || aligned(amax_out, 4), FRT_EALIGN, "amax_out must be 4-byte aligned");
-  if (rows == 0) return FRT_OK;
+  const long pre_units = pre ? pre->units : 0;
+  if (rows == 0 && pre_units == 0) return FRT_OK;
 
   ProducerArgs a{};
   a.rows = rows; a.D = D; a.C = D / 8; a.eps = eps;
@@ -277,26 +314,56 @@ extern "C" int frt_ada_norm_quant_fp8(
   a.x = x; a.temb = temb; a.chunks = chunks; a.table = table;
   a.shift_idx = shift_idx; a.scale_idx = scale_idx;
   a.act_scale = act_scale; a.x8 = x8_out; a.gate_out = gate_out; a.amax = amax_out;
+  if (pre) a.pre = *pre;
   int vpt;
-  if (a.C <= 128) { a.G = 32; vpt = (a.C + 31) / 32; }
-  else { vpt = 4; a.G = ((a.C + 127) / 128) * 32; }
+  const int sms = num_sms();
+  if (rows <= 2 * sms) {  // latency regime: many threads per row
+    vpt = a.C <= 512 ? 1 : a.C <= 1024 ? 2 : 4;
+    a.G = ((a.C + vpt - 1) / vpt + 31) / 32 * 32;
+  } else if (a.C <= 128) {
+    a.G = 32;
+    vpt = (a.C + 31) / 32;
+  } else {
+    vpt = 4;
+    a.G = ((a.C + 127) / 128) * 32;
+  }
   const int rpb = a.G == 32 ? 4 : 1;
-  const dim3 block(a.G * rpb), grid((rows + rpb - 1) / rpb);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  a.row_blocks = (rows + rpb - 1) / rpb;
+  const int block = a.G * rpb;
+  int pre_blocks = 0;
+  if (pre_units > 0) {
+    const long need = (pre_units + block - 1) / block;
+    pre_blocks = int(need < 2L * sms ? need : 2L * sms);
+  }
+  const dim3 grid(a.row_blocks + pre_blocks);
   if (mode == FRT_NORM_ADARMS) {
     switch (vpt) {
-      case 1: frt::adarms_kernel<1><<<grid, block, 0, s>>>(a); break;
-      case 2: frt::adarms_kernel<2><<<grid, block, 0, s>>>(a); break;
-      case 3: frt::adarms_kernel<3><<<grid, block, 0, s>>>(a); break;
-      default: frt::adarms_kernel<4><<<grid, block, 0, s>>>(a); break;
-    }
-  } else {
-    switch (vpt) {
-      case 1: frt::ln_table_kernel<1><<<grid, block, 0, s>>>(a); break;
-      case 2: frt::ln_table_kernel<2><<<grid, block, 0, s>>>(a); break;
-      case 3: frt::ln_table_kernel<3><<<grid, block, 0, s>>>(a); break;
-      default: frt::ln_table_kernel<4><<<grid, block, 0, s>>>(a); break;
+      case 1: return launch_pdl("adarms_kernel", adarms_kernel<1>, grid, block, 0, s, a);
+      case 2: return launch_pdl("adarms_kernel", adarms_kernel<2>, grid, block, 0, s, a);
+      case 3: return launch_pdl("adarms_kernel", adarms_kernel<3>, grid, block, 0, s, a);
+      default: return launch_pdl("adarms_kernel", adarms_kernel<4>, grid, block, 0, s, a);
     }
   }
-  return frt::check_launch("frt_ada_norm_quant_fp8");
+  switch (vpt) {
+    case 1: return launch_pdl("ln_table_kernel", ln_table_kernel<1>, grid, block, 0, s, a);
+    case 2: return launch_pdl("ln_table_kernel", ln_table_kernel<2>, grid, block, 0, s, a);
+    case 3: return launch_pdl("ln_table_kernel", ln_table_kernel<3>, grid, block, 0, s, a);
+    default: return launch_pdl("ln_table_kernel", ln_table_kernel<4>, grid, block, 0, s, a);
+  }
+}
+
+}  // namespace frt
+
+extern "C" int frt_ada_norm_quant_fp8(
+    int mode, int rows, int D, float eps, frt_bf16* res, const frt_bf16* delta,
+    const frt_bf16* prev_gate, long gate_row_stride, const frt_bf16* weight,
+    const frt_bf16* style, long style_row_stride, const frt_bf16* x,
+    const frt_bf16* temb, int chunks, const float* table, int shift_idx,
+    int scale_idx, const float* act_scale, frt_e4m3* x8_out, frt_bf16* gate_out,
+    float* amax_out, void* stream) {
+  frt::clear_error();
+  return frt::producer_call(mode, rows, D, eps, res, delta, prev_gate, gate_row_stride, weight,
+                            style, style_row_stride, x, temb, chunks, table, shift_idx,
+                            scale_idx, act_scale, x8_out, gate_out, amax_out, nullptr,
+                            static_cast<cudaStream_t>(stream));
 }

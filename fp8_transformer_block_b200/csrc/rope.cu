@@ -10,7 +10,7 @@
 //
 // All three are HBM-bound streams: 16-byte loads and stores, one 8-element
 // chunk per thread step, grid-stride loops sized to the SM count.
-#include "frt_common.cuh"
+#include "frt_internal.cuh"
 
 namespace frt {
 namespace {
@@ -37,11 +37,8 @@ struct SplitArgs {
   uint16_t* q_out;
   uint16_t* k_cache;
   uint16_t* v_cache;
-  // prefix
-  int Pcopy, T_src, interleave;
-  const uint16_t* pk;
-  const uint16_t* pv;
-  long suffix_units, prefix_units;
+  long suffix_units;
+  PrefixArgs pre;  // pre.units == 0: no prefix copy
 };
 
 // Rotate 4 adjacent pairs of x (8 bf16) with 4 (cos, sin) pairs of r.
@@ -62,7 +59,9 @@ __global__ void split_rope_kernel(SplitArgs a) {
   const int hd8 = a.hd / 8;
   const int heads = a.hq + 2 * a.hkv;
   const long N8 = long(heads) * hd8;
-  const long total = a.suffix_units + a.prefix_units;
+  const long total = a.suffix_units + a.pre.units;
+  pdl_trigger();
+  pdl_wait();
   for (long g = blockIdx.x * long(blockDim.x) + threadIdx.x; g < total;
        g += long(gridDim.x) * blockDim.x) {
     if (g < a.suffix_units) {
@@ -83,47 +82,17 @@ __global__ void split_rope_kernel(SplitArgs a) {
         *reinterpret_cast<uint4*>(a.v_cache + ((long(b) * a.T + a.P + s) * a.hkv + hv) * a.hd + d0) = xv;
       }
     } else {
-      // prefix unit: (b, p, h, chunk, which) with which = 0 key, 1 value
-      long u = g - a.suffix_units;
-      const int which = int(u & 1);
-      u >>= 1;
-      const int c = int(u % hd8);
-      u /= hd8;
-      const int h = int(u % a.hkv);
-      u /= a.hkv;
-      const int p = int(u % a.Pcopy);
-      const int b = int(u / a.Pcopy);
-      const long src_row = ((long(b) * a.hkv + h) * a.T_src + p) * a.hd;
-      const long dst = ((long(b) * a.T + p) * a.hkv + h) * a.hd + 8 * c;
-      if (which == 1 || !a.interleave) {
-        const uint16_t* src = (which ? a.pv : a.pk) + src_row + 8 * c;
-        uint16_t* d = (which ? a.v_cache : a.k_cache) + dst;
-        *reinterpret_cast<uint4*>(d) = __ldg(reinterpret_cast<const uint4*>(src));
-      } else {
-        // destination d0..d0+7 (d0 = 8c) takes sources 4c..4c+3 at even
-        // slots and hd/2 + 4c .. +3 at odd slots
-        const uint2 lo = __ldg(reinterpret_cast<const uint2*>(a.pk + src_row + 4 * c));
-        const uint2 hi = __ldg(reinterpret_cast<const uint2*>(a.pk + src_row + a.hd / 2 + 4 * c));
-        const uint32_t l[2] = {lo.x, lo.y}, m[2] = {hi.x, hi.y};
-        uint32_t o[4];
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          o[2 * k] = (l[k] & 0xFFFFu) | (m[k] << 16);
-          o[2 * k + 1] = (l[k] >> 16) | (m[k] & 0xFFFF0000u);
-        }
-        *reinterpret_cast<uint4*>(a.k_cache + dst) = make_uint4(o[0], o[1], o[2], o[3]);
-      }
+      prefix_unit(a.pre, g - a.suffix_units);
     }
   }
 }
 
 int launch_split(const SplitArgs& a, cudaStream_t s) {
-  const long total = a.suffix_units + a.prefix_units;
+  const long total = a.suffix_units + a.pre.units;
   if (total == 0) return FRT_OK;
   const long blocks_needed = (total + 255) / 256;
   const int grid = int(blocks_needed < num_sms() * 16L ? blocks_needed : num_sms() * 16L);
-  split_rope_kernel<<<grid, 256, 0, s>>>(a);
-  return check_launch("split_rope_kernel");
+  return launch_pdl("split_rope_kernel", split_rope_kernel, dim3(grid), dim3(256), 0, s, a);
 }
 
 }  // namespace
@@ -144,16 +113,27 @@ extern "C" int frt_build_rope_table(int M, int hd, int P, double theta, frt_bf16
   return frt::check_launch("frt_build_rope_table");
 }
 
-static int validate_prefix(int B, int hkv, int hd, int P, int T, int T_src, const void* pk,
-                           const void* pv) {
-  using frt::aligned;
+namespace frt {
+
+int prefix_args(int B, int hkv, int hd, int P, int T, int T_src, const uint16_t* pk,
+                const uint16_t* pv, int interleave, uint16_t* k_cache, uint16_t* v_cache,
+                PrefixArgs* a) {
+  FRT_REQUIRE(B >= 0 && hkv >= 1, FRT_ESHAPE, "bad B/hkv");
+  FRT_REQUIRE(hd >= 8 && hd % 8 == 0, FRT_ESHAPE, "hd must be a multiple of 8, got %d", hd);
   FRT_REQUIRE(pk && pv, FRT_EINVAL, "prefix_k and prefix_v are both required");
+  FRT_REQUIRE(k_cache && v_cache, FRT_EINVAL, "k_cache and v_cache are required");
   FRT_REQUIRE(P >= 0 && P <= T && P <= T_src, FRT_ERANGE,
               "prefix rows P=%d must fit the cache (T=%d) and the source (T_src=%d)", P, T, T_src);
-  FRT_REQUIRE(aligned(pk, 16) && aligned(pv, 16), FRT_EALIGN, "prefix tensors must be 16-byte aligned");
-  (void)B; (void)hkv; (void)hd;
+  FRT_REQUIRE(aligned(pk, 16) && aligned(pv, 16) && aligned(k_cache, 16) && aligned(v_cache, 16),
+              FRT_EALIGN, "prefix tensors and caches must be 16-byte aligned");
+  a->B = B; a->hkv = hkv; a->hd = hd; a->P = P; a->T = T; a->T_src = T_src;
+  a->interleave = interleave != 0;
+  a->pk = pk; a->pv = pv; a->k_cache = k_cache; a->v_cache = v_cache;
+  a->units = 2L * B * P * hkv * (hd / 8);
   return FRT_OK;
 }
+
+}  // namespace frt
 
 extern "C" int frt_split_rope_kvcache(int B, int M, int hq, int hkv, int hd, int P, int T,
                                       const frt_bf16* qkv, const frt_bf16* rope, frt_bf16* q_out,
@@ -178,11 +158,9 @@ extern "C" int frt_split_rope_kvcache(int B, int M, int hq, int hkv, int hd, int
   a.qkv = qkv; a.rope = rope; a.q_out = q_out; a.k_cache = k_cache; a.v_cache = v_cache;
   a.suffix_units = long(B) * M * (hq + 2 * hkv) * (hd / 8);
   if (prefix_k) {
-    int rc = validate_prefix(B, hkv, hd, P, T, prefix_T_src, prefix_k, prefix_v);
+    int rc = frt::prefix_args(B, hkv, hd, P, T, prefix_T_src, prefix_k, prefix_v,
+                              prefix_interleave, k_cache, v_cache, &a.pre);
     if (rc) return rc;
-    a.Pcopy = P; a.T_src = prefix_T_src; a.interleave = prefix_interleave != 0;
-    a.pk = prefix_k; a.pv = prefix_v;
-    a.prefix_units = 2L * B * P * hkv * (hd / 8);
   }
   return frt::launch_split(a, static_cast<cudaStream_t>(stream));
 }
@@ -190,19 +168,11 @@ extern "C" int frt_split_rope_kvcache(int B, int M, int hq, int hkv, int hd, int
 extern "C" int frt_prefix_copy_kv(int B, int hkv, int hd, int P, int T, int T_src,
                                   const frt_bf16* prefix_k, const frt_bf16* prefix_v, int interleave,
                                   frt_bf16* k_cache, frt_bf16* v_cache, void* stream) {
-  using frt::aligned;
   frt::clear_error();
-  FRT_REQUIRE(B >= 0 && hkv >= 1, FRT_ESHAPE, "bad B/hkv");
-  FRT_REQUIRE(hd >= 8 && hd % 8 == 0, FRT_ESHAPE, "hd must be a multiple of 8, got %d", hd);
-  FRT_REQUIRE(k_cache && v_cache, FRT_EINVAL, "k_cache and v_cache are required");
-  FRT_REQUIRE(aligned(k_cache, 16) && aligned(v_cache, 16), FRT_EALIGN, "caches must be 16-byte aligned");
-  int rc = validate_prefix(B, hkv, hd, P, T, T_src, prefix_k, prefix_v);
-  if (rc) return rc;
   frt::SplitArgs a{};
-  a.B = B; a.M = 1; a.hq = 0; a.hkv = hkv; a.hd = hd; a.P = P; a.T = T;
-  a.k_cache = k_cache; a.v_cache = v_cache;
-  a.Pcopy = P; a.T_src = T_src; a.interleave = interleave != 0;
-  a.pk = prefix_k; a.pv = prefix_v;
-  a.prefix_units = 2L * B * P * hkv * (hd / 8);
+  int rc = frt::prefix_args(B, hkv, hd, P, T, T_src, prefix_k, prefix_v, interleave, k_cache,
+                            v_cache, &a.pre);
+  if (rc) return rc;
+  a.hkv = hkv; a.hd = hd;
   return frt::launch_split(a, static_cast<cudaStream_t>(stream));
 }

@@ -1,0 +1,299 @@
+"""GPU parity of the whole chain (frt_chain_layer and the MLP sequence)
+against the oracle's chain run on the same seeded inputs.
+
+The oracle runs the chain from the same inputs on its own (its x8 is its
+own), so end-to-end outputs carry the rare one-step code flips of the
+producer through the GEMM: they are held to max|err| <= 2e-2 * rms(ref);
+the producer's codes are held to the 99.99 % bar.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from fp8_transformer_block_b200 import synth
+from fp8_transformer_block_b200.synth import bf16_value
+from parity import assert_codes, assert_rms, e4m3_step_distance
+from chain_cases import SENTINEL, calibrate_adarms, calibrate_dit
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rt():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from fp8_transformer_block_b200 import build
+    build.build()
+    from fp8_transformer_block_b200 import frt, runtime
+    return frt, runtime, torch
+
+
+def _sentinel_cache(torch, B, T, hkv, hd):
+    t = torch.full((B, T, hkv, hd), SENTINEL, dtype=torch.int16, device="cuda")
+    return t.view(torch.bfloat16)
+
+
+def _oracle_layer(w, inp, a, pk_ref, prefix, style=None):
+    """Oracle chain layer: producer -> GEMM -> split/RoPE/KV (+ prefix)."""
+    st = inp["style"] if style is None else style
+    pr = oracle.ada_rms_norm_quant(inp["res"], inp["delta"], inp["prev_gate"],
+                                   st, a, eps=w.eps)
+    qkv = oracle.fp8_gemm(pr["x8"], pk_ref["w8"], a, pk_ref["w_scale"],
+                          pk_ref["bias"] if w.bias else None)
+    kc = np.full((w.B, w.T, w.hkv, w.hd), SENTINEL, np.uint16)
+    vc = kc.copy()
+    if prefix is not None:
+        kc, vc = oracle.prefix_copy(prefix[0], prefix[1], w.P, kc, vc, True)
+    q, kc, vc = oracle.split_rope_kvcache(
+        qkv, oracle.rope_table(w.M, w.hd, w.P, w.theta), w.B, w.M, w.hq,
+        w.hkv, w.hd, w.P, kc, vc)
+    return pr, q, kc, vc
+
+
+@pytest.mark.parametrize("name", ["tiny_adarms", "vla_action_expert"])
+@pytest.mark.parametrize("fused", [True, False])
+def test_chain_layer_adarms(rt, name, fused):
+    frt, runtime, torch = rt
+    w = synth.WORKLOADS[name]
+    inp = synth.adarms_inputs(w.rows, w.D, w.seed, outliers=w.outliers)
+    a = calibrate_adarms(w)
+    ws, _ = synth.qkv_weights(w.hq, w.hkv, w.hd, w.D, w.seed)
+    pk_ref = oracle.pack_weights_fp8(ws, layout=1, hd=w.hd)
+    prefix = None
+    if w.P > 0:
+        prefix = synth.prefix_cache(w.B, w.hkv, 1024, w.hd, w.seed)
+    pr, qr, kr, vr = _oracle_layer(w, inp, a, pk_ref, prefix)
+
+    pk = runtime.pack(ws, layout=frt.FRT_PACK_QK_INTERLEAVE, hd=w.hd)
+    rope = runtime.empty_bf16(w.M, w.hd)
+    frt.frt_build_rope_table(w.M, w.hd, w.P, w.theta, rope)
+    res = runtime.bf16_dev(inp["res"])
+    x8 = runtime.empty_u8(w.rows, w.D)
+    gate_out = runtime.empty_bf16(w.rows, w.D)
+    q = runtime.empty_bf16(w.B, w.M, w.hq, w.hd)
+    kc = _sentinel_cache(torch, w.B, w.T, w.hkv, w.hd)
+    vc = _sentinel_cache(torch, w.B, w.T, w.hkv, w.hd)
+    qkv = runtime.empty_bf16(w.rows, w.N) if not fused else None
+    d = runtime.chain_desc(
+        B=w.B, M=w.M, D=w.D, hq=w.hq, hkv=w.hkv, hd=w.hd, P=w.P, T=w.T,
+        eps=w.eps, norm_mode=frt.FRT_NORM_ADARMS,
+        flags=frt.FRT_CHAIN_FUSED_ROPE if fused else frt.FRT_CHAIN_UNFUSED,
+        res=res, delta=runtime.bf16_dev(inp["delta"]),
+        prev_gate=runtime.bf16_dev(inp["prev_gate"]), gate_row_stride=0,
+        style=runtime.bf16_dev(inp["style"]), style_row_stride=0,
+        gate_out=gate_out, act_scale=runtime.scale_dev(a), x8=x8, w8=pk.w8,
+        w_scale=pk.w_scale, rope=rope, q_out=q, k_cache=kc, v_cache=vc,
+        prefix_k=None if prefix is None else runtime.bf16_dev(prefix[0]),
+        prefix_v=None if prefix is None else runtime.bf16_dev(prefix[1]),
+        prefix_T_src=0 if prefix is None else 1024, prefix_interleave=1,
+        qkv=qkv)
+    wsb = frt.frt_chain_workspace_size(d)
+    wsp = runtime.workspace(wsb)
+    d.workspace, d.workspace_bytes = frt.ptr(wsp), wsb
+    frt.frt_chain_layer(d)
+    torch.cuda.synchronize()
+    assert frt.frt_device_status(True) == frt.FRT_OK
+    h = runtime.bf16_host
+    assert np.array_equal(h(res), pr["res"])
+    assert np.array_equal(h(gate_out), pr["gate_out"])
+    assert_codes(runtime.u8_host(x8), pr["x8"], what="x8")
+    assert_rms(h(q), qr, what="q_out")
+    sl = slice(w.P, w.P + w.M)
+    assert_rms(h(kc)[:, sl], kr[:, sl], what="k rows")
+    assert_rms(h(vc)[:, sl], vr[:, sl], what="v rows")
+    # prefix rows bit-exact, rows past the suffix untouched
+    assert np.array_equal(h(kc)[:, :w.P], kr[:, :w.P])
+    assert np.array_equal(h(vc)[:, :w.P], vr[:, :w.P])
+    assert np.array_equal(h(kc)[:, w.P + w.M:], kr[:, w.P + w.M:])
+    assert np.array_equal(h(vc)[:, w.P + w.M:], vr[:, w.P + w.M:])
+
+
+def test_chain_layer_video_dit_sampled(rt):
+    """Full-size video-DiT chain on the GPU; the oracle recomputes a seeded
+    sample of rows (rows are independent through the whole chain)."""
+    frt, runtime, torch = rt
+    w = synth.WORKLOADS["video_dit"]
+    inp = synth.dit_inputs(w.rows, w.D, w.seed)
+    a = calibrate_dit(w, inp["table"])
+    ws, bs = synth.qkv_weights(w.hq, w.hkv, w.hd, w.D, w.seed, bias=True)
+    pk = runtime.pack(ws, bs)
+    rope = runtime.empty_bf16(w.M, w.hd)
+    frt.frt_build_rope_table(w.M, w.hd, w.P, w.theta, rope)
+    x8 = runtime.empty_u8(w.rows, w.D)
+    q = runtime.empty_bf16(w.B, w.M, w.hq, w.hd)
+    kc = _sentinel_cache(torch, w.B, w.T, w.hkv, w.hd)
+    vc = _sentinel_cache(torch, w.B, w.T, w.hkv, w.hd)
+    d = runtime.chain_desc(
+        B=w.B, M=w.M, D=w.D, hq=w.hq, hkv=w.hkv, hd=w.hd, P=w.P, T=w.T,
+        eps=w.eps, norm_mode=frt.FRT_NORM_LAYERNORM_TABLE,
+        flags=frt.FRT_CHAIN_FUSED_ROPE, x=runtime.bf16_dev(inp["x"]),
+        temb=runtime.bf16_dev(inp["temb"]), chunks=6,
+        table=runtime.f32_dev(inp["table"]), shift_idx=0, scale_idx=1,
+        act_scale=runtime.scale_dev(a), x8=x8, w8=pk.w8, w_scale=pk.w_scale,
+        bias=pk.bias, rope=rope, q_out=q, k_cache=kc, v_cache=vc)
+    wsb = frt.frt_chain_workspace_size(d)
+    assert wsb == 0
+    frt.frt_chain_layer(d)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(3)
+    sel = np.unique(np.concatenate([[0, w.M - 1, w.M, w.rows - 1],
+                                    rng.choice(w.rows, 60, replace=False)]))
+    pr = oracle.ada_layer_norm_quant_table(inp["x"][sel], inp["temb"][sel],
+                                           inp["table"], 0, 1, a)
+    x8g = runtime.u8_host(x8)
+    assert_codes(x8g[sel], pr["x8"], what="x8 (sampled rows)")
+    pk_ref = oracle.pack_weights_fp8(ws, bs)
+    qkv = oracle.fp8_gemm(pr["x8"], pk_ref["w8"], a, pk_ref["w_scale"],
+                          pk_ref["bias"])
+    table = oracle.rope_table(w.M, w.hd, w.P)
+    h = runtime.bf16_host
+    qg, kg, vg = h(q), h(kc), h(vc)
+    got_q, got_k, got_v, ref_q, ref_k, ref_v = [], [], [], [], [], []
+    for i, r in enumerate(sel):
+        b, s = divmod(int(r), w.M)
+        one = np.zeros((1, 1, w.hkv, w.hd), np.uint16)
+        qo, ko, vo = oracle.split_rope_kvcache(qkv[i:i + 1], table[s:s + 1], 1,
+                                               1, w.hq, w.hkv, w.hd, 0, one,
+                                               one)
+        ref_q.append(qo.ravel()); ref_k.append(ko.ravel()); ref_v.append(vo.ravel())
+        got_q.append(qg[b, s].ravel()); got_k.append(kg[b, s].ravel())
+        got_v.append(vg[b, s].ravel())
+    assert_rms(np.stack(got_q), np.stack(ref_q), what="q_out")
+    assert_rms(np.stack(got_k), np.stack(ref_k), what="k cache")
+    assert_rms(np.stack(got_v), np.stack(ref_v), what="v cache")
+
+
+def test_chain_stack_residual_carried(rt):
+    """18 AdaRMS chain layers of the tiny shape, M=16 tokens behind an
+    816-token prefix, residual carried (layer l+1 takes layer l's q_out as
+    delta and its gate_out as gate); the oracle runs the same stack."""
+    frt, runtime, torch = rt
+    w = synth.WORKLOADS["adarms_stack18"].with_M(16)
+    L, D, rows = w.layers, w.D, w.rows
+    inp = synth.adarms_inputs(rows, D, w.seed)
+    cal = synth.adarms_inputs(rows, D, w.seed + synth.CAL_OFFSET)
+    lays = [synth.stack_layer_inputs(w, l) for l in range(L)]
+    packs = [oracle.pack_weights_fp8(li["w"], layout=1, hd=w.hd) for li in lays]
+    table = oracle.rope_table(w.M, w.hd, w.P)
+
+    def oracle_stack(res, scales=None):
+        out, delta, gate = [], np.zeros((rows, D), np.uint16), \
+            np.zeros((1, D), np.uint16)
+        amaxes = []
+        for l in range(L):
+            a = 1.0 if scales is None else scales[l]
+            if scales is None:
+                a = oracle.ada_rms_norm_quant(res, delta, gate, lays[l]["style"],
+                                              1.0)["amax"] / 448.0
+                amaxes.append(a)
+            pr = oracle.ada_rms_norm_quant(res, delta, gate, lays[l]["style"], a)
+            qkv = oracle.fp8_gemm(pr["x8"], packs[l]["w8"], a,
+                                  packs[l]["w_scale"])
+            kc = np.zeros((1, w.T, w.hkv, w.hd), np.uint16)
+            kc, vc = oracle.prefix_copy(lays[l]["prefix_k"], lays[l]["prefix_v"],
+                                        w.P, kc, kc, True)
+            q, kc, vc = oracle.split_rope_kvcache(qkv, table, 1, w.M, w.hq,
+                                                  w.hkv, w.hd, w.P, kc, vc)
+            out.append((pr["res"], pr["x8"], q, kc, vc))
+            res, delta, gate = pr["res"], q.reshape(rows, D), pr["gate_out"]
+        return out, amaxes
+
+    _, scales = oracle_stack(cal["res"])
+    ref, _ = oracle_stack(inp["res"], scales)
+
+    res = runtime.bf16_dev(inp["res"])
+    zero = torch.zeros(rows, D, dtype=torch.bfloat16, device="cuda")
+    x8 = runtime.empty_u8(rows, D)
+    q = [runtime.empty_bf16(1, w.M, w.hq, w.hd) for _ in range(2)]
+    g = [runtime.empty_bf16(rows, D) for _ in range(2)]
+    rope = runtime.empty_bf16(w.M, w.hd)
+    frt.frt_build_rope_table(w.M, w.hd, w.P, w.theta, rope)
+    keep = []
+    descs = []
+    for l in range(L):
+        pk = runtime.pack(lays[l]["w"], layout=frt.FRT_PACK_QK_INTERLEAVE,
+                          hd=w.hd)
+        kc = torch.zeros(1, w.T, w.hkv, w.hd, dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        pkd = runtime.bf16_dev(lays[l]["prefix_k"])
+        pvd = runtime.bf16_dev(lays[l]["prefix_v"])
+        sc = runtime.scale_dev(scales[l])
+        st = runtime.bf16_dev(lays[l]["style"])
+        keep += [pk, kc, vc, pkd, pvd, sc, st]
+        d = runtime.chain_desc(
+            B=1, M=w.M, D=D, hq=w.hq, hkv=w.hkv, hd=w.hd, P=w.P, T=w.T,
+            eps=w.eps, norm_mode=frt.FRT_NORM_ADARMS,
+            flags=frt.FRT_CHAIN_FUSED_ROPE, res=res,
+            delta=zero if l == 0 else q[(l - 1) % 2],
+            prev_gate=zero if l == 0 else g[(l - 1) % 2],
+            gate_row_stride=0 if l == 0 else D, style=st, gate_out=g[l % 2],
+            act_scale=sc, x8=x8, w8=pk.w8, w_scale=pk.w_scale, rope=rope,
+            q_out=q[l % 2], k_cache=kc, v_cache=vc, prefix_k=pkd,
+            prefix_v=pvd, prefix_T_src=w.P, prefix_interleave=1)
+        descs.append((d, kc, vc))
+    wsb = frt.frt_chain_workspace_size(descs[0][0])
+    wsp = runtime.workspace(wsb)
+    h = runtime.bf16_host
+    for l, (d, kc, vc) in enumerate(descs):
+        d.workspace, d.workspace_bytes = frt.ptr(wsp), wsb
+        frt.frt_chain_layer(d)
+        torch.cuda.synchronize()
+        r_res, r_x8, r_q, r_k, r_v = ref[l]
+        dist = e4m3_step_distance(runtime.u8_host(x8), r_x8)
+        if l == 0:
+            assert_codes(runtime.u8_host(x8), r_x8, what="layer 0 x8")
+        else:
+            assert (dist == 0).mean() >= 0.999, f"layer {l} x8"
+        assert_rms(h(q[l % 2]), r_q, what=f"layer {l} q_out")
+        assert_rms(h(kc)[:, w.P:], r_k[:, w.P:], what=f"layer {l} k rows")
+        assert np.array_equal(h(kc)[:, :w.P], r_k[:, :w.P])
+        assert_rms(h(res), r_res, what=f"layer {l} residual")
+    assert frt.frt_device_status(True) == frt.FRT_OK
+
+
+def test_gateup_mlp_chain(rt):
+    """Producer -> gate/up GEMM with the fused GEGLU requant -> down GEMM on
+    the gate/up MLP's weights (D=2048, H=16384) at 64 tokens."""
+    frt, runtime, torch = rt
+    w = synth.WORKLOADS["gateup_mlp"]
+    M, D, H = 64, w.D, w.H
+    mw = synth.mlp_weights(D, H, w.seed)
+    inp = synth.adarms_inputs(M, D, w.seed)
+    a_gu = calibrate_adarms(w)
+    pr = oracle.ada_rms_norm_quant(inp["res"], inp["delta"], inp["prev_gate"],
+                                   inp["style"], a_gu)
+    gu_ref = oracle.pack_weights_fp8([mw["gate"], mw["up"]])
+    dn_ref = oracle.pack_weights_fp8([mw["down"]])
+    gu = oracle.fp8_gemm(pr["x8"], gu_ref["w8"], a_gu, gu_ref["w_scale"])
+    _, amax = oracle.geglu_quant(gu, 1.0)
+    a_dn = amax / 448.0
+    hid_ref, _ = oracle.geglu_quant(gu, a_dn)
+    out_ref = oracle.fp8_gemm(hid_ref, dn_ref["w8"], a_dn, dn_ref["w_scale"])
+
+    blk = runtime.pack([mw["gate"], mw["up"]],
+                       layout=frt.FRT_PACK_GATE_UP_BLOCKS)
+    dn = runtime.pack([mw["down"]])
+    res = runtime.bf16_dev(inp["res"])
+    x8 = runtime.empty_u8(M, D)
+    s_gu, s_dn = runtime.scale_dev(a_gu), runtime.scale_dev(a_dn)
+    frt.frt_ada_norm_quant_fp8(frt.FRT_NORM_ADARMS, M, D, w.eps, res,
+                               runtime.bf16_dev(inp["delta"]),
+                               runtime.bf16_dev(inp["prev_gate"]), 0, None,
+                               runtime.bf16_dev(inp["style"]), 0, None, None,
+                               0, None, 0, 0, s_gu, x8, None, None)
+    hid = runtime.empty_u8(M, H)
+    ws1 = frt.frt_gemm_workspace_size(M, 2 * H, D, frt.FRT_EPI_GEGLU_E4M3)
+    frt.frt_packed_fp8_gemm(M, 2 * H, D, x8, blk.w8, s_gu, blk.w_scale, None,
+                            frt.FRT_EPI_GEGLU_E4M3, hid, H, s_dn,
+                            runtime.workspace(ws1), ws1)
+    out = runtime.empty_bf16(M, D)
+    ws2 = frt.frt_gemm_workspace_size(M, D, H)
+    frt.frt_packed_fp8_gemm(M, D, H, hid, dn.w8, s_dn, dn.w_scale, None,
+                            frt.FRT_EPI_BF16, out, D, None,
+                            runtime.workspace(ws2), ws2)
+    torch.cuda.synchronize()
+    assert_codes(runtime.u8_host(x8), pr["x8"], what="x8")
+    d = e4m3_step_distance(runtime.u8_host(hid), hid_ref)
+    assert (d <= 1).all() and (d == 0).mean() >= 0.99, "hid8 end to end"
+    assert_rms(runtime.bf16_host(out), out_ref, what="down projection")
