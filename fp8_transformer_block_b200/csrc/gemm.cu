@@ -18,11 +18,12 @@
 //               double-buffered accumulator lets it overlap the next unit's
 //               main loop.
 // Large M: A = x8 (tokens on TMEM lanes), B = w8, BN = 256 (or 128).
-// Small M (<= 128): swap A and B so the packed weights fill the 128 MMA rows
-// and the few tokens are the MMA N (16..128); K is split over CTAs so the
-// weight stream is spread across the SMs, and the CTA that finishes a tile
-// last sums the fp32 partials in split order (deterministic, no atomics on
-// data, no waiting between CTAs).
+// Small M (<= 128): swap A and B so the packed weights fill the MMA rows (64
+// per tile, twice the tiles of 128-row tiles) and the few tokens are the MMA
+// N (64 or 128); when the tiles still leave most SMs idle, K is split over
+// CTAs so the weight stream is spread across the SMs, and the CTA that
+// finishes a tile last sums the fp32 partials in split order (deterministic,
+// no atomics on data, no waiting between CTAs).
 // Every wait on an mbarrier is bounded in time; a wait that runs out records
 // FRT_ETIMEOUT, the CTA drains its in-flight copies and MMAs (again bounded),
 // frees its TMEM and returns.  No TMA multicast is used anywhere.
@@ -34,14 +35,17 @@
 namespace frt {
 namespace {
 
-constexpr int BM = 128;             // MMA M = TMEM lanes
+constexpr int BM = 128;             // MMA M of the normal orientation
 constexpr int BK = 128;             // K bytes per stage: one swizzle row
 constexpr int kThreads = 192;
-constexpr int A_BYTES = BM * BK;    // 16 KB
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per wait
 constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s to drain after an abort
 
 enum { EPI_BF16 = 0, EPI_GEGLU = 1, EPI_ROPE = 2 };
+
+#ifndef FRT_MIN_KB_PER_SPLIT
+#define FRT_MIN_KB_PER_SPLIT 4  // K-blocks (of 128) per split at least
+#endif
 
 struct GemmParams {
   int M, N, K;
@@ -169,19 +173,32 @@ __device__ __forceinline__ void epi_geglu_chunk(const GemmParams& p, const float
   }
 }
 
+// TMEM lane holding accumulator row r of an MMA with M = BMT rows: all 128
+// lanes for M = 128; for M = 64 the rows fill the first 16 lanes of each
+// 32-lane quarter (rows 16q .. 16q+15 in lanes 32q .. 32q+15).  The epilogue
+// warp of quarter q therefore owns rows 16q + lane (lane < 16) when BMT = 64.
+template <int BMT>
+__device__ __forceinline__ int acc_row(int q, int lane) {
+  return BMT == 128 ? 32 * q + lane : 16 * q + lane;
+}
+template <int BMT>
+__device__ __forceinline__ bool acc_row_valid(int lane) {
+  return BMT == 128 || lane < 16;
+}
+
 // Run the epilogue of one tile.  load(c, v) fills v with accumulator chunk c
 // (32 columns of this thread's TMEM lane); it is called warp-uniformly.
 // done() runs once every chunk has been loaded (it releases the TMEM
 // accumulator when the chunks come from TMEM).
 // Swapped orientation: the chunks are staged in the shared-memory tile T
-// (fp32 [128 output columns][BN tokens], row stride BN + 4) and read back
+// (fp32 [BMT output columns][BN tokens], row stride BN + 4) and read back
 // transposed, so each thread then owns one token row with 32 contiguous
 // output columns and the row epilogue applies unchanged.
-template <bool SWAP, int BN, class Load, class Done>
+template <bool SWAP, int BMT, int BN, class Load, class Done>
 __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int tb, int q, int lane,
                                               float alpha, float* T, Load load, Done done) {
   if (!SWAP && p.epi == EPI_GEGLU) {
-    const int m = ta * BM + 32 * q + lane;
+    const int m = ta * BMT + 32 * q + lane;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       float g[32], u[32];
@@ -194,7 +211,7 @@ __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int t
     return;
   }
   if (!SWAP) {
-    const int m = ta * BM + 32 * q + lane;
+    const int m = ta * BMT + 32 * q + lane;
     int c_last = BN / 32 - 1;
     while (c_last > 0 && tb * BN + 32 * c_last >= p.N) --c_last;
 #pragma unroll 1
@@ -207,26 +224,30 @@ __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int t
     return;
   }
   constexpr int TS = BN + 4;
-  const int row = 32 * q + lane;
+  const int row = acc_row<BMT>(q, lane);
+  const bool valid = acc_row_valid<BMT>(lane);
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     float v[32];
     load(c, v);
-    float4* d4 = reinterpret_cast<float4*>(T + row * TS + 32 * c);
+    if (valid) {
+      float4* d4 = reinterpret_cast<float4*>(T + row * TS + 32 * c);
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+      for (int k = 0; k < 8; ++k)
+        d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+    }
   }
   done();
   named_bar_sync(2, 128);
-  constexpr int COLS = BM * BN / 128;   // output columns per thread (BN for BN <= 128)
+  constexpr int COLS = BMT * BN / 128;  // output columns per thread
+  static_assert(COLS % 32 == 0, "each thread takes whole 32-column chunks");
   const int t = int(threadIdx.x) - 64;  // 0 .. 127 over the four epilogue warps
   const int m_local = t % BN, g = t / BN;
   const int m = tb * BN + m_local;
 #pragma unroll 1
   for (int cc = 0; cc < COLS / 32; ++cc) {
     const int nl0 = g * COLS + 32 * cc;
-    const int n0 = ta * BM + nl0;
+    const int n0 = ta * BMT + nl0;
     if (n0 >= p.N) break;
     float v[32];
 #pragma unroll
@@ -238,20 +259,22 @@ __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int t
 
 // ------------------------------------------------------------------ kernel --
 
-template <bool SWAP, int BN>
+template <bool SWAP, int BMT, int BN>
 __host__ __device__ constexpr int t_tile_bytes() {
-  return SWAP ? BM * (BN + 4) * 4 : 0;
+  return SWAP ? BMT * (BN + 4) * 4 : 0;
 }
 
-template <bool SWAP, int BN, int STAGES>
+template <bool SWAP, int BMT, int BN, int STAGES>
 __host__ __device__ constexpr int smem_total() {
-  return STAGES * (A_BYTES + BN * BK) + t_tile_bytes<SWAP, BN>() + 1024 + 256;
+  return STAGES * (BMT * BK + BN * BK) + t_tile_bytes<SWAP, BMT, BN>() + 1024 + 256;
 }
 
-template <bool SWAP, int BN, int STAGES>
+template <bool SWAP, int BMT, int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const GemmParams p) {
+  static_assert(SWAP || BMT == 128, "the normal orientation uses 128-row tiles");
+  constexpr int A_BYTES = BMT * BK;
   constexpr int B_BYTES = BN * BK;
   constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * BN);
   extern __shared__ uint8_t smem_raw[];
@@ -260,7 +283,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
   float* T = reinterpret_cast<float*>(sB + STAGES * B_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES + t_tile_bytes<SWAP, BN>());
+  uint64_t* full =
+      reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES + t_tile_bytes<SWAP, BMT, BN>());
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -303,9 +327,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
-      // The packed weights are never written by an earlier kernel: the first
-      // unit's weight slices are requested before waiting on the producer
-      // kernel of the activations, so they stream in while it finishes.
+      // The packed weights are not written by the kernel this one may
+      // overlap: the first unit's weight slices are requested before waiting
+      // on the kernel that produces the activations, so they stream in while
+      // it finishes.
       const CUtensorMap* wmap = SWAP ? &tmA : &tmB;
       const CUtensorMap* xmap = SWAP ? &tmB : &tmA;
       const int u0 = blockIdx.x;
@@ -318,7 +343,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         n_pre = kb1 - kb0 < STAGES ? kb1 - kb0 : STAGES;
         for (int i = 0; i < n_pre; ++i) {
           mbar_arrive_expect_tx(&full[i], A_BYTES + B_BYTES);
-          if (SWAP) tma_load_2d(sA + i * A_BYTES, wmap, &full[i], (kb0 + i) * BK, ta * BM);
+          if (SWAP) tma_load_2d(sA + i * A_BYTES, wmap, &full[i], (kb0 + i) * BK, ta * BMT);
           else tma_load_2d(sB + i * B_BYTES, wmap, &full[i], (kb0 + i) * BK, tb * BN);
         }
       }
@@ -339,11 +364,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
               break;
             }
             mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES);
-            if (SWAP) tma_load_2d(sA + stage * A_BYTES, wmap, &full[stage], kb * BK, ta * BM);
+            if (SWAP) tma_load_2d(sA + stage * A_BYTES, wmap, &full[stage], kb * BK, ta * BMT);
             else tma_load_2d(sB + stage * B_BYTES, wmap, &full[stage], kb * BK, tb * BN);
           }
           if (SWAP) tma_load_2d(sB + stage * B_BYTES, xmap, &full[stage], kb * BK, tb * BN);
-          else tma_load_2d(sA + stage * A_BYTES, xmap, &full[stage], kb * BK, ta * BM);
+          else tma_load_2d(sA + stage * A_BYTES, xmap, &full[stage], kb * BK, ta * BMT);
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -363,7 +388,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      constexpr uint32_t idesc = idesc_e4m3_f32(BMT, BN);
       const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
       int stage = 0, local = 0;
       uint32_t phase = 0;
@@ -403,6 +428,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     pdl_wait();
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
+    const int row = acc_row<BMT>(q, lane);
+    const bool valid = acc_row_valid<BMT>(lane);
     int local = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++local) {
       const int tile = u / p.splits, split = u % p.splits;
@@ -430,21 +457,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         if (lane == 0) mbar_arrive(&tempty[ab]);
       };
       if (p.splits == 1) {
-        tile_epilogue<SWAP, BN>(
+        tile_epilogue<SWAP, BMT, BN>(
             p, ta, tb, q, lane, alpha, T,
             [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); }, release_tmem);
       } else {
-        // spill this split's fp32 partial: row (lane of TMEM) major
-        const int row = 32 * q + lane;
-        float* part = p.partials + (long(tile) * p.splits + split) * (BM * BN) + long(row) * BN;
+        // spill this split's fp32 partial, accumulator-row major
+        float* part = p.partials + (long(tile) * p.splits + split) * (BMT * BN) + long(row) * BN;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
           tmem_ld32(tbase + 32 * c, v);
-          float4* d4 = reinterpret_cast<float4*>(part + 32 * c);
+          if (valid) {
+            float4* d4 = reinterpret_cast<float4*>(part + 32 * c);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            for (int k = 0; k < 8; ++k)
+              d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          }
         }
         release_tmem();
         __threadfence();
@@ -456,18 +484,37 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         named_bar_sync(1, 128);
         if (*last_flag) {
           __threadfence();
-          const float* base = p.partials + long(tile) * p.splits * (BM * BN) + long(row) * BN;
-          tile_epilogue<SWAP, BN>(
+          const float* base = p.partials + long(tile) * p.splits * (BMT * BN) + long(row) * BN;
+          tile_epilogue<SWAP, BMT, BN>(
               p, ta, tb, q, lane, alpha, T,
               [&](int c, float (&v)[32]) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-                for (int s = 0; s < p.splits; ++s) {
-                  const float4* src =
-                      reinterpret_cast<const float4*>(base + long(s) * (BM * BN) + 32 * c);
+                if (!valid) return;
+                // two splits per step keep 16 loads in flight per thread
+                int s = 0;
+                for (; s + 1 < p.splits; s += 2) {
+                  const float4* s0 =
+                      reinterpret_cast<const float4*>(base + long(s) * (BMT * BN) + 32 * c);
+                  const float4* s1 =
+                      reinterpret_cast<const float4*>(base + long(s + 1) * (BMT * BN) + 32 * c);
+                  float4 f0[8], f1[8];
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) { f0[k] = __ldcg(s0 + k); f1[k] = __ldcg(s1 + k); }
 #pragma unroll
                   for (int k = 0; k < 8; ++k) {
-                    const float4 f = __ldcg(src + k);
+                    v[4 * k] = __fadd_rn(__fadd_rn(v[4 * k], f0[k].x), f1[k].x);
+                    v[4 * k + 1] = __fadd_rn(__fadd_rn(v[4 * k + 1], f0[k].y), f1[k].y);
+                    v[4 * k + 2] = __fadd_rn(__fadd_rn(v[4 * k + 2], f0[k].z), f1[k].z);
+                    v[4 * k + 3] = __fadd_rn(__fadd_rn(v[4 * k + 3], f0[k].w), f1[k].w);
+                  }
+                }
+                if (s < p.splits) {
+                  const float4* s0 =
+                      reinterpret_cast<const float4*>(base + long(s) * (BMT * BN) + 32 * c);
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) {
+                    const float4 f = __ldcg(s0 + k);
                     v[4 * k] = __fadd_rn(v[4 * k], f.x);
                     v[4 * k + 1] = __fadd_rn(v[4 * k + 1], f.y);
                     v[4 * k + 2] = __fadd_rn(v[4 * k + 2], f.z);
@@ -530,52 +577,56 @@ int make_map(CUtensorMap* m, const void* ptr, long rows, int K, int box_rows) {
 
 struct Plan {
   bool swap;
-  int bn, a_tiles, b_tiles, k_blocks, splits, units, grid;
+  int bmt, bn, a_tiles, b_tiles, k_blocks, splits, units, grid;
   size_t counters_bytes, ws_bytes;
 };
 
 Plan make_plan(int M, int N, int K, int epi) {
   Plan pl{};
   pl.k_blocks = (K + BK - 1) / BK;
+  pl.bmt = 128;
   if (epi == EPI_GEGLU) { pl.swap = false; pl.bn = 256; }
-  else if (M <= 128) { pl.swap = true; pl.bn = M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+  else if (M <= 128) { pl.swap = true; pl.bmt = 64; pl.bn = M <= 64 ? 64 : 128; }
   else { pl.swap = false; pl.bn = (N % 256 == 0) ? 256 : 128; }
   const long a_rows = pl.swap ? N : M, b_rows = pl.swap ? M : N;
-  pl.a_tiles = int((a_rows + BM - 1) / BM);
+  pl.a_tiles = int((a_rows + pl.bmt - 1) / pl.bmt);
   pl.b_tiles = int((b_rows + pl.bn - 1) / pl.bn);
   const int tiles = pl.a_tiles * pl.b_tiles;
   const int sms = num_sms();
   pl.splits = 1;
+  // split K only when the tiles leave most SMs idle and each split keeps at
+  // least FRT_MIN_KB_PER_SPLIT K-blocks of work
   if (tiles * 2 <= sms) {
-    pl.splits = sms / tiles;
-    if (pl.splits > pl.k_blocks) pl.splits = pl.k_blocks;
-    if (pl.splits > 16) pl.splits = 16;
-    if (pl.splits < 1) pl.splits = 1;
+    int s = sms / tiles;
+    const int by_k = pl.k_blocks / FRT_MIN_KB_PER_SPLIT;
+    if (s > by_k) s = by_k;
+    if (s > 16) s = 16;
+    pl.splits = s < 1 ? 1 : s;
   }
   pl.units = tiles * pl.splits;
   pl.grid = pl.units < sms ? pl.units : sms;
   if (pl.splits > 1) {
     pl.counters_bytes = (size_t(tiles) * sizeof(unsigned) + 255) & ~size_t(255);
-    pl.ws_bytes = pl.counters_bytes + size_t(tiles) * pl.splits * BM * pl.bn * sizeof(float);
+    pl.ws_bytes = pl.counters_bytes + size_t(tiles) * pl.splits * pl.bmt * pl.bn * sizeof(float);
   }
   return pl;
 }
 
-template <bool SWAP, int BN, int STAGES>
+template <bool SWAP, int BMT, int BN, int STAGES>
 int launch_t(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
              cudaStream_t s) {
-  constexpr int smem = smem_total<SWAP, BN, STAGES>();
+  constexpr int smem = smem_total<SWAP, BMT, BN, STAGES>();
   static_assert(smem <= 232448, "shared memory budget");
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(gemm_kernel<SWAP, BN, STAGES>,
+    if (cudaFuncSetAttribute(gemm_kernel<SWAP, BMT, BN, STAGES>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return fail(FRT_ECUDA, "cudaFuncSetAttribute(max dynamic smem %d)", smem);
     attr_set[dev] = true;
   }
-  return launch_pdl("gemm_kernel", gemm_kernel<SWAP, BN, STAGES>, dim3(pl.grid), dim3(kThreads),
+  return launch_pdl("gemm_kernel", gemm_kernel<SWAP, BMT, BN, STAGES>, dim3(pl.grid), dim3(kThreads),
                     size_t(smem), s, ta, tb, p);
 }
 
@@ -600,14 +651,13 @@ int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void
     if ((rc = make_map(&ta, x8, p.M, p.K, BM))) return rc;
     if ((rc = make_map(&tb, w8, p.N, p.K, pl.bn))) return rc;
   } else {
-    if ((rc = make_map(&ta, w8, p.N, p.K, BM))) return rc;
+    if ((rc = make_map(&ta, w8, p.N, p.K, pl.bmt))) return rc;
     if ((rc = make_map(&tb, x8, p.M, p.K, pl.bn))) return rc;
   }
-  if (!pl.swap && pl.bn == 256) return launch_t<false, 256, 4>(pl, ta, tb, p, s);
-  if (!pl.swap) return launch_t<false, 128, 6>(pl, ta, tb, p, s);
-  if (pl.bn == 32) return launch_t<true, 32, 8>(pl, ta, tb, p, s);
-  if (pl.bn == 64) return launch_t<true, 64, 7>(pl, ta, tb, p, s);
-  return launch_t<true, 128, 4>(pl, ta, tb, p, s);
+  if (!pl.swap && pl.bn == 256) return launch_t<false, 128, 256, 4>(pl, ta, tb, p, s);
+  if (!pl.swap) return launch_t<false, 128, 128, 6>(pl, ta, tb, p, s);
+  if (pl.bn == 64) return launch_t<true, 64, 64, 12>(pl, ta, tb, p, s);
+  return launch_t<true, 64, 128, 7>(pl, ta, tb, p, s);
 }
 
 int validate_common(int M, int N, int K, const void* x8, const void* w8, const float* act_scale,

@@ -48,6 +48,11 @@ __global__ void pack_amax_kernel(PackArgs a) {
   if ((threadIdx.x & 31) == 0) atomic_max_nonneg(a.scale, mx);
 }
 
+// Launched (without programmatic overlap) after the quantize kernel so the
+// packed weights are complete and visible before any later kernel starts:
+// the GEMM may read weights before its own dependency wait.
+__global__ void pack_fence_kernel() {}
+
 __global__ void pack_finalize_kernel(float* scale) {
   const float s = __fdiv_rn(*scale, 448.0f);
   *scale = s < 1e-8f ? 1e-8f : s;
@@ -139,5 +144,6 @@ extern "C" int frt_pack_weights_fp8(int n_siblings, const frt_bf16* const* w,
   frt::pack_amax_kernel<<<sms * 4, 256, 0, s>>>(a);
   frt::pack_finalize_kernel<<<1, 1, 0, s>>>(w_scale_out);
   frt::pack_quant_kernel<<<sms * 8, 256, 0, s>>>(a);
+  frt::pack_fence_kernel<<<1, 32, 0, s>>>();
   return frt::check_launch("frt_pack_weights_fp8");
 }

@@ -162,9 +162,13 @@ size_t frt_gemm_workspace_size(int M, int N, int K, int epilogue);
  *                  out[m, j] = e4m3(gelu_tanh(g) * u / out_scale)
  *                  out: [M, ldo] e4m3, ldo >= N / 2; N % 256 == 0.
  * x8: [M, K] e4m3; w8: [N, K] e4m3; bias: [N] bf16 or NULL.
- * Requires K % 16 == 0, N % 32 == 0, 16-byte aligned x8/w8/out, ldo % 16 == 0
- * (bytes of a row).  M == 0 is a no-op.  workspace: see
+ * Requires K % 16 == 0, N % 32 == 0, 16-byte aligned x8/w8/out/bias, ldo %
+ * 16 == 0 (bytes of a row).  M == 0 is a no-op.  workspace: see
  * frt_gemm_workspace_size (may be NULL when that is 0).
+ * The kernel starts loading w8 while the kernel before it on the stream
+ * finishes (programmatic dependent launch): w8 must not be written by the
+ * immediately preceding kernel on the stream (frt_pack_weights_fp8 ends with
+ * a fence launch, so weights it packed are always safe).
  */
 int frt_packed_fp8_gemm(int M, int N, int K, const frt_e4m3* x8,
                         const frt_e4m3* w8, const float* act_scale,
