@@ -4,6 +4,10 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "frt_common.cuh"
 #include "frt_sm100.cuh"
 
@@ -57,6 +61,15 @@ int num_sms() {
     g_sms[dev] = n > 0 ? n : 148;
   }
   return g_sms[dev];
+}
+
+bool first_use(const void* kernel) {
+  static std::mutex mu;
+  static std::set<std::pair<int, const void*>> seen;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  return seen.insert({dev, kernel}).second;
 }
 
 // A single CTA waits on an mbarrier whose arrival count is never reached.

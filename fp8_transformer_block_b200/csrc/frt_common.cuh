@@ -26,6 +26,8 @@ int check_launch(const char* what);
 int* device_status_ptr();
 // Streaming multiprocessors of the current device (cached per device).
 int num_sms();
+// True the first time it is called for this kernel on the current device.
+bool first_use(const void* kernel);
 
 inline bool aligned(const void* p, size_t a) {
   return (reinterpret_cast<uintptr_t>(p) % a) == 0;
@@ -55,6 +57,11 @@ int launch_pdl(const char* what, void (*kern)(KArgs...), dim3 grid, dim3 block, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // every kernel of the chain asks for the same L1 / shared-memory split as
+  // the GEMM, so an SM never has to drain to reconfigure between them
+  if (first_use(reinterpret_cast<const void*>(kern)))
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
   if (e != cudaSuccess) {
     cudaGetLastError();

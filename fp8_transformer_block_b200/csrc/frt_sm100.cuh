@@ -64,6 +64,10 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
+}
+
 // ----------------------------------------------------------------- TMA ----
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {

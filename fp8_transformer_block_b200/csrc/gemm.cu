@@ -44,7 +44,7 @@ constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s to drain after an abort
 enum { EPI_BF16 = 0, EPI_GEGLU = 1, EPI_ROPE = 2 };
 
 #ifndef FRT_MIN_KB_PER_SPLIT
-#define FRT_MIN_KB_PER_SPLIT 4  // K-blocks (of 128) per split at least
+#define FRT_MIN_KB_PER_SPLIT 16  // K-blocks (of 128) per split at least
 #endif
 
 struct GemmParams {
@@ -425,6 +425,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     }
   } else {
     // ----------------------------------------------------------- epilogue --
+    // The rope table is bind-time data: pull this CTA's first-unit rows into
+    // L2 before waiting on the previous kernel, so the epilogue finds them.
+    if (p.epi == EPI_ROPE && blockIdx.x < unsigned(p.units)) {
+      const int tile0 = int(blockIdx.x) / p.splits;
+      const int tok_tile = SWAP ? tile0 / p.a_tiles : tile0 % p.a_tiles;
+      const int tok_rows = SWAP ? BN : BMT;
+      const long row_bytes = long(p.hd) * 2;
+      const int t = int(threadIdx.x) - 64;
+      for (int r = t; r < tok_rows; r += 128) {
+        const int m = tok_tile * tok_rows + r;
+        if (m >= p.M) break;
+        const char* base = reinterpret_cast<const char*>(p.rope + long(m % p.Mseq) * p.hd);
+        for (long off = 0; off < row_bytes; off += 128) prefetch_l2(base + off);
+      }
+    }
     pdl_wait();
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
@@ -587,7 +602,13 @@ Plan make_plan(int M, int N, int K, int epi) {
   pl.bmt = 128;
   if (epi == EPI_GEGLU) { pl.swap = false; pl.bn = 256; }
   else if (M <= 128) { pl.swap = true; pl.bmt = 64; pl.bn = M <= 64 ? 64 : 128; }
-  else { pl.swap = false; pl.bn = (N % 256 == 0) ? 256 : 128; }
+  else {
+    pl.swap = false;
+    pl.bn = (N % 256 == 0) ? 256 : 128;
+    // narrower tiles before splitting K when 256-wide tiles underfill the SMs
+    const long t256 = ((M + 127L) / 128) * ((N + 255L) / 256);
+    if (pl.bn == 256 && t256 < num_sms()) pl.bn = 128;
+  }
   const long a_rows = pl.swap ? N : M, b_rows = pl.swap ? M : N;
   pl.a_tiles = int((a_rows + pl.bmt - 1) / pl.bmt);
   pl.b_tiles = int((b_rows + pl.bn - 1) / pl.bn);
@@ -624,6 +645,9 @@ int launch_t(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const
     if (cudaFuncSetAttribute(gemm_kernel<SWAP, BMT, BN, STAGES>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return fail(FRT_ECUDA, "cudaFuncSetAttribute(max dynamic smem %d)", smem);
+    cudaFuncSetAttribute(gemm_kernel<SWAP, BMT, BN, STAGES>,
+                         cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
     attr_set[dev] = true;
   }
   return launch_pdl("gemm_kernel", gemm_kernel<SWAP, BMT, BN, STAGES>, dim3(pl.grid), dim3(kThreads),
