@@ -179,8 +179,11 @@ GEMM_CASES = [
     (128, 2560, 2048, False),
     (129, 640, 512, False),        # first normal-orientation size
     (300, 672, 528, True),         # ragged everywhere, BN = 128
-    (1000, 2560, 2048, True),      # BN = 256, persistent
+    (1000, 2560, 2048, True),      # 128-wide tiles (256-wide would underfill)
     (256, 9216, 3072, True),       # video-DiT projection width
+    (1200, 4096, 1024, False),     # 256-wide tiles, persistent
+    (64, 2048, 16384, False),      # long K: split over 4 CTAs per tile
+    (100, 1024, 4096, True),       # split in 2, ragged token tile
 ]
 
 
