@@ -79,11 +79,13 @@ __global__ void bounded_wait_probe(int* status, uint64_t timeout_ns) {
     mbar_init(&bar, 1);
     fence_barrier_init();
   }
+  __syncwarp();
   __syncthreads();
   if (threadIdx.x == 0) {
     bool ok = mbar_wait_bounded(&bar, 0, timeout_ns, nullptr);
     if (!ok) atomicExch(status, FRT_ETIMEOUT);
   }
+  __syncwarp();
   __syncthreads();
 }
 

@@ -319,6 +319,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
   }
+  __syncwarp();  // warp 0's lanes wait for lane 0's barrier set-up
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -385,6 +386,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         }
       }
     }
+    // the other 31 lanes wait here for lane 0, so the warp reaches the block
+    // barrier below converged (an aligned barrier must not be met by part of
+    // a warp while the rest is still working)
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0) {
@@ -423,6 +428,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         mbar_wait_bounded(drain, 0, kDrainNs, nullptr);
       }
     }
+    __syncwarp();  // converge before the block barrier and the TMEM release
   } else {
     // ----------------------------------------------------------- epilogue --
     // The rope table is bind-time data: pull this CTA's first-unit rows into

@@ -16,7 +16,9 @@ import ctypes as C
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfrt.so")
+# FRT_LIBRARY may name another build of the same ABI (e.g. an instrumented
+# one); by default the in-tree libfrt.so is loaded.
+LIB_PATH = os.environ.get("FRT_LIBRARY") or os.path.join(_HERE, "libfrt.so")
 
 FRT_OK, FRT_EINVAL, FRT_ESHAPE, FRT_EALIGN, FRT_ERANGE, FRT_ECUDA, \
     FRT_ETIMEOUT = 0, -1, -2, -3, -4, -5, -6
