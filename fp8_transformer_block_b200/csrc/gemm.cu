@@ -186,6 +186,27 @@ __device__ __forceinline__ bool acc_row_valid(int lane) {
   return BMT == 128 || lane < 16;
 }
 
+// Swapped orientation, emitting half: the tile's (32-column chunk, token)
+// items, this thread taking items first + stride * t, t = 0, 1, ... over the
+// 128 epilogue threads.  fetch(c, m_local, v) gathers the item's 32 fp32
+// accumulators (output columns 32c .. 32c+31 of token m_local).
+template <int BMT, int BN, class Fetch>
+__device__ __forceinline__ void emit_swap_items(const GemmParams& p, int ta, int tb, float alpha,
+                                                int first, int stride, Fetch fetch) {
+  constexpr int ITEMS = (BMT / 32) * BN;
+  const int t = int(threadIdx.x) - 64;  // 0 .. 127 over the four epilogue warps
+#pragma unroll 1
+  for (int it = first + stride * t; it < ITEMS; it += stride * 128) {
+    const int c = it / BN, m_local = it % BN;
+    const int n0 = ta * BMT + 32 * c;
+    const int m = tb * BN + m_local;
+    if (n0 >= p.N || m >= p.M) continue;
+    float v[32];
+    fetch(c, m_local, v);
+    epi_rows_chunk(p, v, m, n0, alpha);
+  }
+}
+
 // Run the epilogue of one tile.  load(c, v) fills v with accumulator chunk c
 // (32 columns of this thread's TMEM lane); it is called warp-uniformly.
 // done() runs once every chunk has been loaded (it releases the TMEM
@@ -223,7 +244,7 @@ __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int t
     }
     return;
   }
-  constexpr int TS = BN + 4;
+  constexpr int TS = BMT + 4;
   const int row = acc_row<BMT>(q, lane);
   const bool valid = acc_row_valid<BMT>(lane);
 #pragma unroll 1
@@ -231,37 +252,47 @@ __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int t
     float v[32];
     load(c, v);
     if (valid) {
-      float4* d4 = reinterpret_cast<float4*>(T + row * TS + 32 * c);
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+      for (int j = 0; j < 32; ++j) T[(32 * c + j) * TS + row] = v[j];
     }
   }
   done();
   named_bar_sync(2, 128);
-  constexpr int COLS = BMT * BN / 128;  // output columns per thread
-  static_assert(COLS % 32 == 0, "each thread takes whole 32-column chunks");
-  const int t = int(threadIdx.x) - 64;  // 0 .. 127 over the four epilogue warps
-  const int m_local = t % BN, g = t / BN;
-  const int m = tb * BN + m_local;
-#pragma unroll 1
-  for (int cc = 0; cc < COLS / 32; ++cc) {
-    const int nl0 = g * COLS + 32 * cc;
-    const int n0 = ta * BMT + nl0;
-    if (n0 >= p.N) break;
-    float v[32];
+  emit_swap_items<BMT, BN>(p, ta, tb, alpha, 0, 1, [&](int c, int m_local, float (&v)[32]) {
+    const float4* src = reinterpret_cast<const float4*>(T + m_local * TS + 32 * c);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = T[(nl0 + j) * TS + m_local];
-    epi_rows_chunk(p, v, m, n0, alpha);
-  }
+    for (int k = 0; k < 8; ++k) {
+      const float4 f = src[k];
+      v[4 * k] = f.x; v[4 * k + 1] = f.y; v[4 * k + 2] = f.z; v[4 * k + 3] = f.w;
+    }
+  });
   named_bar_sync(2, 128);
+}
+
+// Swapped orientation, staging half: the accumulator of this thread's TMEM
+// lane (an output column) goes to the token-major tile T
+// ([BN tokens][BMT + 4] fp32) in this CTA's shared memory.
+template <int BMT, int BN, class Load>
+__device__ __forceinline__ void stage_swap_tile(float* T, int q, int lane, Load load) {
+  constexpr int TS = BMT + 4;
+  const int row = acc_row<BMT>(q, lane);
+  const bool valid = acc_row_valid<BMT>(lane);
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    load(c, v);
+    if (valid) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) T[(32 * c + j) * TS + row] = v[j];
+    }
+  }
 }
 
 // ------------------------------------------------------------------ kernel --
 
 template <bool SWAP, int BMT, int BN>
 __host__ __device__ constexpr int t_tile_bytes() {
-  return SWAP ? BMT * (BN + 4) * 4 : 0;
+  return SWAP ? BN * (BMT + 4) * 4 : 0;
 }
 
 template <bool SWAP, int BMT, int BN, int STAGES>
@@ -269,11 +300,17 @@ __host__ __device__ constexpr int smem_total() {
   return STAGES * (BMT * BK + BN * BK) + t_tile_bytes<SWAP, BMT, BN>() + 1024 + 256;
 }
 
-template <bool SWAP, int BMT, int BN, int STAGES>
+// CLUSTER: the p.splits K-splits of a tile run as one thread-block cluster
+// (rank = split, one unit per CTA); each CTA stages its fp32 partial in its
+// shared memory and, after a cluster barrier, the ranks share the tile's
+// epilogue, each summing its items over all ranks' partials (distributed
+// shared memory, rank order) -- no global partials, no atomics.
+template <bool SWAP, int BMT, int BN, int STAGES, bool CLUSTER>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const GemmParams p) {
   static_assert(SWAP || BMT == 128, "the normal orientation uses 128-row tiles");
+  static_assert(!CLUSTER || SWAP, "cluster K-splits serve the swapped orientation");
   constexpr int A_BYTES = BMT * BK;
   constexpr int B_BYTES = BN * BK;
   constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * BN);
@@ -472,6 +509,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + uint32_t(ab * BN) + (uint32_t(32 * q) << 16);
+      if (CLUSTER) {
+        // one unit per CTA: stage the partial; the cluster reduces it below
+        stage_swap_tile<BMT, BN>(T, q, lane,
+                                 [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); });
+        break;
+      }
       auto release_tmem = [&]() {
         tc_fence_before();
         __syncwarp();
@@ -551,6 +594,38 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     }
   }
 
+  if (CLUSTER) {
+    cluster_sync_all();  // every rank's partial is staged and visible
+    if (warp >= 2 && blockIdx.x < unsigned(p.units)) {
+      const int tile = int(blockIdx.x) / p.splits;
+      const int ta = tile % p.a_tiles, tb = tile / p.a_tiles;
+      const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
+      const uint32_t t_addr = smem_u32(T);
+      constexpr int TS = BMT + 4;
+      emit_swap_items<BMT, BN>(
+          p, ta, tb, alpha, int(cluster_ctarank()), p.splits,
+          [&](int c, int m_local, float (&v)[32]) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+            const uint32_t off = t_addr + uint32_t((m_local * TS + 32 * c) * 4);
+            for (int r = 0; r < p.splits; ++r) {
+              const uint32_t a = map_cluster(off, uint32_t(r));
+              float4 f[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) f[k] = ld_cluster_f4(a + 16u * k);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                v[4 * k] = __fadd_rn(v[4 * k], f[k].x);
+                v[4 * k + 1] = __fadd_rn(v[4 * k + 1], f[k].y);
+                v[4 * k + 2] = __fadd_rn(v[4 * k + 2], f[k].z);
+                v[4 * k + 3] = __fadd_rn(v[4 * k + 3], f[k].w);
+              }
+            }
+          });
+    }
+    cluster_sync_all();  // no rank leaves while another still reads its tile
+  }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -597,10 +672,15 @@ int make_map(CUtensorMap* m, const void* ptr, long rows, int K, int box_rows) {
 }
 
 struct Plan {
-  bool swap;
+  bool swap, cluster;
   int bmt, bn, a_tiles, b_tiles, k_blocks, splits, units, grid;
   size_t counters_bytes, ws_bytes;
 };
+
+#ifndef FRT_MIN_KB_PER_CLUSTER_SPLIT
+#define FRT_MIN_KB_PER_CLUSTER_SPLIT 2  // K-blocks per split of a cluster tile
+#endif
+constexpr int kMaxCluster = 8;  // portable cluster size
 
 Plan make_plan(int M, int N, int K, int epi) {
   Plan pl{};
@@ -621,6 +701,23 @@ Plan make_plan(int M, int N, int K, int epi) {
   const int tiles = pl.a_tiles * pl.b_tiles;
   const int sms = num_sms();
   pl.splits = 1;
+  if (pl.swap) {
+    // few weight tiles: split K over a cluster per tile so the weight stream
+    // is pulled by (almost) every SM; the cluster reduces on chip
+    int s_max = 1;
+    if (tiles * 2 <= sms) {
+      s_max = sms / tiles;
+      const int by_k = pl.k_blocks / FRT_MIN_KB_PER_CLUSTER_SPLIT;
+      if (s_max > by_k) s_max = by_k;
+      if (s_max > kMaxCluster) s_max = kMaxCluster;
+      if (s_max < 1) s_max = 1;
+    }
+    pl.cluster = s_max > 1;
+    pl.splits = s_max;
+    pl.units = tiles * pl.splits;
+    pl.grid = pl.cluster ? pl.units : (tiles < sms ? tiles : sms);
+    return pl;
+  }
   // split K only when the tiles leave most SMs idle and each split keeps at
   // least FRT_MIN_KB_PER_SPLIT K-blocks of work
   if (tiles * 2 <= sms) {
@@ -639,25 +736,103 @@ Plan make_plan(int M, int N, int K, int epi) {
   return pl;
 }
 
+template <bool SWAP, int BMT, int BN, int STAGES, bool CLUSTER>
+int prepare_kernel() {
+  constexpr int smem = smem_total<SWAP, BMT, BN, STAGES>();
+  static_assert(smem <= 232448, "shared memory budget");
+  auto kern = gemm_kernel<SWAP, BMT, BN, STAGES, CLUSTER>;
+  if (first_use(reinterpret_cast<const void*>(kern))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return fail(FRT_ECUDA, "cudaFuncSetAttribute(max dynamic smem %d)", smem);
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+  }
+  return FRT_OK;
+}
+
 template <bool SWAP, int BMT, int BN, int STAGES>
 int launch_t(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
              cudaStream_t s) {
   constexpr int smem = smem_total<SWAP, BMT, BN, STAGES>();
-  static_assert(smem <= 232448, "shared memory budget");
-  static bool attr_set[64] = {false};
+  int rc = prepare_kernel<SWAP, BMT, BN, STAGES, false>();
+  if (rc) return rc;
+  return launch_pdl("gemm_kernel", gemm_kernel<SWAP, BMT, BN, STAGES, false>, dim3(pl.grid),
+                    dim3(kThreads), size_t(smem), s, ta, tb, p);
+}
+
+// Most clusters of `size` CTAs of this kernel the device can hold at once.
+template <int BMT, int BN, int STAGES>
+int max_active_clusters(int size, int grid) {
+  constexpr int smem = smem_total<true, BMT, BN, STAGES>();
+  static int cache[64][kMaxCluster + 1];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(gemm_kernel<SWAP, BMT, BN, STAGES>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return fail(FRT_ECUDA, "cudaFuncSetAttribute(max dynamic smem %d)", smem);
-    cudaFuncSetAttribute(gemm_kernel<SWAP, BMT, BN, STAGES>,
-                         cudaFuncAttributePreferredSharedMemoryCarveout,
-                         cudaSharedmemCarveoutMaxShared);
-    attr_set[dev] = true;
+  if (dev < 64 && cache[dev][size] > 0) return cache[dev][size];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = size;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<true, BMT, BN, STAGES, true>, &cfg) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
   }
-  return launch_pdl("gemm_kernel", gemm_kernel<SWAP, BMT, BN, STAGES>, dim3(pl.grid), dim3(kThreads),
-                    size_t(smem), s, ta, tb, p);
+  if (dev < 64 && n > 0) cache[dev][size] = n;
+  return n;
+}
+
+// Swapped orientation: a cluster per tile when the plan splits K and the
+// device can hold every tile's cluster at once (else fewer splits).
+template <int BMT, int BN, int STAGES>
+int launch_swap(Plan pl, const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p,
+                cudaStream_t s) {
+  constexpr int smem = smem_total<true, BMT, BN, STAGES>();
+  if (pl.cluster) {
+    int rc = prepare_kernel<true, BMT, BN, STAGES, true>();
+    if (rc) return rc;
+    const int tiles = pl.a_tiles * pl.b_tiles;
+    int size = pl.splits;
+    while (size > 1 && max_active_clusters<BMT, BN, STAGES>(size, tiles * size) < tiles) --size;
+    if (size > 1) {
+      p.splits = size;
+      p.units = tiles * size;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(p.units);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = size;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 2;
+      cudaError_t e =
+          cudaLaunchKernelEx(&cfg, gemm_kernel<true, BMT, BN, STAGES, true>, ta, tb, p);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(FRT_ECUDA, "gemm_kernel (cluster %d): %s", size, cudaGetErrorString(e));
+      }
+      return FRT_OK;
+    }
+    // no cluster size fits: one CTA per tile, no K split
+    p.splits = 1;
+    p.units = tiles;
+    pl.grid = tiles < num_sms() ? tiles : num_sms();
+  }
+  return launch_t<true, BMT, BN, STAGES>(pl, ta, tb, p, s);
 }
 
 int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void* workspace,
@@ -686,8 +861,8 @@ int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void
   }
   if (!pl.swap && pl.bn == 256) return launch_t<false, 128, 256, 4>(pl, ta, tb, p, s);
   if (!pl.swap) return launch_t<false, 128, 128, 6>(pl, ta, tb, p, s);
-  if (pl.bn == 64) return launch_t<true, 64, 64, 12>(pl, ta, tb, p, s);
-  return launch_t<true, 64, 128, 7>(pl, ta, tb, p, s);
+  if (pl.bn == 64) return launch_swap<64, 64, 12>(pl, ta, tb, p, s);
+  return launch_swap<64, 128, 7>(pl, ta, tb, p, s);
 }
 
 int validate_common(int M, int N, int K, const void* x8, const void* w8, const float* act_scale,

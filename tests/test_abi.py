@@ -86,13 +86,15 @@ def test_gemm_validation(frt):
     assert _gemm(frt, epilogue=1, N=640, ldo=320) == frt.FRT_ESHAPE
     assert _gemm(frt, epilogue=1, N=512, ldo=256) == frt.FRT_EINVAL
     assert _gemm(frt, M=0) == frt.FRT_OK
-    # few tiles over a long K split K over the SMs and need a workspace
-    need = frt.frt_gemm_workspace_size(64, 2048, 16384)
+    # few 128-row tiles over a long K split K through a global workspace
+    need = frt.frt_gemm_workspace_size(200, 256, 16384)
     assert need > 0
-    assert _gemm(frt, M=64, N=2048, K=16384, ldo=2048) == frt.FRT_EINVAL
-    assert _gemm(frt, M=64, N=2048, K=16384, ldo=2048, workspace=A16 * 16,
+    assert _gemm(frt, M=200, N=256, K=16384, ldo=256) == frt.FRT_EINVAL
+    assert _gemm(frt, M=200, N=256, K=16384, ldo=256, workspace=A16 * 16,
                  workspace_bytes=need - 1) == frt.FRT_ERANGE
+    # small M splits K inside thread-block clusters: no workspace
     assert frt.frt_gemm_workspace_size(50, 2560, 2048) == 0
+    assert frt.frt_gemm_workspace_size(64, 2048, 16384) == 0
     assert frt.frt_gemm_workspace_size(8192, 9216, 3072) == 0
 
 

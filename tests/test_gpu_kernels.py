@@ -170,7 +170,7 @@ def _x8_codes(rows, K, seed):
 
 
 GEMM_CASES = [
-    # M, N, K, bias   (M <= 128 runs the swapped, split-K schedule)
+    # M, N, K, bias   (M <= 128 runs the swapped schedule, K split in clusters)
     (1, 640, 512, False),
     (16, 640, 512, False),
     (50, 2560, 2048, False),
@@ -182,8 +182,9 @@ GEMM_CASES = [
     (1000, 2560, 2048, True),      # 128-wide tiles (256-wide would underfill)
     (256, 9216, 3072, True),       # video-DiT projection width
     (1200, 4096, 1024, False),     # 256-wide tiles, persistent
-    (64, 2048, 16384, False),      # long K: split over 4 CTAs per tile
-    (100, 1024, 4096, True),       # split in 2, ragged token tile
+    (64, 2048, 16384, False),      # long K: K split in a 4-CTA cluster
+    (100, 1024, 4096, True),       # 8-CTA clusters, ragged token tile
+    (200, 256, 16384, True),       # 128-row tiles, K split via workspace
 ]
 
 
