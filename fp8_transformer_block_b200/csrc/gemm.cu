@@ -38,6 +38,7 @@ namespace {
 constexpr int BM = 128;             // MMA M of the normal orientation
 constexpr int BK = 128;             // K bytes per stage: one swizzle row
 constexpr int kThreads = 192;
+constexpr int kMaxCluster = 8;      // portable thread-block cluster size
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per wait
 constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s to drain after an abort
 
@@ -98,6 +99,56 @@ __device__ __forceinline__ void load32_bf16(const uint16_t* src, float (&f)[32])
 #pragma unroll
     for (int j = 0; j < 8; ++j) f[8 * k + j] = t[j];
   }
+}
+
+// One token row m, output columns n0 .. n0 + 7 (n0 % 8 == 0, inside one head):
+// the same arithmetic as epi_rows_chunk at 16-byte granularity.  The rope
+// and bias loads are issued by the caller before the accumulators arrive.
+__device__ __forceinline__ void epi_rows8(const GemmParams& p, const float (&v)[8], int m, int n0,
+                                          float alpha, const uint4& bias8, const uint4& rope8) {
+  float y[8];
+  if (p.bias) {
+    float b[8];
+    unpack8(bias8, b);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = bf2f(f2bf(__fadd_rn(__fmul_rn(v[j], alpha), b[j])));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = bf2f(f2bf(__fmul_rn(v[j], alpha)));
+  }
+  uint16_t* dst;
+  if (p.epi == EPI_BF16) {
+    dst = static_cast<uint16_t*>(p.out) + long(m) * p.ldo + n0;
+  } else {
+    const int b = m / p.Mseq, s = m % p.Mseq;
+    const int h = n0 / p.hd, d0 = n0 % p.hd;
+    if (h < p.hq + p.hkv) {
+      float r[8];
+      unpack8(rope8, r);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float c = r[2 * i], sn = r[2 * i + 1];
+        const float x0 = y[2 * i], x1 = y[2 * i + 1];
+        y[2 * i] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, sn));
+        y[2 * i + 1] = __fadd_rn(__fmul_rn(x0, sn), __fmul_rn(x1, c));
+      }
+      dst = h < p.hq ? p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d0
+                     : p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d0;
+    } else {
+      const int hv = h - p.hq - p.hkv;
+      dst = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + hv) * p.hd + d0;
+    }
+  }
+  *reinterpret_cast<uint4*>(dst) = pack8_bf16(y);
+}
+
+// The rope pairs and bias an 8-column item needs (zeros when unused).
+__device__ __forceinline__ void epi_rows8_operands(const GemmParams& p, int m, int n0, uint4& bias8,
+                                                   uint4& rope8) {
+  bias8 = p.bias ? __ldg(reinterpret_cast<const uint4*>(p.bias + n0)) : make_uint4(0, 0, 0, 0);
+  rope8 = make_uint4(0, 0, 0, 0);
+  if (p.epi == EPI_ROPE && n0 / p.hd < p.hq + p.hkv)
+    rope8 = __ldg(reinterpret_cast<const uint4*>(p.rope + long(m % p.Mseq) * p.hd + n0 % p.hd));
 }
 
 // This thread owns token row m, output columns n0 .. n0 + 31 (the normal
@@ -186,24 +237,28 @@ __device__ __forceinline__ bool acc_row_valid(int lane) {
   return BMT == 128 || lane < 16;
 }
 
-// Swapped orientation, emitting half: the tile's (32-column chunk, token)
-// items, this thread taking items first + stride * t, t = 0, 1, ... over the
-// 128 epilogue threads.  fetch(c, m_local, v) gathers the item's 32 fp32
-// accumulators (output columns 32c .. 32c+31 of token m_local).
+// Swapped orientation, emitting half: the tile's (token, 8-column) items,
+// numbered token-major so neighbouring threads write neighbouring 16-byte
+// pieces of one token row.  This thread takes items [lo, hi) with stride
+// 128 over the four epilogue warps.  fetch(m_local, c8, v) gathers the
+// item's 8 fp32 accumulators (output columns 8*c8 .. 8*c8+7 of token
+// m_local); the item's rope and bias loads are issued before it.
 template <int BMT, int BN, class Fetch>
 __device__ __forceinline__ void emit_swap_items(const GemmParams& p, int ta, int tb, float alpha,
-                                                int first, int stride, Fetch fetch) {
-  constexpr int ITEMS = (BMT / 32) * BN;
+                                                int lo, int hi, Fetch fetch) {
+  constexpr int C8 = BMT / 8;
   const int t = int(threadIdx.x) - 64;  // 0 .. 127 over the four epilogue warps
 #pragma unroll 1
-  for (int it = first + stride * t; it < ITEMS; it += stride * 128) {
-    const int c = it / BN, m_local = it % BN;
-    const int n0 = ta * BMT + 32 * c;
+  for (int it = lo + t; it < hi; it += 128) {
+    const int m_local = it / C8, c8 = it % C8;
+    const int n0 = ta * BMT + 8 * c8;
     const int m = tb * BN + m_local;
     if (n0 >= p.N || m >= p.M) continue;
-    float v[32];
-    fetch(c, m_local, v);
-    epi_rows_chunk(p, v, m, n0, alpha);
+    uint4 bias8, rope8;
+    epi_rows8_operands(p, m, n0, bias8, rope8);
+    float v[8];
+    fetch(m_local, c8, v);
+    epi_rows8(p, v, m, n0, alpha, bias8, rope8);
   }
 }
 
@@ -258,13 +313,12 @@ __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int t
   }
   done();
   named_bar_sync(2, 128);
-  emit_swap_items<BMT, BN>(p, ta, tb, alpha, 0, 1, [&](int c, int m_local, float (&v)[32]) {
-    const float4* src = reinterpret_cast<const float4*>(T + m_local * TS + 32 * c);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float4 f = src[k];
-      v[4 * k] = f.x; v[4 * k + 1] = f.y; v[4 * k + 2] = f.z; v[4 * k + 3] = f.w;
-    }
+  emit_swap_items<BMT, BN>(p, ta, tb, alpha, 0, BN * (BMT / 8),
+                           [&](int m_local, int c8, float (&v)[8]) {
+    const float4* src = reinterpret_cast<const float4*>(T + m_local * TS + 8 * c8);
+    const float4 a = src[0], b = src[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   });
   named_bar_sync(2, 128);
 }
@@ -602,23 +656,32 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
       const uint32_t t_addr = smem_u32(T);
       constexpr int TS = BMT + 4;
+      // the ranks share the tile's items in contiguous ranges
+      constexpr int ITEMS = BN * (BMT / 8);
+      const int r = int(cluster_ctarank());
+      const int lo = r * ITEMS / p.splits, hi = (r + 1) * ITEMS / p.splits;
       emit_swap_items<BMT, BN>(
-          p, ta, tb, alpha, int(cluster_ctarank()), p.splits,
-          [&](int c, int m_local, float (&v)[32]) {
+          p, ta, tb, alpha, lo, hi, [&](int m_local, int c8, float (&v)[8]) {
+            const uint32_t off = t_addr + uint32_t((m_local * TS + 8 * c8) * 4);
+            float4 f[2 * kMaxCluster];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-            const uint32_t off = t_addr + uint32_t((m_local * TS + 32 * c) * 4);
-            for (int r = 0; r < p.splits; ++r) {
-              const uint32_t a = map_cluster(off, uint32_t(r));
-              float4 f[8];
+            for (int q2 = 0; q2 < kMaxCluster; ++q2) {
+              if (q2 < p.splits) {
+                const uint32_t a = map_cluster(off, uint32_t(q2));
+                f[2 * q2] = ld_cluster_f4(a);
+                f[2 * q2 + 1] = ld_cluster_f4(a + 16u);
+              }
+            }
 #pragma unroll
-              for (int k = 0; k < 8; ++k) f[k] = ld_cluster_f4(a + 16u * k);
+            for (int j = 0; j < 8; ++j) v[j] = 0.0f;
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                v[4 * k] = __fadd_rn(v[4 * k], f[k].x);
-                v[4 * k + 1] = __fadd_rn(v[4 * k + 1], f[k].y);
-                v[4 * k + 2] = __fadd_rn(v[4 * k + 2], f[k].z);
-                v[4 * k + 3] = __fadd_rn(v[4 * k + 3], f[k].w);
+            for (int q2 = 0; q2 < kMaxCluster; ++q2) {
+              if (q2 < p.splits) {
+                const float4 a = f[2 * q2], b = f[2 * q2 + 1];
+                v[0] = __fadd_rn(v[0], a.x); v[1] = __fadd_rn(v[1], a.y);
+                v[2] = __fadd_rn(v[2], a.z); v[3] = __fadd_rn(v[3], a.w);
+                v[4] = __fadd_rn(v[4], b.x); v[5] = __fadd_rn(v[5], b.y);
+                v[6] = __fadd_rn(v[6], b.z); v[7] = __fadd_rn(v[7], b.w);
               }
             }
           });
@@ -680,7 +743,6 @@ struct Plan {
 #ifndef FRT_MIN_KB_PER_CLUSTER_SPLIT
 #define FRT_MIN_KB_PER_CLUSTER_SPLIT 2  // K-blocks per split of a cluster tile
 #endif
-constexpr int kMaxCluster = 8;  // portable cluster size
 
 Plan make_plan(int M, int N, int K, int epi) {
   Plan pl{};
