@@ -741,6 +741,23 @@ def run_gpu(args):
     torch.cuda.synchronize()
     assert frt.frt_device_status(True) == frt.FRT_OK
 
+    # The step is also captured once into a CUDA graph (its kernels keep their
+    # programmatic-dependent-launch edges); the timed loop replays it.
+    graph = None
+    if not args.no_graph:
+        cap = torch.cuda.Stream(device=dev)
+        cap.wait_stream(torch.cuda.current_stream())
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            runner.step()
+        torch.cuda.current_stream().wait_stream(cap)
+        for _ in range(3):
+            runner.reset()
+            graph.replay()
+        torch.cuda.synchronize()
+        assert frt.frt_device_status(True) == frt.FRT_OK
+    run_step = graph.replay if graph is not None else runner.step
+
     K = args.steps
     mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     s_ev = [(mk(), mk()) for _ in range(K)]
@@ -759,12 +776,34 @@ def run_gpu(args):
         flush.fill_(i & 0xFF)
         torch.cuda._sleep(sleep_cycles)
         s_ev[i][0].record()
-        runner.step()
+        run_step()
         s_ev[i][1].record()
     torch.cuda.synchronize()
     barrier()
     wall = time.perf_counter() - t_wall
     clk = clocks.stop()
+
+    # the same steps launched directly (no graph), for reference
+    d_ev = [(mk(), mk()) for _ in range(min(K, 200))]
+    for i in range(len(d_ev)):
+        runner.reset()
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(sleep_cycles)
+        d_ev[i][0].record()
+        runner.step()
+        d_ev[i][1].record()
+    # an empty kernel between the same events: the fixed event/launch cost
+    z = torch.zeros(1, device=dev)
+    z_ev = [(mk(), mk()) for _ in range(50)]
+    for i in range(len(z_ev)):
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(sleep_cycles)
+        z_ev[i][0].record()
+        z.add_(1)
+        z_ev[i][1].record()
+    torch.cuda.synchronize()
+    direct_us = 1e3 * sum(a.elapsed_time(b) for a, b in d_ev) / len(d_ev)
+    empty_us = 1e3 * sum(a.elapsed_time(b) for a, b in z_ev) / len(z_ev)
     assert frt.frt_device_status(True) == frt.FRT_OK
 
     step_ms = [a.elapsed_time(b) for a, b in s_ev]
@@ -856,7 +895,11 @@ def run_gpu(args):
                    "l2": "flushed before every timed step (256 MB write)",
                    "parallelism": "replicas" if world > 1 else "single",
                    "timing": "CUDA events per step on the launching stream; "
-                             "kernels timed alone the same way"},
+                             "step replayed from a CUDA graph"
+                             + (" (disabled)" if graph is None else "")
+                             + "; kernels timed alone the same way",
+                   "direct_launch_us_per_step": round(direct_us, 3),
+                   "empty_kernel_between_events_us": round(empty_us, 3)},
         "roofline": {"bound": kd.bound, "kernel": kd.name,
                      "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic,
@@ -888,6 +931,7 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="frt", choices=["frt", "reference"])
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:

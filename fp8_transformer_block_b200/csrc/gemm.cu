@@ -28,6 +28,7 @@
 // FRT_ETIMEOUT, the CTA drains its in-flight copies and MMAs (again bounded),
 // frees its TMEM and returns.  No TMA multicast is used anywhere.
 #include <mutex>
+#include <type_traits>
 
 #include "frt_common.cuh"
 #include "frt_sm100.cuh"
@@ -101,54 +102,67 @@ __device__ __forceinline__ void load32_bf16(const uint16_t* src, float (&f)[32])
   }
 }
 
-// One token row m, output columns n0 .. n0 + 7 (n0 % 8 == 0, inside one head):
-// the same arithmetic as epi_rows_chunk at 16-byte granularity.  The rope
-// and bias loads are issued by the caller before the accumulators arrive.
-__device__ __forceinline__ void epi_rows8(const GemmParams& p, const float (&v)[8], int m, int n0,
-                                          float alpha, const uint4& bias8, const uint4& rope8) {
-  float y[8];
-  if (p.bias) {
-    float b[8];
-    unpack8(bias8, b);
+// One token row m, output columns n0 .. n0 + W - 1 (W = 8 or 16, n0 % W == 0,
+// inside one head): the same arithmetic as epi_rows_chunk at 16-byte
+// granularity.  The rope and bias pieces are loaded by the caller before the
+// accumulators arrive.
+template <int W>
+__device__ __forceinline__ void epi_rows_w(const GemmParams& p, const float (&v)[W], int m, int n0,
+                                           float alpha, const uint4 (&bias8)[W / 8],
+                                           const uint4 (&rope8)[W / 8]) {
+  const int b = m / p.Mseq, s = m % p.Mseq;
+  const int h = n0 / p.hd, d00 = n0 % p.hd;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = bf2f(f2bf(__fadd_rn(__fmul_rn(v[j], alpha), b[j])));
-  } else {
+  for (int g = 0; g < W / 8; ++g) {
+    float y[8];
+    if (p.bias) {
+      float bb[8];
+      unpack8(bias8[g], bb);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = bf2f(f2bf(__fmul_rn(v[j], alpha)));
-  }
-  uint16_t* dst;
-  if (p.epi == EPI_BF16) {
-    dst = static_cast<uint16_t*>(p.out) + long(m) * p.ldo + n0;
-  } else {
-    const int b = m / p.Mseq, s = m % p.Mseq;
-    const int h = n0 / p.hd, d0 = n0 % p.hd;
-    if (h < p.hq + p.hkv) {
-      float r[8];
-      unpack8(rope8, r);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float c = r[2 * i], sn = r[2 * i + 1];
-        const float x0 = y[2 * i], x1 = y[2 * i + 1];
-        y[2 * i] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, sn));
-        y[2 * i + 1] = __fadd_rn(__fmul_rn(x0, sn), __fmul_rn(x1, c));
-      }
-      dst = h < p.hq ? p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d0
-                     : p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d0;
+      for (int j = 0; j < 8; ++j) y[j] = bf2f(f2bf(__fadd_rn(__fmul_rn(v[8 * g + j], alpha), bb[j])));
     } else {
-      const int hv = h - p.hq - p.hkv;
-      dst = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + hv) * p.hd + d0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[j] = bf2f(f2bf(__fmul_rn(v[8 * g + j], alpha)));
     }
+    uint16_t* dst;
+    if (p.epi == EPI_BF16) {
+      dst = static_cast<uint16_t*>(p.out) + long(m) * p.ldo + n0 + 8 * g;
+    } else {
+      const int d0 = d00 + 8 * g;
+      if (h < p.hq + p.hkv) {
+        float r[8];
+        unpack8(rope8[g], r);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float c = r[2 * i], sn = r[2 * i + 1];
+          const float x0 = y[2 * i], x1 = y[2 * i + 1];
+          y[2 * i] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, sn));
+          y[2 * i + 1] = __fadd_rn(__fmul_rn(x0, sn), __fmul_rn(x1, c));
+        }
+        dst = h < p.hq ? p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d0
+                       : p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d0;
+      } else {
+        const int hv = h - p.hq - p.hkv;
+        dst = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + hv) * p.hd + d0;
+      }
+    }
+    *reinterpret_cast<uint4*>(dst) = pack8_bf16(y);
   }
-  *reinterpret_cast<uint4*>(dst) = pack8_bf16(y);
 }
 
-// The rope pairs and bias an 8-column item needs (zeros when unused).
-__device__ __forceinline__ void epi_rows8_operands(const GemmParams& p, int m, int n0, uint4& bias8,
-                                                   uint4& rope8) {
-  bias8 = p.bias ? __ldg(reinterpret_cast<const uint4*>(p.bias + n0)) : make_uint4(0, 0, 0, 0);
-  rope8 = make_uint4(0, 0, 0, 0);
-  if (p.epi == EPI_ROPE && n0 / p.hd < p.hq + p.hkv)
-    rope8 = __ldg(reinterpret_cast<const uint4*>(p.rope + long(m % p.Mseq) * p.hd + n0 % p.hd));
+// The rope pairs and bias an item of W columns needs (zeros when unused).
+template <int W>
+__device__ __forceinline__ void epi_rows_w_operands(const GemmParams& p, int m, int n0,
+                                                    uint4 (&bias8)[W / 8], uint4 (&rope8)[W / 8]) {
+  const bool rot = p.epi == EPI_ROPE && n0 / p.hd < p.hq + p.hkv;
+#pragma unroll
+  for (int g = 0; g < W / 8; ++g) {
+    bias8[g] = p.bias ? __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * g))
+                      : make_uint4(0, 0, 0, 0);
+    rope8[g] = rot ? __ldg(reinterpret_cast<const uint4*>(p.rope + long(m % p.Mseq) * p.hd +
+                                                          n0 % p.hd + 8 * g))
+                   : make_uint4(0, 0, 0, 0);
+  }
 }
 
 // This thread owns token row m, output columns n0 .. n0 + 31 (the normal
@@ -237,28 +251,28 @@ __device__ __forceinline__ bool acc_row_valid(int lane) {
   return BMT == 128 || lane < 16;
 }
 
-// Swapped orientation, emitting half: the tile's (token, 8-column) items,
+// Swapped orientation, emitting half: the tile's (token, W-column) items,
 // numbered token-major so neighbouring threads write neighbouring 16-byte
 // pieces of one token row.  This thread takes items [lo, hi) with stride
-// 128 over the four epilogue warps.  fetch(m_local, c8, v) gathers the
-// item's 8 fp32 accumulators (output columns 8*c8 .. 8*c8+7 of token
+// 128 over the four epilogue warps.  fetch(m_local, cw, v) gathers the
+// item's W fp32 accumulators (output columns W*cw .. W*cw+W-1 of token
 // m_local); the item's rope and bias loads are issued before it.
-template <int BMT, int BN, class Fetch>
+template <int BMT, int BN, int W, class Fetch>
 __device__ __forceinline__ void emit_swap_items(const GemmParams& p, int ta, int tb, float alpha,
                                                 int lo, int hi, Fetch fetch) {
-  constexpr int C8 = BMT / 8;
+  constexpr int CW = BMT / W;
   const int t = int(threadIdx.x) - 64;  // 0 .. 127 over the four epilogue warps
 #pragma unroll 1
   for (int it = lo + t; it < hi; it += 128) {
-    const int m_local = it / C8, c8 = it % C8;
-    const int n0 = ta * BMT + 8 * c8;
+    const int m_local = it / CW, cw = it % CW;
+    const int n0 = ta * BMT + W * cw;
     const int m = tb * BN + m_local;
     if (n0 >= p.N || m >= p.M) continue;
-    uint4 bias8, rope8;
-    epi_rows8_operands(p, m, n0, bias8, rope8);
-    float v[8];
-    fetch(m_local, c8, v);
-    epi_rows8(p, v, m, n0, alpha, bias8, rope8);
+    uint4 bias8[W / 8], rope8[W / 8];
+    epi_rows_w_operands<W>(p, m, n0, bias8, rope8);
+    float v[W];
+    fetch(m_local, cw, v);
+    epi_rows_w<W>(p, v, m, n0, alpha, bias8, rope8);
   }
 }
 
@@ -313,8 +327,8 @@ __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int t
   }
   done();
   named_bar_sync(2, 128);
-  emit_swap_items<BMT, BN>(p, ta, tb, alpha, 0, BN * (BMT / 8),
-                           [&](int m_local, int c8, float (&v)[8]) {
+  emit_swap_items<BMT, BN, 8>(p, ta, tb, alpha, 0, BN * (BMT / 8),
+                              [&](int m_local, int c8, float (&v)[8]) {
     const float4* src = reinterpret_cast<const float4*>(T + m_local * TS + 8 * c8);
     const float4 a = src[0], b = src[1];
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
@@ -656,35 +670,46 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
       const uint32_t t_addr = smem_u32(T);
       constexpr int TS = BMT + 4;
-      // the ranks share the tile's items in contiguous ranges
-      constexpr int ITEMS = BN * (BMT / 8);
+      // the ranks share the tile's items in contiguous ranges; items of 16
+      // columns when that leaves at most one item per thread
       const int r = int(cluster_ctarank());
-      const int lo = r * ITEMS / p.splits, hi = (r + 1) * ITEMS / p.splits;
-      emit_swap_items<BMT, BN>(
-          p, ta, tb, alpha, lo, hi, [&](int m_local, int c8, float (&v)[8]) {
-            const uint32_t off = t_addr + uint32_t((m_local * TS + 8 * c8) * 4);
-            float4 f[2 * kMaxCluster];
+      auto reduce_emit = [&](auto wtag) {
+        constexpr int W = decltype(wtag)::value;
+        constexpr int ITEMS = BN * (BMT / W);
+        const int lo = r * ITEMS / p.splits, hi = (r + 1) * ITEMS / p.splits;
+        emit_swap_items<BMT, BN, W>(
+            p, ta, tb, alpha, lo, hi, [&](int m_local, int cw, float (&v)[W]) {
+              const uint32_t off = t_addr + uint32_t((m_local * TS + W * cw) * 4);
+              constexpr int Q = W / 4;  // float4 per rank
+              constexpr int RMAX = W == 16 ? 4 : kMaxCluster;
+              float4 f[RMAX * Q];
 #pragma unroll
-            for (int q2 = 0; q2 < kMaxCluster; ++q2) {
-              if (q2 < p.splits) {
-                const uint32_t a = map_cluster(off, uint32_t(q2));
-                f[2 * q2] = ld_cluster_f4(a);
-                f[2 * q2 + 1] = ld_cluster_f4(a + 16u);
+              for (int q2 = 0; q2 < RMAX; ++q2) {
+                if (q2 < p.splits) {
+                  const uint32_t a = map_cluster(off, uint32_t(q2));
+#pragma unroll
+                  for (int k = 0; k < Q; ++k) f[q2 * Q + k] = ld_cluster_f4(a + 16u * k);
+                }
               }
-            }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+              for (int j = 0; j < W; ++j) v[j] = 0.0f;
 #pragma unroll
-            for (int q2 = 0; q2 < kMaxCluster; ++q2) {
-              if (q2 < p.splits) {
-                const float4 a = f[2 * q2], b = f[2 * q2 + 1];
-                v[0] = __fadd_rn(v[0], a.x); v[1] = __fadd_rn(v[1], a.y);
-                v[2] = __fadd_rn(v[2], a.z); v[3] = __fadd_rn(v[3], a.w);
-                v[4] = __fadd_rn(v[4], b.x); v[5] = __fadd_rn(v[5], b.y);
-                v[6] = __fadd_rn(v[6], b.z); v[7] = __fadd_rn(v[7], b.w);
+              for (int q2 = 0; q2 < RMAX; ++q2) {
+                if (q2 < p.splits) {
+#pragma unroll
+                  for (int k = 0; k < Q; ++k) {
+                    const float4 a = f[q2 * Q + k];
+                    v[4 * k] = __fadd_rn(v[4 * k], a.x);
+                    v[4 * k + 1] = __fadd_rn(v[4 * k + 1], a.y);
+                    v[4 * k + 2] = __fadd_rn(v[4 * k + 2], a.z);
+                    v[4 * k + 3] = __fadd_rn(v[4 * k + 3], a.w);
+                  }
+                }
               }
-            }
-          });
+            });
+      };
+      if (p.splits <= 4) reduce_emit(std::integral_constant<int, 16>{});
+      else reduce_emit(std::integral_constant<int, 8>{});
     }
     cluster_sync_all();  // no rank leaves while another still reads its tile
   }
