@@ -704,6 +704,40 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- GPU arm --
 
+L2_BYTES = 126 << 20
+
+
+def _footprint(runner, torch):
+    """Device bytes a step of this runner reads or writes (its own tensors)."""
+    seen, total = set(), 0
+    for v in vars(runner).values():
+        ts = []
+        if isinstance(v, torch.Tensor):
+            ts = [v]
+        elif isinstance(v, (list, tuple)):
+            ts = [x for x in v if isinstance(x, torch.Tensor)]
+            for x in v:
+                if isinstance(x, dict):
+                    ts += [y for y in x.values() if isinstance(y, torch.Tensor)]
+                    pk = x.get("pk")
+                    if pk is not None:
+                        ts += [pk.w8]
+        elif hasattr(v, "w8"):
+            ts = [v.w8]
+        for t in ts:
+            if t.data_ptr() not in seen:
+                seen.add(t.data_ptr())
+                total += t.numel() * t.element_size()
+    return total
+
+
+def _smallest_divisor_at_least(K, r):
+    for d in range(max(1, r), K + 1):
+        if K % d == 0:
+            return d
+    return K
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -725,132 +759,138 @@ def run_gpu(args):
     from fp8_transformer_block_b200 import frt, synth
     from fp8_transformer_block_b200 import runtime as rt
 
-    runner = make_runner(args.config, torch, frt, rt, synth)
-    w = runner.w
-    L = getattr(runner, "L", 1)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    sleep_cycles = max(1_000_000, 300_000 * runner.launches)
-
     def barrier():
         if world > 1:
             dist.barrier()
 
-    for i in range(args.warmup):
-        runner.reset()
-        runner.step()
+    # ---- R independent copies of the workload (weights, inputs, caches), so
+    # that consecutive steps read data no earlier step left in L2: the
+    # copies together exceed 1.5x the L2 (or one copy already does)
+    first = make_runner(args.config, torch, frt, rt, synth)
+    w = first.w
+    L = getattr(first, "L", 1)
+    fp = _footprint(first, torch)
+    K = args.steps
+    r_min = 1 if fp >= 1.5 * L2_BYTES else -(-int(1.5 * L2_BYTES) // fp)
+    R = _smallest_divisor_at_least(K, min(r_min, K))
+    runners = [first] + [make_runner(args.config, torch, frt, rt, synth)
+                         for _ in range(R - 1)]
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        for r in runners:
+            r.step()
     torch.cuda.synchronize()
     assert frt.frt_device_status(True) == frt.FRT_OK
 
-    # The step is also captured once into a CUDA graph (its kernels keep their
-    # programmatic-dependent-launch edges); the timed loop replays it.
-    graph = None
-    if not args.no_graph:
+    def capture(calls):
         cap = torch.cuda.Stream(device=dev)
         cap.wait_stream(torch.cuda.current_stream())
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=cap):
-            runner.step()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for c in calls:
+                c()
         torch.cuda.current_stream().wait_stream(cap)
-        for _ in range(3):
-            runner.reset()
-            graph.replay()
-        torch.cuda.synchronize()
-        assert frt.frt_device_status(True) == frt.FRT_OK
-    run_step = graph.replay if graph is not None else runner.step
+        return g
 
-    K = args.steps
+    g_steps = capture([r.step for r in runners])
+    for _ in range(2):
+        g_steps.replay()
+    torch.cuda.synchronize()
+    assert frt.frt_device_status(True) == frt.FRT_OK
+
     mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    s_ev = [(mk(), mk()) for _ in range(K)]
     gpu_id = str(local)
     try:
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:  # noqa: BLE001
         pass
     clocks = ClockSampler(gpu_id)
+    reps = K // R
+    e0, e1 = mk(), mk()
     barrier()
     torch.cuda.synchronize()
     clocks.start()
     t_wall = time.perf_counter()
-    for i in range(K):
-        runner.reset()
-        flush.fill_(i & 0xFF)
-        torch.cuda._sleep(sleep_cycles)
-        s_ev[i][0].record()
-        run_step()
-        s_ev[i][1].record()
+    torch.cuda._sleep(2_000_000)   # hold the GPU while the replays queue
+    e0.record()
+    for _ in range(reps):
+        g_steps.replay()
+    e1.record()
     torch.cuda.synchronize()
     barrier()
     wall = time.perf_counter() - t_wall
     clk = clocks.stop()
-
-    # the same steps launched directly (no graph), for reference
-    d_ev = [(mk(), mk()) for _ in range(min(K, 200))]
-    for i in range(len(d_ev)):
-        runner.reset()
-        flush.fill_(i & 0xFF)
-        torch.cuda._sleep(sleep_cycles)
-        d_ev[i][0].record()
-        runner.step()
-        d_ev[i][1].record()
-    # an empty kernel between the same events: the fixed event/launch cost
-    z = torch.zeros(1, device=dev)
-    z_ev = [(mk(), mk()) for _ in range(50)]
-    for i in range(len(z_ev)):
-        flush.fill_(i & 0xFF)
-        torch.cuda._sleep(sleep_cycles)
-        z_ev[i][0].record()
-        z.add_(1)
-        z_ev[i][1].record()
-    torch.cuda.synchronize()
-    direct_us = 1e3 * sum(a.elapsed_time(b) for a, b in d_ev) / len(d_ev)
-    empty_us = 1e3 * sum(a.elapsed_time(b) for a, b in z_ev) / len(z_ev)
     assert frt.frt_device_status(True) == frt.FRT_OK
-
-    step_ms = [a.elapsed_time(b) for a, b in s_ev]
-    total_ms = sum(step_ms)
+    total_ms = e0.elapsed_time(e1)
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     max_total_ms = float(t.item())
     ms_per_step = max_total_ms / K
-    value = world * runner.tokens * K / (max_total_ms / 1e3)
+    value = world * first.tokens * K / (max_total_ms / 1e3)
 
-    # ---- each kernel alone (cold L2, GPU held until the launch is queued)
-    KK = max(20, min(K, 200))
-    kern_ms = []
-    for kd, call in runner.kernel_calls():
-        evs = [(mk(), mk()) for _ in range(KK)]
-        for i in range(KK):
-            runner.reset()
-            flush.fill_(i & 0xFF)
-            torch.cuda._sleep(1_000_000)
-            evs[i][0].record()
-            call()
-            evs[i][1].record()
+    # ---- each kernel alone, back to back over the same R copies
+    kinds, kern_ms = [], []
+    for kk in range(len(first.kernel_calls())):
+        calls = [r.kernel_calls()[kk][1] for r in runners]
+        kinds.append(first.kernel_calls()[kk][0])
+        gk = capture(calls)
+        gk.replay()
         torch.cuda.synchronize()
-        kern_ms.append(sum(a.elapsed_time(b) for a, b in evs) / KK)
-    kinds = [kd for kd, _ in runner.kernel_calls()]
+        a, b = mk(), mk()
+        torch.cuda._sleep(2_000_000)
+        a.record()
+        for _ in range(reps):
+            gk.replay()
+        b.record()
+        torch.cuda.synchronize()
+        kern_ms.append(a.elapsed_time(b) / (reps * R))
+        del gk
+
+    # ---- one step per event pair after an L2 flush (latency of an isolated
+    # step, with the fixed cost of an empty kernel between the same events)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    g_one = capture([first.step])
+    n_iso = min(K, 100)
+    iso = [(mk(), mk()) for _ in range(n_iso)]
+    z = torch.zeros(1, device=dev)
+    z_ev = [(mk(), mk()) for _ in range(n_iso)]
+    for i in range(n_iso):
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(1_000_000)
+        iso[i][0].record()
+        g_one.replay()
+        iso[i][1].record()
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(1_000_000)
+        z_ev[i][0].record()
+        z.add_(1)
+        z_ev[i][1].record()
+    torch.cuda.synchronize()
+    iso_us = 1e3 * sum(a.elapsed_time(b) for a, b in iso) / n_iso
+    empty_us = 1e3 * sum(a.elapsed_time(b) for a, b in z_ev) / n_iso
+    del g_one, g_steps
 
     # ---- e2e through the public entry points with host buffers
-    runner.e2e_setup()
+    first.e2e_setup()
     for _ in range(3):
-        runner.e2e_step()
+        first.e2e_step()
     torch.cuda.synchronize()
     KE = min(K, 200)
     e_ev = [(mk(), mk()) for _ in range(KE)]
     barrier()
     for i in range(KE):
         flush.fill_(i & 0xFF)
-        torch.cuda._sleep(sleep_cycles)
+        torch.cuda._sleep(1_000_000)
         e_ev[i][0].record()
-        runner.e2e_step()
+        first.e2e_step()
         e_ev[i][1].record()
     torch.cuda.synchronize()
     e_ms = sum(a.elapsed_time(b) for a, b in e_ev)
     te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * runner.tokens * KE / (float(te.item()) / 1e3)
+    e2e_value = world * first.tokens * KE / (float(te.item()) / 1e3)
 
     # ---- roofline of the dominant kernel (largest share of a step)
     hbm, bf16_burst, bf16_sust, src = _peaks()
@@ -881,6 +921,8 @@ def run_gpu(args):
         kern_list.append(e)
 
     if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
         return 0
     cpu = None
     if world == 1 and not args.no_cpu:
@@ -892,13 +934,16 @@ def run_gpu(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3/fp32", "data": "synthetic",
         "config": {"workload": workload_text(w),
-                   "l2": "flushed before every timed step (256 MB write)",
+                   "l2": (f"inputs larger than L2: {R} independent copies of "
+                          f"the workload ({R * fp / 2**20:.0f} MiB) rotated "
+                          "step by step" if R > 1 else
+                          f"inputs larger than L2 ({fp / 2**20:.0f} MiB per "
+                          "step)"),
                    "parallelism": "replicas" if world > 1 else "single",
-                   "timing": "CUDA events per step on the launching stream; "
-                             "step replayed from a CUDA graph"
-                             + (" (disabled)" if graph is None else "")
-                             + "; kernels timed alone the same way",
-                   "direct_launch_us_per_step": round(direct_us, 3),
+                   "timing": "K back-to-back steps replayed from CUDA graphs, "
+                             "CUDA events around the K steps on the launching "
+                             "stream; kernels timed the same way",
+                   "isolated_step_us_after_l2_flush": round(iso_us, 3),
                    "empty_kernel_between_events_us": round(empty_us, 3)},
         "roofline": {"bound": kd.bound, "kernel": kd.name,
                      "achieved": achieved, "peak": peak, "unit": unit,
@@ -911,9 +956,9 @@ def run_gpu(args):
         "kernels": kern_list,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s",
-                "h2d_bytes_per_step": int(runner.h2d_bytes),
-                "d2h_bytes_per_step": int(runner.d2h_bytes)},
-        "gpu_launches": runner.launches * K,
+                "h2d_bytes_per_step": int(first.h2d_bytes),
+                "d2h_bytes_per_step": int(first.d2h_bytes)},
+        "gpu_launches": first.launches * K,
         "clocks": clk,
         "wall_s_timed_loop": round(wall, 3),
     }
@@ -931,7 +976,6 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="frt", choices=["frt", "reference"])
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:
