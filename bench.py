@@ -847,28 +847,20 @@ def run_gpu(args):
         kern_ms.append(a.elapsed_time(b) / (reps * R))
         del gk
 
-    # ---- one step per event pair after an L2 flush (latency of an isolated
-    # step, with the fixed cost of an empty kernel between the same events)
+    # ---- one step per event pair after an L2 flush: the latency of an
+    # isolated step as a stream sees it (event and launch costs included)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     g_one = capture([first.step])
     n_iso = min(K, 100)
     iso = [(mk(), mk()) for _ in range(n_iso)]
-    z = torch.zeros(1, device=dev)
-    z_ev = [(mk(), mk()) for _ in range(n_iso)]
     for i in range(n_iso):
         flush.fill_(i & 0xFF)
         torch.cuda._sleep(1_000_000)
         iso[i][0].record()
         g_one.replay()
         iso[i][1].record()
-        flush.fill_(i & 0xFF)
-        torch.cuda._sleep(1_000_000)
-        z_ev[i][0].record()
-        z.add_(1)
-        z_ev[i][1].record()
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
     iso_us = 1e3 * sum(a.elapsed_time(b) for a, b in iso) / n_iso
-    empty_us = 1e3 * sum(a.elapsed_time(b) for a, b in z_ev) / n_iso
     del g_one, g_steps
 
     # ---- e2e through the public entry points with host buffers
@@ -943,8 +935,7 @@ def run_gpu(args):
                    "timing": "K back-to-back steps replayed from CUDA graphs, "
                              "CUDA events around the K steps on the launching "
                              "stream; kernels timed the same way",
-                   "isolated_step_us_after_l2_flush": round(iso_us, 3),
-                   "empty_kernel_between_events_us": round(empty_us, 3)},
+                   "isolated_step_us_after_l2_flush": round(iso_us, 3)},
         "roofline": {"bound": kd.bound, "kernel": kd.name,
                      "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic,
