@@ -1040,3 +1040,78 @@ extern "C" int frt_packed_fp8_gemm_rope_kvcache(
   return frt::run_gemm(pl, p, x8, w8, workspace, workspace_bytes,
                        static_cast<cudaStream_t>(stream));
 }
+
+// ------------------------------------------------- no-allocation variant --
+//
+// Some callers cannot allocate device memory for the split-K workspace:
+// plug-ins whose host engine owns every byte of device memory and forbids
+// allocation from inside the plug-in, real-time loops that must not enter
+// the CUDA allocator (cudaMalloc can synchronise the device), and code that
+// runs while a stream is being captured, where a fresh allocation cannot be
+// recorded.  frt_packed_fp8_gemm_noalloc serves them with a workspace that
+// lives in this file: a static device array of kNoAllocScratchBytes, which
+// every GPU that loads the library holds until the process exits.
+namespace frt {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name only stands in for the symbol; the address the kernels
+// need comes from cudaGetSymbolAddress, once per device, with that device
+// current (the first call on a device does this).
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(FRT_ECUDA, "no current CUDA device for the static scratch");
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(FRT_ECUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FRT_OK;
+}
+
+}  // namespace
+}  // namespace frt
+
+extern "C" int frt_packed_fp8_gemm_noalloc(int M, int N, int K, const frt_e4m3* x8,
+                                           const frt_e4m3* w8, const float* act_scale,
+                                           const float* w_scale, const frt_bf16* bias,
+                                           int epilogue, void* out, long ldo,
+                                           const float* out_scale, void* stream) {
+  frt::clear_error();
+  if (M > 0 && N > 0 && K > 0) {
+    const size_t need = frt_gemm_workspace_size(M, N, K, epilogue);
+    FRT_REQUIRE(need <= frt::kNoAllocScratchBytes, FRT_ERANGE,
+                "this shape needs %zu bytes of split-K workspace; the static scratch of "
+                "frt_packed_fp8_gemm_noalloc holds %zu (use frt_packed_fp8_gemm with a "
+                "caller workspace)",
+                need, frt::kNoAllocScratchBytes);
+    if (need > 0) {
+      void* ws = nullptr;
+      int rc = frt::noalloc_scratch(&ws);
+      if (rc) return rc;
+      // the split counters at the head of the workspace must start at zero;
+      // a completed call leaves them zero, an interrupted one might not
+      const size_t counters = (size_t(frt::make_plan(M, N, K, epilogue == FRT_EPI_GEGLU_E4M3
+                                                                   ? frt::EPI_GEGLU
+                                                                   : frt::EPI_BF16)
+                                            .counters_bytes));
+      if (counters > 0 &&
+          cudaMemsetAsync(ws, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return frt::fail(FRT_ECUDA, "clearing the static scratch counters");
+      return frt_packed_fp8_gemm(M, N, K, x8, w8, act_scale, w_scale, bias, epilogue, out, ldo,
+                                 out_scale, ws, need, stream);
+    }
+  }
+  return frt_packed_fp8_gemm(M, N, K, x8, w8, act_scale, w_scale, bias, epilogue, out, ldo,
+                             out_scale, nullptr, 0, stream);
+}

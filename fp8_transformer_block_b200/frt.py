@@ -82,6 +82,8 @@ _SIGS = {
     "frt_gemm_workspace_size": (_z, [_i, _i, _i, _i]),
     "frt_packed_fp8_gemm": (_i, [_i, _i, _i, _p, _p, _p, _p, _p, _i, _p, _l,
                                  _p, _p, _z, _p]),
+    "frt_packed_fp8_gemm_noalloc": (_i, [_i, _i, _i, _p, _p, _p, _p, _p, _i,
+                                         _p, _l, _p, _p]),
     "frt_packed_fp8_gemm_rope_kvcache": (_i, [_i, _i, _i, _i, _i, _i, _i, _i,
                                               _p, _p, _p, _p, _p, _p, _p, _p,
                                               _p, _p, _z, _p]),
@@ -180,6 +182,17 @@ def frt_packed_fp8_gemm(M, N, K, x8, w8, act_scale, w_scale, bias, epilogue,
         M, N, K, ptr(x8), ptr(w8), ptr(act_scale), ptr(w_scale), ptr(bias),
         epilogue, ptr(out), ldo, ptr(out_scale), ptr(workspace),
         workspace_bytes, _stream(stream)), "frt_packed_fp8_gemm")
+
+
+def frt_packed_fp8_gemm_noalloc(M, N, K, x8, w8, act_scale, w_scale, bias,
+                                epilogue, out, ldo, out_scale=None,
+                                stream=None):
+    """frt_packed_fp8_gemm without a workspace argument: for callers that
+    cannot allocate device memory (the library's static scratch is used)."""
+    return _check(_lib.frt_packed_fp8_gemm_noalloc(
+        M, N, K, ptr(x8), ptr(w8), ptr(act_scale), ptr(w_scale), ptr(bias),
+        epilogue, ptr(out), ldo, ptr(out_scale), _stream(stream)),
+        "frt_packed_fp8_gemm_noalloc")
 
 
 def frt_packed_fp8_gemm_rope_kvcache(B, M, K, hq, hkv, hd, P, T, x8, w8,

@@ -178,6 +178,28 @@ int frt_packed_fp8_gemm(int M, int N, int K, const frt_e4m3* x8,
                         size_t workspace_bytes, void* stream);
 
 /*
+ * frt_packed_fp8_gemm_noalloc -- frt_packed_fp8_gemm for callers that cannot
+ * allocate device memory (a plug-in whose host engine owns all device
+ * memory, a real-time loop that must not enter the CUDA allocator, code
+ * running while a stream is captured).  The pages have no counterpart; this
+ * is a convenience of this library.  Same arguments and results as
+ * frt_packed_fp8_gemm without the workspace: shapes whose split-K schedule
+ * needs a workspace use a static device array of 8 MiB that the library
+ * holds on every GPU that loads it, until the process exits.  Shapes that
+ * need more are rejected with FRT_ERANGE (nothing is launched).  The call
+ * allocates nothing.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress); make that first call before any
+ * stream capture.  Every call shares the one array and zeroes its split
+ * counters first: calls that may overlap on the GPU (other streams, other
+ * threads) race on it and must be serialised by the caller.
+ */
+int frt_packed_fp8_gemm_noalloc(int M, int N, int K, const frt_e4m3* x8,
+                                const frt_e4m3* w8, const float* act_scale,
+                                const float* w_scale, const frt_bf16* bias,
+                                int epilogue, void* out, long ldo,
+                                const float* out_scale, void* stream);
+
+/*
  * frt_packed_fp8_gemm_rope_kvcache -- the packed q/k/v GEMM with the split +
  * RoPE + KV write fused into its epilogue (qkv_pack/fp8_static.py joint
  * slots: q and k are one contiguous run consumed together; attention_core
