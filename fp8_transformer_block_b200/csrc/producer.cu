@@ -24,6 +24,7 @@
 // (when the chain passes a prefix) copy the cache prefix in the same grid.
 
 #include "frt_internal.cuh"
+#include "frt_sm100.cuh"
 
 namespace frt {
 namespace {
@@ -47,6 +48,7 @@ struct ProducerArgs {
   uint8_t* x8;
   uint16_t* gate_out;
   float* amax;
+  int* status;
   PrefixArgs pre;  // pre.units == 0: no prefix blocks
 };
 
@@ -264,6 +266,200 @@ __global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
   }
 }
 
+// ------------------------------------------------ staged (bandwidth) form --
+//
+// Many rows: persistent CTAs of 256 threads walk rows r = blockIdx.x,
+// + row_blocks, ...; thread 0 keeps the next kStages rows' streamed inputs
+// in flight as bulk copies into a shared-memory ring (one mbarrier per
+// stage), so HBM always has work queued while the CTA reduces and
+// quantizes the current row.  Same arithmetic as the register kernels.
+constexpr int kStagedThreads = 256;
+constexpr int kStages = 3;
+constexpr uint64_t kRowWaitNs = 2000000000ull;   // 2 s per wait
+constexpr uint64_t kRowDrainNs = 200000000ull;
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kStagedThreads / 32; ++i) s = __fadd_rn(s, red[i]);
+  return s;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kStagedThreads) producer_staged_kernel(ProducerArgs a) {
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ float red[kStagedThreads / 32];
+  constexpr int NS = MODE == FRT_NORM_LAYERNORM_TABLE ? 3 : 2;  // streamed inputs per row
+  pdl_trigger();
+  pdl_wait();
+  if (prefix_block(a)) return;
+  const int D = a.D, C = a.C, tid = threadIdx.x;
+  const uint32_t row_bytes = 2u * uint32_t(D);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * NS * row_bytes);
+  const long stride = a.row_blocks;
+
+  auto issue = [&](long r, int st) {
+    uint8_t* dst = ring + st * NS * row_bytes;
+    mbar_arrive_expect_tx(&full[st], NS * row_bytes);
+    if (MODE == FRT_NORM_LAYERNORM_TABLE) {
+      const uint16_t* tr = a.temb + r * long(a.chunks) * D;
+      bulk_load(dst, a.x + r * D, row_bytes, &full[st]);
+      bulk_load(dst + row_bytes, tr + long(a.shift_idx) * D, row_bytes, &full[st]);
+      bulk_load(dst + 2 * row_bytes, tr + long(a.scale_idx) * D, row_bytes, &full[st]);
+    } else {
+      bulk_load(dst, a.res + r * D, row_bytes, &full[st]);
+      bulk_load(dst + row_bytes, a.delta + r * D, row_bytes, &full[st]);
+    }
+  };
+  if (tid == 0) {
+    for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
+    fence_barrier_init();
+    for (int st = 0; st < kStages; ++st) {
+      const long r = blockIdx.x + st * stride;
+      if (r < a.rows) issue(r, st);
+    }
+  }
+  __syncthreads();
+
+  const float as = __ldg(a.act_scale);
+  float mx = 0.0f;
+  int k = 0;
+  bool aborted = false;
+  for (long r = blockIdx.x; r < a.rows; r += stride, ++k) {
+    const int st = k % kStages;
+    const bool got = mbar_wait_bounded(&full[st], uint32_t((k / kStages) & 1), kRowWaitNs,
+                                       nullptr);
+    if (!__syncthreads_and(got)) {
+      aborted = true;
+      break;
+    }
+    uint16_t* s0 = reinterpret_cast<uint16_t*>(ring + st * NS * row_bytes);
+    uint16_t* s1 = s0 + D;
+    if (MODE == FRT_NORM_ADARMS) {
+      // s0: residual row, s1: delta row
+      const uint16_t* gg = a.gate + r * a.gate_stride;
+      uint16_t* rr = a.res + r * D;
+      float ss = 0.0f;
+      for (int c = tid; c < C; c += kStagedThreads) {
+        float rv[8], dv[8], gv[8], h[8];
+        unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), rv);
+        unpack8(*reinterpret_cast<const uint4*>(s1 + 8 * c), dv);
+        unpack8(__ldg(reinterpret_cast<const uint4*>(gg + 8 * c)), gv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) h[j] = __fadd_rn(rv[j], __fmul_rn(gv[j], dv[j]));
+        const uint4 hb = pack8_bf16(h);
+        *reinterpret_cast<uint4*>(rr + 8 * c) = hb;
+        *reinterpret_cast<uint4*>(s0 + 8 * c) = hb;
+        float hf[8];
+        unpack8(hb, hf);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss = __fadd_rn(ss, __fmul_rn(hf[j], hf[j]));
+      }
+      ss = block_sum(ss, red);
+      const float ms = __fdiv_rn(ss, float(D));
+      const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
+      const uint16_t* sty = a.style + r * a.style_stride;
+      for (int c = tid; c < C; c += kStagedThreads) {
+        float hf[8], wv[8], sc[8], sh[8], q[8];
+        unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), hf);
+        if (a.weight) unpack8(__ldg(reinterpret_cast<const uint4*>(a.weight + 8 * c)), wv);
+        else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) wv[j] = 1.0f;
+        }
+        unpack8(__ldg(reinterpret_cast<const uint4*>(sty + 8 * c)), sc);
+        unpack8(__ldg(reinterpret_cast<const uint4*>(sty + D + 8 * c)), sh);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float v = __fmul_rn(hf[j], inv);
+          v = __fmul_rn(v, wv[j]);
+          v = __fmul_rn(v, __fadd_rn(1.0f, sc[j]));
+          const float y = __fadd_rn(v, sh[j]);
+          mx = fmaxf(mx, fabsf(y));
+          q[j] = __fdiv_rn(y, as);
+        }
+        *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
+        if (a.gate_out)
+          *reinterpret_cast<uint4*>(a.gate_out + r * D + 8 * c) =
+              __ldg(reinterpret_cast<const uint4*>(sty + 2 * D + 8 * c));
+      }
+    } else {
+      // s0: x row, s1: shift chunk of temb, s2: scale chunk of temb
+      const uint16_t* s2 = s1 + D;
+      float sum = 0.0f;
+      for (int c = tid; c < C; c += kStagedThreads) {
+        float xv[8];
+        unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), xv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sum = __fadd_rn(sum, xv[j]);
+      }
+      sum = block_sum(sum, red);
+      const float mu = __fdiv_rn(sum, float(D));
+      float sq = 0.0f;
+      for (int c = tid; c < C; c += kStagedThreads) {
+        float xv[8];
+        unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), xv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float d = __fsub_rn(xv[j], mu);
+          sq = __fadd_rn(sq, __fmul_rn(d, d));
+        }
+      }
+      sq = block_sum(sq, red);
+      const float var = __fdiv_rn(sq, float(D));
+      const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
+      const float* bsh = a.table + long(a.shift_idx) * D;
+      const float* bsc = a.table + long(a.scale_idx) * D;
+      for (int c = tid; c < C; c += kStagedThreads) {
+        float xv[8], esh[8], esc[8], q[8];
+        unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), xv);
+        unpack8(*reinterpret_cast<const uint4*>(s1 + 8 * c), esh);
+        unpack8(*reinterpret_cast<const uint4*>(s2 + 8 * c), esc);
+        const float4 h0 = __ldg(reinterpret_cast<const float4*>(bsh + 8 * c));
+        const float4 h1 = __ldg(reinterpret_cast<const float4*>(bsh + 8 * c + 4));
+        const float4 c0 = __ldg(reinterpret_cast<const float4*>(bsc + 8 * c));
+        const float4 c1 = __ldg(reinterpret_cast<const float4*>(bsc + 8 * c + 4));
+        const float tsh8[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        const float tsc8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float shift = __fadd_rn(tsh8[j], esh[j]);
+          const float scale = __fadd_rn(tsc8[j], esc[j]);
+          float v = __fmul_rn(__fsub_rn(xv[j], mu), inv);
+          v = __fmul_rn(v, __fadd_rn(1.0f, scale));
+          const float y = __fadd_rn(v, shift);
+          mx = fmaxf(mx, fabsf(y));
+          q[j] = __fdiv_rn(y, as);
+        }
+        *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
+      }
+    }
+    __syncthreads();  // every thread is done with this stage
+    if (tid == 0) {
+      const long rn = r + kStages * stride;
+      if (rn < a.rows) issue(rn, st);
+    }
+  }
+  if (aborted && tid == 0) {
+    if (a.status) atomicExch(a.status, FRT_ETIMEOUT);
+    // drain the copies still in flight (bounded)
+    for (int j = 0; j < kStages; ++j) {
+      const long r = blockIdx.x + long(k + j) * stride;
+      if (r >= a.rows) break;
+      mbar_wait_bounded(&full[(k + j) % kStages], uint32_t(((k + j) / kStages) & 1), kRowDrainNs,
+                        nullptr);
+    }
+  }
+  if (a.amax) {
+    mx = warp_max(mx);
+    if ((threadIdx.x & 31) == 0) atomic_max_nonneg(a.amax, mx);
+  }
+}
+
 }  // namespace
 
 int producer_call(int mode, int rows, int D, float eps, uint16_t* res, const uint16_t* delta,
@@ -315,8 +511,36 @@ int producer_call(int mode, int rows, int D, float eps, uint16_t* res, const uin
   a.shift_idx = shift_idx; a.scale_idx = scale_idx;
   a.act_scale = act_scale; a.x8 = x8_out; a.gate_out = gate_out; a.amax = amax_out;
   if (pre) a.pre = *pre;
-  int vpt;
+  a.status = device_status_ptr();
   const int sms = num_sms();
+  const int ns = mode == FRT_NORM_LAYERNORM_TABLE ? 3 : 2;
+  const size_t staged_smem = size_t(3) * ns * 2 * D + 64;
+  if (rows > 2 * sms && staged_smem <= 72 * 1024) {
+    // bandwidth regime: persistent CTAs with a bulk-copy row ring
+    auto kern = mode == FRT_NORM_ADARMS ? producer_staged_kernel<FRT_NORM_ADARMS>
+                                        : producer_staged_kernel<FRT_NORM_LAYERNORM_TABLE>;
+    if (first_use(reinterpret_cast<const void*>(kern)) &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             72 * 1024 + 64) != cudaSuccess)
+      return fail(FRT_ECUDA, "cudaFuncSetAttribute(producer smem)");
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kStagedThreads,
+                                                      staged_smem) != cudaSuccess ||
+        per_sm < 1) {
+      cudaGetLastError();
+      per_sm = 1;
+    }
+    a.row_blocks = rows < sms * per_sm ? rows : sms * per_sm;
+    const int block = kStagedThreads;
+    int pre_blocks = 0;
+    if (pre_units > 0) {
+      const long need = (pre_units + block - 1) / block;
+      pre_blocks = int(need < 2L * sms ? need : 2L * sms);
+    }
+    const dim3 grid(a.row_blocks + pre_blocks);
+    return launch_pdl("producer_staged_kernel", kern, grid, dim3(block), staged_smem, s, a);
+  }
+  int vpt;
   if (rows <= 2 * sms) {  // latency regime: many threads per row
     vpt = a.C <= 512 ? 1 : a.C <= 1024 ? 2 : 4;
     a.G = ((a.C + vpt - 1) / vpt + 31) / 32 * 32;

@@ -51,18 +51,22 @@ def _oracle_layer(w, inp, a, pk_ref, prefix, style=None):
     return pr, q, kc, vc
 
 
-@pytest.mark.parametrize("name", ["tiny_adarms", "vla_action_expert"])
+@pytest.mark.parametrize("name", ["tiny_adarms", "vla_action_expert",
+                                  "adarms_stack18:512"])
 @pytest.mark.parametrize("fused", [True, False])
 def test_chain_layer_adarms(rt, name, fused):
+    """One chain layer; the 512-token case runs the producer's streaming
+    (bulk-copy ring) form with the prefix copy in the same launch."""
     frt, runtime, torch = rt
-    w = synth.WORKLOADS[name]
+    base, _, m = name.partition(":")
+    w = synth.WORKLOADS[base].with_M(int(m)) if m else synth.WORKLOADS[base]
     inp = synth.adarms_inputs(w.rows, w.D, w.seed, outliers=w.outliers)
     a = calibrate_adarms(w)
     ws, _ = synth.qkv_weights(w.hq, w.hkv, w.hd, w.D, w.seed)
     pk_ref = oracle.pack_weights_fp8(ws, layout=1, hd=w.hd)
     prefix = None
     if w.P > 0:
-        prefix = synth.prefix_cache(w.B, w.hkv, 1024, w.hd, w.seed)
+        prefix = synth.prefix_cache(w.B, w.hkv, max(1024, w.P), w.hd, w.seed)
     pr, qr, kr, vr = _oracle_layer(w, inp, a, pk_ref, prefix)
 
     pk = runtime.pack(ws, layout=frt.FRT_PACK_QK_INTERLEAVE, hd=w.hd)
@@ -86,7 +90,8 @@ def test_chain_layer_adarms(rt, name, fused):
         w_scale=pk.w_scale, rope=rope, q_out=q, k_cache=kc, v_cache=vc,
         prefix_k=None if prefix is None else runtime.bf16_dev(prefix[0]),
         prefix_v=None if prefix is None else runtime.bf16_dev(prefix[1]),
-        prefix_T_src=0 if prefix is None else 1024, prefix_interleave=1,
+        prefix_T_src=0 if prefix is None else prefix[0].shape[2],
+        prefix_interleave=1,
         qkv=qkv)
     wsb = frt.frt_chain_workspace_size(d)
     wsp = runtime.workspace(wsb)
