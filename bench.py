@@ -812,10 +812,12 @@ def run_gpu(args):
     clocks.start()
     t_wall = time.perf_counter()
     torch.cuda._sleep(2_000_000)   # hold the GPU while the replays queue
+    torch.cuda.nvtx.range_push("timed_steps")
     e0.record()
     for _ in range(reps):
         g_steps.replay()
     e1.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     barrier()
     wall = time.perf_counter() - t_wall
@@ -839,10 +841,12 @@ def run_gpu(args):
         torch.cuda.synchronize()
         a, b = mk(), mk()
         torch.cuda._sleep(2_000_000)
+        torch.cuda.nvtx.range_push(f"kernel_{kinds[-1].name}")
         a.record()
         for _ in range(reps):
             gk.replay()
         b.record()
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
         kern_ms.append(a.elapsed_time(b) / (reps * R))
         del gk
