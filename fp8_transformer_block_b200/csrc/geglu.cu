@@ -19,7 +19,7 @@ __global__ void geglu_kernel(int M, int H, const uint16_t* gu, long ld, const fl
   const long total = long(M) * h8;
   pdl_trigger();
   pdl_wait();
-  const float os = __ldg(out_scale);
+  const float inv_os = __frcp_rn(__ldg(out_scale));  // quantize: h * (1 / scale)
   float mx = 0.0f;
   for (long g = blockIdx.x * long(blockDim.x) + threadIdx.x; g < total;
        g += long(gridDim.x) * blockDim.x) {
@@ -32,7 +32,7 @@ __global__ void geglu_kernel(int M, int H, const uint16_t* gu, long ld, const fl
     for (int j = 0; j < 8; ++j) {
       const float h = gelu_tanh_mul(gv[j], uv[j]);
       mx = fmaxf(mx, fabsf(h));
-      q[j] = __fdiv_rn(h, os);
+      q[j] = __fmul_rn(h, inv_os);
     }
     *reinterpret_cast<uint2*>(hid8 + m * H + 8 * c) = pack8_e4m3(q);
   }

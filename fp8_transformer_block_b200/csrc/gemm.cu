@@ -219,13 +219,13 @@ __device__ __forceinline__ void epi_geglu_chunk(const GemmParams& p, const float
                                                 const float (&u)[32], int m, int n_gate0,
                                                 int n_up0, int out_col0, float alpha) {
   if (m >= p.M) return;
-  const float os = __ldg(p.out_scale);
+  const float inv_os = __frcp_rn(__ldg(p.out_scale));
   float q[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     const float gv = scale_bias_bf16(g[j], alpha, p.bias, n_gate0 + j);
     const float uv = scale_bias_bf16(u[j], alpha, p.bias, n_up0 + j);
-    q[j] = __fdiv_rn(gelu_tanh_mul(gv, uv), os);
+    q[j] = __fmul_rn(gelu_tanh_mul(gv, uv), inv_os);
   }
   uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + long(m) * p.ldo + out_col0);
 #pragma unroll

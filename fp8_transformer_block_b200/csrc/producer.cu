@@ -18,8 +18,10 @@
 // threads (VPT = 1); many rows use VPT = 4.  G == 32 packs 4 rows per block;
 // larger G uses one row per block and a shared-memory cross-warp reduction.
 // Arithmetic is fp32 with explicitly rounded operations (no contraction into
-// FMA), IEEE division and square root, so the only difference from a
-// sequential evaluation is the order of the row sums.
+// FMA), IEEE division and square root for the row statistics; the quantizer
+// multiplies by the correctly rounded fp32 reciprocal of the static scale
+// (y * (1/s) and y / s differ by at most an ulp or two, which changes a code
+// only when y / s sits that close to a rounding midpoint).
 // Launched with programmatic dependent launch; blocks past the row blocks
 // (when the chain passes a prefix) copy the cache prefix in the same grid.
 
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(512) adarms_kernel(ProducerArgs a) {
   if (!ok) return;
   const float ms = __fdiv_rn(ss, float(D));
   const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
-  const float as = __ldg(a.act_scale);
+  const float inv_as = __frcp_rn(__ldg(a.act_scale));  // quantize: y * (1 / scale)
   const uint16_t* st = a.style + r * a.style_stride;
   float mx = 0.0f;
 #pragma unroll
@@ -154,7 +156,7 @@ __global__ void __launch_bounds__(512) adarms_kernel(ProducerArgs a) {
         v = __fmul_rn(v, __fadd_rn(1.0f, sc[j]));
         const float y = __fadd_rn(v, sh[j]);
         mx = fmaxf(mx, fabsf(y));
-        q[j] = __fdiv_rn(y, as);
+        q[j] = __fmul_rn(y, inv_as);
       }
       *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
       if (a.gate_out)
@@ -229,7 +231,7 @@ __global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
   if (!ok) return;
   const float var = __fdiv_rn(sq, float(D));
   const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
-  const float as = __ldg(a.act_scale);
+  const float inv_as = __frcp_rn(__ldg(a.act_scale));  // quantize: y * (1 / scale)
   const float* bsh = a.table + long(a.shift_idx) * D;
   const float* bsc = a.table + long(a.scale_idx) * D;
   float mx = 0.0f;
@@ -255,7 +257,7 @@ __global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
         v = __fmul_rn(v, __fadd_rn(1.0f, scale));
         const float y = __fadd_rn(v, shift);
         mx = fmaxf(mx, fabsf(y));
-        q[j] = __fdiv_rn(y, as);
+        q[j] = __fmul_rn(y, inv_as);
       }
       *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
     }
@@ -325,7 +327,7 @@ __global__ void __launch_bounds__(kStagedThreads) producer_staged_kernel(Produce
   }
   __syncthreads();
 
-  const float as = __ldg(a.act_scale);
+  const float inv_as = __frcp_rn(__ldg(a.act_scale));  // quantize: y * (1 / scale)
   float mx = 0.0f;
   int k = 0;
   bool aborted = false;
@@ -380,7 +382,7 @@ __global__ void __launch_bounds__(kStagedThreads) producer_staged_kernel(Produce
           v = __fmul_rn(v, __fadd_rn(1.0f, sc[j]));
           const float y = __fadd_rn(v, sh[j]);
           mx = fmaxf(mx, fabsf(y));
-          q[j] = __fdiv_rn(y, as);
+          q[j] = __fmul_rn(y, inv_as);
         }
         *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
         if (a.gate_out)
@@ -433,7 +435,7 @@ __global__ void __launch_bounds__(kStagedThreads) producer_staged_kernel(Produce
           v = __fmul_rn(v, __fadd_rn(1.0f, scale));
           const float y = __fadd_rn(v, shift);
           mx = fmaxf(mx, fabsf(y));
-          q[j] = __fdiv_rn(y, as);
+          q[j] = __fmul_rn(y, inv_as);
         }
         *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
       }

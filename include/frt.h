@@ -96,7 +96,9 @@ enum { FRT_NORM_ADARMS = 0, FRT_NORM_LAYERNORM_TABLE = 1 };
  * static calibration of fp8_chain.py `bind_adarms_fp8_chain`).
  * Requires 8 <= D <= 16384, D % 8 == 0, 16-byte aligned bf16 pointers and
  * row strides that are multiples of 8, x8_out 8-byte aligned.  rows == 0 is
- * a no-op.  All arithmetic fp32; divisions and square roots IEEE-rounded.
+ * a no-op.  All arithmetic fp32; the row statistics use IEEE-rounded
+ * division and square root; the quantizer multiplies y by the fp32
+ * reciprocal of act_scale.
  */
 int frt_ada_norm_quant_fp8(int mode, int rows, int D, float eps,
                            frt_bf16* res, const frt_bf16* delta,
@@ -159,7 +161,7 @@ size_t frt_gemm_workspace_size(int M, int N, int K, int epilogue);
  *   FRT_EPI_GEGLU_E4M3 (fp8_chain.py `down_project`, the merged GEGLU +
  *   requant kernel): w8 packed with FRT_PACK_GATE_UP_BLOCKS; with
  *   g, u = bf16(acc * alpha + bias) of matching gate/up columns,
- *                  out[m, j] = e4m3(gelu_tanh(g) * u / out_scale)
+ *                  out[m, j] = e4m3(gelu_tanh(g) * u * (1 / out_scale))
  *                  out: [M, ldo] e4m3, ldo >= N / 2; N % 256 == 0.
  * x8: [M, K] e4m3; w8: [N, K] e4m3; bias: [N] bf16 or NULL.
  * Requires K % 16 == 0, N % 32 == 0, 16-byte aligned x8/w8/out/bias, ldo %
@@ -266,7 +268,7 @@ int frt_prefix_copy_kv(int B, int hkv, int hd, int P, int T, int T_src,
  * frt_geglu_quant_fp8 (fp8_chain.py `down_project`; tanh-GELU required by
  * `bind_adarms_fp8_chain`): gu [M, 2H] bf16 (gate in columns [0, H), up in
  * [H, 2H)), row stride ld_gu elements;
- *   hid8[m, j] = e4m3(gelu_tanh(g) * u / out_scale),
+ *   hid8[m, j] = e4m3(gelu_tanh(g) * u * (1 / out_scale)) (fp32 reciprocal),
  *   gelu_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
  * hid8: [M, H].  amax_out: NULL or zeroed device fp32 [1] raised to
  * max |gelu_tanh(g) * u| (calibration).  H % 8 == 0.
