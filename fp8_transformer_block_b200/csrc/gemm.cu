@@ -722,6 +722,225 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   }
 }
 
+// ------------------------------------------------------- CTA-pair kernel --
+//
+// Normal orientation, tiles of 256 rows x BN columns per CTA pair (a
+// cluster of 2): each CTA loads its 128 rows of x8 and BN/2 rows of w8 per
+// K-block, the even CTA issues tcgen05.mma.cta_group::2 (M = 256, N = BN)
+// over both CTAs' shared memory, and each CTA's epilogue drains its own 128
+// accumulator rows from its own TMEM.  Per K-block an SM moves 16 KB +
+// BN*64 B instead of 16 KB + BN*128 B for the same MMA work, so the same
+// shared-memory ring hides more latency.
+//   full[s]   (even CTA) 2 arrivals: each CTA's producer arms its bytes;
+//             both CTAs' TMA loads complete on it
+//   empty[s]  (each CTA) released by the even CTA's multicast commit
+//   tfull[b]  (each CTA) accumulator b ready, multicast commit
+//   tempty[b] (even CTA) 8 arrivals: the four epilogue warps of each CTA
+// All waits are bounded; a final cluster barrier keeps both CTAs (their
+// shared memory and TMEM) alive until the pair is done.
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const GemmParams p) {
+  constexpr int A_BYTES = 128 * BK;
+  constexpr int B_BYTES = (BN / 2) * BK;
+  constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * BN);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* epi_ok = abort_flag + 2;  // [4]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool lead = rank == 0;
+  const int pair = int(blockIdx.x >> 1), npairs = int(gridDim.x >> 1);
+  pdl_trigger();
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 2);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint32_t full_lead = map_cluster(smem_u32(full), 0);
+  const uint32_t tempty_lead = map_cluster(smem_u32(tempty), 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      const int u0 = pair;
+      int n_pre = 0;
+      if (u0 < p.units) {  // weights first, before the dependency wait
+        const int tn = u0 / p.a_tiles;
+        n_pre = p.k_blocks < STAGES ? p.k_blocks : STAGES;
+        for (int i = 0; i < n_pre; ++i) {
+          mbar_arrive_expect_tx_cluster(full_lead + 8u * i, A_BYTES + B_BYTES);
+          tma_load_2d_pair(sB + i * B_BYTES, &tmB, full_lead + 8u * i, i * BK,
+                           tn * BN + int(rank) * (BN / 2));
+        }
+      }
+      pdl_wait();
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = u0; u < p.units && ok; u += npairs) {
+        const int tm = u % p.a_tiles, tn = u / p.a_tiles;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          const bool pre = (u == u0) && (kb < n_pre);
+          if (!pre) {
+            if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitNs, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx_cluster(full_lead + 8u * stage, A_BYTES + B_BYTES);
+            tma_load_2d_pair(sB + stage * B_BYTES, &tmB, full_lead + 8u * stage, kb * BK,
+                             tn * BN + int(rank) * (BN / 2));
+          }
+          tma_load_2d_pair(sA + stage * A_BYTES, &tmA, full_lead + 8u * stage, kb * BK,
+                           tm * 256 + int(rank) * 128);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        record_timeout(p.status);
+        *abort_flag = 1;
+        if (lead) {  // the even CTA's barriers count both CTAs' copies
+          int st = stage;
+          uint32_t ph = phase;
+          for (int i = 0; i < issued && i < STAGES; ++i) {
+            if (--st < 0) { st = STAGES - 1; ph ^= 1u; }
+            mbar_wait_bounded(&full[st], ph, kDrainNs, nullptr);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------ MMA issuer (even CTA) --
+    if (lane == 0 && lead) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(256, BN);
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      int stage = 0, local = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = pair; u < p.units && ok; u += npairs, ++local) {
+        const int ab = local & 1;
+        const uint32_t aph = (local >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[ab], aph ^ 1u, kWaitNs, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dcol = tmem_base + uint32_t(ab * BN);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, kWaitNs, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = sdesc_k_sw128(a_base + stage * A_BYTES);
+          const uint64_t bd = sdesc_k_sw128(b_base + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            umma_pair_e4m3(dcol, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          umma_pair_commit(&empty[stage], 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_pair_commit(&tfull[ab], 0x3);
+      }
+      if (!ok) {
+        record_timeout(p.status);
+        *abort_flag = 1;
+        umma_pair_commit(drain, 0x1);
+        mbar_wait_bounded(drain, 0, kDrainNs, nullptr);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ----------------------------------------------------------- epilogue --
+    pdl_wait();
+    const int q = warp & 3;
+    const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
+    int local = 0;
+    for (int u = pair; u < p.units; u += npairs, ++local) {
+      const int tm = u % p.a_tiles, tn = u / p.a_tiles;
+      const int ab = local & 1;
+      const uint32_t aph = (local >> 1) & 1;
+      const bool got = __all_sync(0xffffffffu,
+                                  mbar_wait_bounded(&tfull[ab], aph, kWaitNs, abort_flag));
+      if (lane == 0) epi_ok[q] = got ? 1 : 0;
+      named_bar_sync(1, 128);
+      const bool all_ok = epi_ok[0] && epi_ok[1] && epi_ok[2] && epi_ok[3];
+      named_bar_sync(1, 128);
+      if (!all_ok) {
+        if (lane == 0) record_timeout(p.status);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + uint32_t(ab * BN) + (uint32_t(32 * q) << 16);
+      auto load = [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); };
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_lead + 8u * ab);
+      };
+      const int m = tm * 256 + int(rank) * 128 + 32 * q + lane;
+      if (p.epi == EPI_GEGLU) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float g[32], uu[32];
+          load(c, g);
+          load(c + 4, uu);
+          if (c == 3) release();
+          epi_geglu_chunk(p, g, uu, m, tn * BN + 32 * c, tn * BN + 128 + 32 * c,
+                          tn * 128 + 32 * c, alpha);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          load(c, v);
+          if (c == BN / 32 - 1) release();
+          epi_rows_chunk(p, v, m, tn * BN + 32 * c, alpha);
+        }
+      }
+    }
+  }
+
+  cluster_sync_all();  // the pair is done with both CTAs' memory
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // -------------------------------------------------------------------- host --
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -760,7 +979,7 @@ int make_map(CUtensorMap* m, const void* ptr, long rows, int K, int box_rows) {
 }
 
 struct Plan {
-  bool swap, cluster;
+  bool swap, cluster, pair;
   int bmt, bn, a_tiles, b_tiles, k_blocks, splits, units, grid;
   size_t counters_bytes, ws_bytes;
 };
@@ -773,14 +992,37 @@ Plan make_plan(int M, int N, int K, int epi) {
   Plan pl{};
   pl.k_blocks = (K + BK - 1) / BK;
   pl.bmt = 128;
-  if (epi == EPI_GEGLU) { pl.swap = false; pl.bn = 256; }
-  else if (M <= 128) { pl.swap = true; pl.bmt = 64; pl.bn = M <= 64 ? 64 : 128; }
+  if (epi != EPI_GEGLU && M <= 128) { pl.swap = true; pl.bmt = 64; pl.bn = M <= 64 ? 64 : 128; }
   else {
     pl.swap = false;
     pl.bn = (N % 256 == 0) ? 256 : 128;
     // narrower tiles before splitting K when 256-wide tiles underfill the SMs
+    // (a GEGLU tile keeps its gate and up halves together: always 256 wide)
     const long t256 = ((M + 127L) / 128) * ((N + 255L) / 256);
-    if (pl.bn == 256 && t256 < num_sms()) pl.bn = 128;
+    if (epi != EPI_GEGLU && pl.bn == 256 && t256 < num_sms()) pl.bn = 128;
+    // CTA pairs (256-row tiles, half the B tile per SM) when they keep at
+    // least as many SMs busy as single-CTA tiles would
+    const int sms = num_sms();
+    const long tiles1 = ((M + 127L) / 128) * ((N + pl.bn - 1L) / pl.bn);
+    const long ctas1 = tiles1 < sms ? tiles1 : sms;
+    const long mt2 = (M + 255L) / 256;
+    int bn2 = 0;
+    if (N % 256 == 0 && (epi == EPI_GEGLU || 2 * mt2 * (N / 256) >= ctas1)) bn2 = 256;
+    else if (epi != EPI_GEGLU && N % 128 == 0) bn2 = 128;
+    if (M >= 256 && bn2) {
+      const long units2 = mt2 * (N / bn2);
+      const long pairs = units2 < sms / 2 ? units2 : sms / 2;
+      if (2 * pairs >= ctas1 && units2 >= 16) {
+        pl.pair = true;
+        pl.bn = bn2;
+        pl.a_tiles = int(mt2);
+        pl.b_tiles = int(N / bn2);
+        pl.splits = 1;
+        pl.units = int(units2);
+        pl.grid = int(2 * pairs);
+        return pl;
+      }
+    }
   }
   const long a_rows = pl.swap ? N : M, b_rows = pl.swap ? M : N;
   pl.a_tiles = int((a_rows + pl.bmt - 1) / pl.bmt);
@@ -922,6 +1164,41 @@ int launch_swap(Plan pl, const CUtensorMap& ta, const CUtensorMap& tb, GemmParam
   return launch_t<true, BMT, BN, STAGES>(pl, ta, tb, p, s);
 }
 
+template <int BN, int STAGES>
+int launch_pair(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+                cudaStream_t s) {
+  constexpr int smem = STAGES * (128 * BK + (BN / 2) * BK) + 1024 + 256;
+  static_assert(smem <= 232448, "shared memory budget");
+  auto kern = gemm_pair_kernel<BN, STAGES>;
+  if (first_use(reinterpret_cast<const void*>(kern))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return fail(FRT_ECUDA, "cudaFuncSetAttribute(max dynamic smem %d)", smem);
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FRT_ECUDA, "gemm_pair_kernel: %s", cudaGetErrorString(e));
+  }
+  return FRT_OK;
+}
+
 int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void* workspace,
              size_t workspace_bytes, cudaStream_t s) {
   if (pl.ws_bytes > 0) {
@@ -939,6 +1216,12 @@ int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void
   p.status = device_status_ptr();
   CUtensorMap ta, tb;
   int rc;
+  if (pl.pair) {  // each CTA loads 128 rows of x8 and BN/2 rows of w8
+    if ((rc = make_map(&ta, x8, p.M, p.K, 128))) return rc;
+    if ((rc = make_map(&tb, w8, p.N, p.K, pl.bn / 2))) return rc;
+    if (pl.bn == 256) return launch_pair<256, 6>(pl, ta, tb, p, s);
+    return launch_pair<128, 8>(pl, ta, tb, p, s);
+  }
   if (!pl.swap) {
     if ((rc = make_map(&ta, x8, p.M, p.K, BM))) return rc;
     if ((rc = make_map(&tb, w8, p.N, p.K, pl.bn))) return rc;

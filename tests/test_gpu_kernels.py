@@ -185,6 +185,11 @@ GEMM_CASES = [
     (64, 2048, 16384, False),      # long K: K split in a 4-CTA cluster
     (100, 1024, 4096, True),       # 8-CTA clusters, ragged token tile
     (200, 256, 16384, True),       # 128-row tiles, K split via workspace
+    # CTA pairs (256-row tiles over two SMs)
+    (300, 4096, 528, True),        # BN = 128; the odd CTA of the last pair
+                                   # holds rows past M only; K tail
+    (1100, 4096, 1024, True),      # BN = 256, ragged last 256-row tile
+    (2048, 4096, 512, False),      # several tiles per pair, K < ring depth
 ]
 
 
@@ -349,7 +354,7 @@ def test_geglu_standalone_parity(rt):
     assert abs(float(am.item()) - amax) <= 1e-5 * amax
 
 
-@pytest.mark.parametrize("M", [64, 300])
+@pytest.mark.parametrize("M", [64, 300, 1100])
 def test_geglu_fused_epilogue(rt, M):
     frt, runtime, torch = rt
     D, H = 512, 1024
