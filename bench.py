@@ -31,7 +31,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -79,58 +78,69 @@ def _peaks():
 # ---------------------------------------------------------------- clocks ----
 
 class ClockSampler:
-    """nvidia-smi samples of the SM clock and throttle reasons while the
-    timed region runs."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """NVML samples of the SM clock and the clock-event (throttle) reasons,
+    taken every millisecond by a thread while the timed region runs (the
+    region is a few milliseconds long, too short for nvidia-smi's loop)."""
 
-    def __init__(self, gpu_id: str):
-        self.gpu_id = gpu_id
-        self.proc = None
-        self.path = os.path.join("/tmp", f"frt_clocks_{os.getpid()}.csv")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+             "sw_power_cap")
+
+    def __init__(self, gpu_uuid: str | None):
+        self.handle = None
+        self.samples: list[tuple[float, int]] = []
+        self.thread = None
+        self.stop_flag = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(gpu_uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(
+                self.handle, pynvml.NVML_CLOCK_SM))
+            self.bits = dict(zip(self.NAMES, (
+                pynvml.nvmlClocksEventReasonHwSlowdown,
+                pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                pynvml.nvmlClocksEventReasonSwPowerCap)))
+        except Exception as exc:  # noqa: BLE001
+            self.handle = None
+            self.why = f"no NVML: {exc}"[:80]
+
+    def _sample(self):
+        nv = self.nv
+        sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        self.samples.append((float(sm), int(rs)))
+
+    def _loop(self):
+        while not self.stop_flag:
+            try:
+                self._sample()
+            except Exception:  # noqa: BLE001
+                return
+            time.sleep(0.001)
 
     def start(self):
-        try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", self.gpu_id], stdout=self.fh,
-                stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+        if self.handle is None:
+            return
+        import threading
+        self.stop_flag = False
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.fh.close()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
-                 "sw_power_cap"]
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.why],
+                    "samples": 0}
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+        if not self.samples:   # the region ended before the first sample
+            self._sample()
+        reasons = sorted(n for n, b in self.bits.items()
+                         if any(r & b for _, r in self.samples))
+        return {"sm_mhz": statistics.median(sm for sm, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "source": "nvml, 1 ms"}
 
 
 # --------------------------------------------------------------- runners ----
@@ -799,7 +809,7 @@ def run_gpu(args):
     assert frt.frt_device_status(True) == frt.FRT_OK
 
     mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    gpu_id = str(local)
+    gpu_id = None
     try:
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:  # noqa: BLE001

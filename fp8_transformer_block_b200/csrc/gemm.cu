@@ -104,64 +104,75 @@ __device__ __forceinline__ void load32_bf16(const uint16_t* src, float (&f)[32])
 
 // One token row m, output columns n0 .. n0 + W - 1 (W = 8 or 16, n0 % W == 0,
 // inside one head): the same arithmetic as epi_rows_chunk at 16-byte
-// granularity.  The rope and bias pieces are loaded by the caller before the
-// accumulators arrive.
+// granularity, in two steps.  item_plan works out, ahead of the
+// accumulators, where each 8-column piece goes and loads the rope and bias
+// pieces it needs; item_apply then only scales, adds, rotates and stores
+// (a short dependency chain: the epilogue of a small tile runs one warp per
+// scheduler, so every dependent instruction after the data arrives counts).
 template <int W>
-__device__ __forceinline__ void epi_rows_w(const GemmParams& p, const float (&v)[W], int m, int n0,
-                                           float alpha, const uint4 (&bias8)[W / 8],
-                                           const uint4 (&rope8)[W / 8]) {
-  const int b = m / p.Mseq, s = m % p.Mseq;
-  const int h = n0 / p.hd, d00 = n0 % p.hd;
+struct ItemPlan {
+  uint16_t* dst[W / 8];  // nullptr: the item lies outside the output
+  uint4 bias8[W / 8], rope8[W / 8];
+  bool rot;
+};
+
+template <int W>
+__device__ __forceinline__ void item_plan(const GemmParams& p, int m, int n0, ItemPlan<W>& it) {
 #pragma unroll
   for (int g = 0; g < W / 8; ++g) {
+    it.dst[g] = nullptr;
+    it.bias8[g] = it.rope8[g] = make_uint4(0, 0, 0, 0);
+  }
+  it.rot = false;
+  if (n0 >= p.N || m >= p.M) return;
+  const int b = m / p.Mseq, s = m % p.Mseq;
+  const int h = n0 / p.hd, d00 = n0 % p.hd;
+  it.rot = p.epi == EPI_ROPE && h < p.hq + p.hkv;
+#pragma unroll
+  for (int g = 0; g < W / 8; ++g) {
+    if (p.bias) it.bias8[g] = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * g));
+    if (it.rot)
+      it.rope8[g] = __ldg(reinterpret_cast<const uint4*>(p.rope + long(s) * p.hd + d00 + 8 * g));
+    const int d0 = d00 + 8 * g;
+    if (p.epi == EPI_BF16)
+      it.dst[g] = static_cast<uint16_t*>(p.out) + long(m) * p.ldo + n0 + 8 * g;
+    else if (h < p.hq)
+      it.dst[g] = p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d0;
+    else if (h < p.hq + p.hkv)
+      it.dst[g] = p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d0;
+    else
+      it.dst[g] = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq - p.hkv)) * p.hd + d0;
+  }
+}
+
+template <int W>
+__device__ __forceinline__ void item_apply(const GemmParams& p, const float (&v)[W], float alpha,
+                                           const ItemPlan<W>& it) {
+#pragma unroll
+  for (int g = 0; g < W / 8; ++g) {
+    if (!it.dst[g]) continue;
     float y[8];
     if (p.bias) {
       float bb[8];
-      unpack8(bias8[g], bb);
+      unpack8(it.bias8[g], bb);
 #pragma unroll
       for (int j = 0; j < 8; ++j) y[j] = bf2f(f2bf(__fadd_rn(__fmul_rn(v[8 * g + j], alpha), bb[j])));
     } else {
 #pragma unroll
       for (int j = 0; j < 8; ++j) y[j] = bf2f(f2bf(__fmul_rn(v[8 * g + j], alpha)));
     }
-    uint16_t* dst;
-    if (p.epi == EPI_BF16) {
-      dst = static_cast<uint16_t*>(p.out) + long(m) * p.ldo + n0 + 8 * g;
-    } else {
-      const int d0 = d00 + 8 * g;
-      if (h < p.hq + p.hkv) {
-        float r[8];
-        unpack8(rope8[g], r);
+    if (it.rot) {
+      float r[8];
+      unpack8(it.rope8[g], r);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float c = r[2 * i], sn = r[2 * i + 1];
-          const float x0 = y[2 * i], x1 = y[2 * i + 1];
-          y[2 * i] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, sn));
-          y[2 * i + 1] = __fadd_rn(__fmul_rn(x0, sn), __fmul_rn(x1, c));
-        }
-        dst = h < p.hq ? p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d0
-                       : p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d0;
-      } else {
-        const int hv = h - p.hq - p.hkv;
-        dst = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + hv) * p.hd + d0;
+      for (int i = 0; i < 4; ++i) {
+        const float c = r[2 * i], sn = r[2 * i + 1];
+        const float x0 = y[2 * i], x1 = y[2 * i + 1];
+        y[2 * i] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, sn));
+        y[2 * i + 1] = __fadd_rn(__fmul_rn(x0, sn), __fmul_rn(x1, c));
       }
     }
-    *reinterpret_cast<uint4*>(dst) = pack8_bf16(y);
-  }
-}
-
-// The rope pairs and bias an item of W columns needs (zeros when unused).
-template <int W>
-__device__ __forceinline__ void epi_rows_w_operands(const GemmParams& p, int m, int n0,
-                                                    uint4 (&bias8)[W / 8], uint4 (&rope8)[W / 8]) {
-  const bool rot = p.epi == EPI_ROPE && n0 / p.hd < p.hq + p.hkv;
-#pragma unroll
-  for (int g = 0; g < W / 8; ++g) {
-    bias8[g] = p.bias ? __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * g))
-                      : make_uint4(0, 0, 0, 0);
-    rope8[g] = rot ? __ldg(reinterpret_cast<const uint4*>(p.rope + long(m % p.Mseq) * p.hd +
-                                                          n0 % p.hd + 8 * g))
-                   : make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(it.dst[g]) = pack8_bf16(y);
   }
 }
 
@@ -268,11 +279,11 @@ __device__ __forceinline__ void emit_swap_items(const GemmParams& p, int ta, int
     const int n0 = ta * BMT + W * cw;
     const int m = tb * BN + m_local;
     if (n0 >= p.N || m >= p.M) continue;
-    uint4 bias8[W / 8], rope8[W / 8];
-    epi_rows_w_operands<W>(p, m, n0, bias8, rope8);
+    ItemPlan<W> ip;
+    item_plan<W>(p, m, n0, ip);
     float v[W];
     fetch(m_local, cw, v);
-    epi_rows_w<W>(p, v, m, n0, alpha, bias8, rope8);
+    item_apply<W>(p, v, alpha, ip);
   }
 }
 
@@ -365,14 +376,19 @@ __host__ __device__ constexpr int t_tile_bytes() {
 
 template <bool SWAP, int BMT, int BN, int STAGES>
 __host__ __device__ constexpr int smem_total() {
-  return STAGES * (BMT * BK + BN * BK) + t_tile_bytes<SWAP, BMT, BN>() + 1024 + 256;
+  return STAGES * (BMT * BK + BN * BK) + t_tile_bytes<SWAP, BMT, BN>() + 1024 + 512;
 }
 
 // CLUSTER: the p.splits K-splits of a tile run as one thread-block cluster
 // (rank = split, one unit per CTA); each CTA stages its fp32 partial in its
-// shared memory and, after a cluster barrier, the ranks share the tile's
-// epilogue, each summing its items over all ranks' partials (distributed
-// shared memory, rank order) -- no global partials, no atomics.
+// shared memory.  Rank 0 (the leader) tells the others when its operand ring
+// is free (its last MMA is done); each other rank then bulk-copies its
+// staged partial into slot rank-1 of the leader's ring, counted as
+// transaction bytes on the leader's barrier red_full, and leaves once the
+// leader confirms receipt.  The leader sums the partials in rank order from
+// its own shared memory and runs the whole tile's epilogue, with the rope
+// and bias operands loaded while the main loop ran -- no global partials,
+// no atomics, no full-cluster barrier on the output path.
 template <bool SWAP, int BMT, int BN, int STAGES, bool CLUSTER>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -394,7 +410,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* red_full = drain + 1;  // CLUSTER leader: the other ranks' partials
+  uint64_t* go = drain + 2;        // CLUSTER other ranks: the leader's ring is free
+  uint64_t* done = drain + 3;      // CLUSTER other ranks: the leader has the partial
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* last_flag = abort_flag + 1;
   volatile int* epi_ok = abort_flag + 2;  // [4], one per epilogue warp
@@ -414,9 +433,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       mbar_init(&tempty[b], 4);
     }
     mbar_init(drain, 1);
+    if (CLUSTER) {
+      mbar_init(red_full, 1);
+      mbar_init(go, 1);
+      mbar_init(done, 1);
+    }
     *abort_flag = 0;
     *last_flag = 0;
     fence_barrier_init();
+    if (CLUSTER && cluster_ctarank() == 0 && p.splits > 1)
+      mbar_arrive_expect_tx(red_full, uint32_t(p.splits - 1) * t_tile_bytes<SWAP, BMT, BN>());
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
@@ -427,6 +453,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   __syncwarp();  // warp 0's lanes wait for lane 0's barrier set-up
   tc_fence_before();
   __syncthreads();
+  if (CLUSTER) cluster_arrive_relaxed();  // this CTA's barriers exist
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -495,6 +522,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     // barrier below converged (an aligned barrier must not be met by part of
     // a warp while the rest is still working)
     __syncwarp();
+    if (CLUSTER) cluster_wait();
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0) {
@@ -534,6 +562,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       }
     }
     __syncwarp();  // converge before the block barrier and the TMEM release
+    if (CLUSTER) cluster_wait();
   } else {
     // ----------------------------------------------------------- epilogue --
     // The rope table is bind-time data: pull this CTA's first-unit rows into
@@ -556,6 +585,23 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
     const int row = acc_row<BMT>(q, lane);
     const bool valid = acc_row_valid<BMT>(lane);
+    // CLUSTER leader: the rope and bias pieces of its items, loaded while
+    // the main loop runs (they are read-only here and written, if at all,
+    // by kernels that completed before the dependency wait above)
+    constexpr int LW = 16;                          // columns per leader item
+    constexpr int LNI = CLUSTER ? BN * (BMT / LW) / 128 : 1;  // items per thread
+    ItemPlan<LW> lplan[LNI];
+    const uint32_t crank = CLUSTER ? cluster_ctarank() : 0u;
+    if (CLUSTER && crank == 0 && blockIdx.x < unsigned(p.units)) {
+      const int tile = int(blockIdx.x) / p.splits;
+      const int ta = tile % p.a_tiles, tb = tile / p.a_tiles;
+#pragma unroll
+      for (int i = 0; i < LNI; ++i) {
+        const int it = int(threadIdx.x) - 64 + 128 * i;
+        item_plan<LW>(p, tb * BN + it / (BMT / LW), ta * BMT + LW * (it % (BMT / LW)), lplan[i]);
+      }
+    }
+    bool staged = false, cwaited = false;
     int local = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++local) {
       const int tile = u / p.splits, split = u % p.splits;
@@ -578,9 +624,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       tc_fence_after();
       const uint32_t tbase = tmem_base + uint32_t(ab * BN) + (uint32_t(32 * q) << 16);
       if (CLUSTER) {
-        // one unit per CTA: stage the partial; the cluster reduces it below
+        // one unit per CTA.  The leader's MMAs are done: its ring is free
+        // for the other ranks' partials.  Then stage this rank's partial.
+        cluster_wait();
+        cwaited = true;
+        if (crank == 0 && threadIdx.x == 64)
+          for (int j = 1; j < p.splits; ++j)
+            mbar_arrive_release_cluster(map_cluster(smem_u32(go), uint32_t(j)));
         stage_swap_tile<BMT, BN>(T, q, lane,
                                  [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); });
+        staged = true;
         break;
       }
       auto release_tmem = [&]() {
@@ -660,59 +713,70 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         named_bar_sync(1, 128);
       }
     }
+    if (CLUSTER) {
+      if (!cwaited) cluster_wait();
+      constexpr uint32_t TB = uint32_t(t_tile_bytes<SWAP, BMT, BN>());
+      const bool fits = uint32_t(p.splits - 1) * TB <= uint32_t(STAGES * (A_BYTES + B_BYTES));
+      if (staged && !fits) {
+        if (threadIdx.x == 64) record_timeout(p.status);  // the host never plans this
+      } else if (staged && crank != 0) {
+        // hand the staged partial to the leader, then wait for its receipt
+        // (this CTA's shared memory must outlive the copy)
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 64) {
+          if (mbar_wait_bounded_cluster(go, 0, kWaitNs)) {
+            bulk_copy_to_peer(map_cluster(smem_u32(smem) + (crank - 1u) * TB, 0), T, TB,
+                              map_cluster(smem_u32(red_full), 0));
+            if (!mbar_wait_bounded_cluster(done, 0, kWaitNs)) record_timeout(p.status);
+          } else {
+            record_timeout(p.status);
+          }
+        }
+        __syncwarp();
+      } else if (staged) {
+        // leader: own partial complete, then the others' in its ring
+        named_bar_sync(1, 128);
+        const bool got = mbar_wait_bounded_cluster(red_full, 0, kWaitNs);
+        if (threadIdx.x == 64) {
+          if (got) {
+            for (int j = 1; j < p.splits; ++j)
+              mbar_arrive_release_cluster(map_cluster(smem_u32(done), uint32_t(j)));
+          } else {
+            record_timeout(p.status);
+          }
+        }
+        if (got) {
+          constexpr int TS = BMT + 4, CW = BMT / LW;
+          const float* slots = reinterpret_cast<const float*>(smem);
+          const int nsl = p.splits - 1;
+#pragma unroll
+          for (int i = 0; i < LNI; ++i) {
+            const int it = int(threadIdx.x) - 64 + 128 * i;
+            const int off = (it / CW) * TS + LW * (it % CW);
+            float v[LW];
+#pragma unroll
+            for (int j = 0; j < LW; ++j) v[j] = 0.0f;
+            auto add = [&](const float* src) {
+              const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+              for (int k = 0; k < LW / 4; ++k) {
+                const float4 f = s4[k];
+                v[4 * k] = __fadd_rn(v[4 * k], f.x);
+                v[4 * k + 1] = __fadd_rn(v[4 * k + 1], f.y);
+                v[4 * k + 2] = __fadd_rn(v[4 * k + 2], f.z);
+                v[4 * k + 3] = __fadd_rn(v[4 * k + 3], f.w);
+              }
+            };
+            add(T + off);  // rank 0, then ranks 1 .. splits-1
+            for (int sl = 0; sl < nsl; ++sl) add(slots + sl * int(TB / 4) + off);
+            item_apply<LW>(p, v, alpha, lplan[i]);
+          }
+        }
+      }
+    }
   }
 
-  if (CLUSTER) {
-    cluster_sync_all();  // every rank's partial is staged and visible
-    if (warp >= 2 && blockIdx.x < unsigned(p.units)) {
-      const int tile = int(blockIdx.x) / p.splits;
-      const int ta = tile % p.a_tiles, tb = tile / p.a_tiles;
-      const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
-      const uint32_t t_addr = smem_u32(T);
-      constexpr int TS = BMT + 4;
-      // the ranks share the tile's items in contiguous ranges; items of 16
-      // columns when that leaves at most one item per thread
-      const int r = int(cluster_ctarank());
-      auto reduce_emit = [&](auto wtag) {
-        constexpr int W = decltype(wtag)::value;
-        constexpr int ITEMS = BN * (BMT / W);
-        const int lo = r * ITEMS / p.splits, hi = (r + 1) * ITEMS / p.splits;
-        emit_swap_items<BMT, BN, W>(
-            p, ta, tb, alpha, lo, hi, [&](int m_local, int cw, float (&v)[W]) {
-              const uint32_t off = t_addr + uint32_t((m_local * TS + W * cw) * 4);
-              constexpr int Q = W / 4;  // float4 per rank
-              constexpr int RMAX = W == 16 ? 4 : kMaxCluster;
-              float4 f[RMAX * Q];
-#pragma unroll
-              for (int q2 = 0; q2 < RMAX; ++q2) {
-                if (q2 < p.splits) {
-                  const uint32_t a = map_cluster(off, uint32_t(q2));
-#pragma unroll
-                  for (int k = 0; k < Q; ++k) f[q2 * Q + k] = ld_cluster_f4(a + 16u * k);
-                }
-              }
-#pragma unroll
-              for (int j = 0; j < W; ++j) v[j] = 0.0f;
-#pragma unroll
-              for (int q2 = 0; q2 < RMAX; ++q2) {
-                if (q2 < p.splits) {
-#pragma unroll
-                  for (int k = 0; k < Q; ++k) {
-                    const float4 a = f[q2 * Q + k];
-                    v[4 * k] = __fadd_rn(v[4 * k], a.x);
-                    v[4 * k + 1] = __fadd_rn(v[4 * k + 1], a.y);
-                    v[4 * k + 2] = __fadd_rn(v[4 * k + 2], a.z);
-                    v[4 * k + 3] = __fadd_rn(v[4 * k + 3], a.w);
-                  }
-                }
-              }
-            });
-      };
-      if (p.splits <= 4) reduce_emit(std::integral_constant<int, 16>{});
-      else reduce_emit(std::integral_constant<int, 8>{});
-    }
-    cluster_sync_all();  // no rank leaves while another still reads its tile
-  }
 
   tc_fence_before();
   __syncthreads();
@@ -1129,7 +1193,9 @@ int launch_swap(Plan pl, const CUtensorMap& ta, const CUtensorMap& tb, GemmParam
     int rc = prepare_kernel<true, BMT, BN, STAGES, true>();
     if (rc) return rc;
     const int tiles = pl.a_tiles * pl.b_tiles;
-    int size = pl.splits;
+    // the leader's operand ring receives the other ranks' staged partials
+    constexpr int kMaxRanks = 1 + STAGES * (BMT * BK + BN * BK) / t_tile_bytes<true, BMT, BN>();
+    int size = pl.splits < kMaxRanks ? pl.splits : kMaxRanks;
     while (size > 1 && max_active_clusters<BMT, BN, STAGES>(size, tiles * size) < tiles) --size;
     if (size > 1) {
       p.splits = size;

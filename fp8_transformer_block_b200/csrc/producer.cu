@@ -270,36 +270,41 @@ __global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
 
 // ------------------------------------------------ staged (bandwidth) form --
 //
-// Many rows: persistent CTAs of 256 threads walk rows r = blockIdx.x,
+// Many rows: persistent CTAs of T threads walk rows r = blockIdx.x,
 // + row_blocks, ...; thread 0 keeps the next kStages rows' streamed inputs
 // in flight as bulk copies into a shared-memory ring (one mbarrier per
-// stage), so HBM always has work queued while the CTA reduces and
-// quantizes the current row.  Same arithmetic as the register kernels.
-constexpr int kStagedThreads = 256;
+// stage).  Thread t owns the column chunks c = t + i*T (i < CPT, 8 columns
+// each): per row it moves its chunks from the ring into registers once, so
+// the stage is handed back to the copy engine right after the first row
+// reduction, and the per-column constants (table rows, norm weight) stay in
+// registers for the CTA's lifetime.  Two block barriers per row, one per
+// row statistic; the first also carries the consensus on a timed-out wait.
+// Same arithmetic, in the same order, as the register kernels.
 constexpr int kStages = 3;
+constexpr int kMaxCpt = 4;
 constexpr uint64_t kRowWaitNs = 2000000000ull;   // 2 s per wait
 constexpr uint64_t kRowDrainNs = 200000000ull;
 
-__device__ __forceinline__ float block_sum(float v, float* red) {
+// Sum over the block of one value per thread; `red` holds one slot per warp.
+__device__ __forceinline__ float block_sum_into(float v, float* red, bool& ok) {
   v = warp_sum(v);
-  __syncthreads();
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
+  ok = __syncthreads_and(ok) != 0;
   float s = 0.0f;
-#pragma unroll
-  for (int i = 0; i < kStagedThreads / 32; ++i) s = __fadd_rn(s, red[i]);
+  const int nw = int(blockDim.x >> 5);
+  for (int i = 0; i < nw; ++i) s = __fadd_rn(s, red[i]);
   return s;
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(kStagedThreads) producer_staged_kernel(ProducerArgs a) {
+template <int MODE, int CPT>
+__global__ void __launch_bounds__(256) producer_staged_kernel(ProducerArgs a) {
   extern __shared__ __align__(128) uint8_t ring[];
-  __shared__ float red[kStagedThreads / 32];
+  __shared__ float red1[8], red2[8];
   constexpr int NS = MODE == FRT_NORM_LAYERNORM_TABLE ? 3 : 2;  // streamed inputs per row
   pdl_trigger();
   pdl_wait();
   if (prefix_block(a)) return;
-  const int D = a.D, C = a.C, tid = threadIdx.x;
+  const int D = a.D, C = a.C, tid = threadIdx.x, T = blockDim.x;
   const uint32_t row_bytes = 2u * uint32_t(D);
   uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * NS * row_bytes);
   const long stride = a.row_blocks;
@@ -327,123 +332,157 @@ __global__ void __launch_bounds__(kStagedThreads) producer_staged_kernel(Produce
   }
   __syncthreads();
 
+  // per-column constants of this thread's chunks
+  bool has[CPT];
+  float k0[CPT][8], k1[CPT][8];  // table: shift / scale rows; AdaRMS: weight
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = tid + i * T;
+    has[i] = c < C;
+    if (MODE == FRT_NORM_LAYERNORM_TABLE) {
+      if (has[i]) {
+        const float* bsh = a.table + long(a.shift_idx) * D + 8 * c;
+        const float* bsc = a.table + long(a.scale_idx) * D + 8 * c;
+        const float4 h0 = __ldg(reinterpret_cast<const float4*>(bsh));
+        const float4 h1 = __ldg(reinterpret_cast<const float4*>(bsh + 4));
+        const float4 c0 = __ldg(reinterpret_cast<const float4*>(bsc));
+        const float4 c1 = __ldg(reinterpret_cast<const float4*>(bsc + 4));
+        k0[i][0] = h0.x; k0[i][1] = h0.y; k0[i][2] = h0.z; k0[i][3] = h0.w;
+        k0[i][4] = h1.x; k0[i][5] = h1.y; k0[i][6] = h1.z; k0[i][7] = h1.w;
+        k1[i][0] = c0.x; k1[i][1] = c0.y; k1[i][2] = c0.z; k1[i][3] = c0.w;
+        k1[i][4] = c1.x; k1[i][5] = c1.y; k1[i][6] = c1.z; k1[i][7] = c1.w;
+      }
+    } else {
+      if (has[i] && a.weight) {
+        unpack8(__ldg(reinterpret_cast<const uint4*>(a.weight + 8 * c)), k0[i]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) k0[i][j] = 1.0f;
+      }
+    }
+  }
+
   const float inv_as = __frcp_rn(__ldg(a.act_scale));  // quantize: y * (1 / scale)
   float mx = 0.0f;
   int k = 0;
   bool aborted = false;
   for (long r = blockIdx.x; r < a.rows; r += stride, ++k) {
     const int st = k % kStages;
-    const bool got = mbar_wait_bounded(&full[st], uint32_t((k / kStages) & 1), kRowWaitNs,
-                                       nullptr);
-    if (!__syncthreads_and(got)) {
-      aborted = true;
-      break;
-    }
-    uint16_t* s0 = reinterpret_cast<uint16_t*>(ring + st * NS * row_bytes);
-    uint16_t* s1 = s0 + D;
+    bool ok = mbar_wait_bounded(&full[st], uint32_t((k / kStages) & 1), kRowWaitNs, nullptr);
+    const uint16_t* s0 = reinterpret_cast<const uint16_t*>(ring + st * NS * row_bytes);
+    const uint16_t* s1 = s0 + D;
+    float xv[CPT][8];
     if (MODE == FRT_NORM_ADARMS) {
-      // s0: residual row, s1: delta row
+      // s0: residual row, s1: delta row; h = res + gate * delta, written back
       const uint16_t* gg = a.gate + r * a.gate_stride;
       uint16_t* rr = a.res + r * D;
       float ss = 0.0f;
-      for (int c = tid; c < C; c += kStagedThreads) {
-        float rv[8], dv[8], gv[8], h[8];
-        unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), rv);
-        unpack8(*reinterpret_cast<const uint4*>(s1 + 8 * c), dv);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(gg + 8 * c)), gv);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) h[j] = __fadd_rn(rv[j], __fmul_rn(gv[j], dv[j]));
-        const uint4 hb = pack8_bf16(h);
-        *reinterpret_cast<uint4*>(rr + 8 * c) = hb;
-        *reinterpret_cast<uint4*>(s0 + 8 * c) = hb;
-        float hf[8];
-        unpack8(hb, hf);
+      for (int i = 0; i < CPT; ++i) {
+        const int c = tid + i * T;
+        if (has[i]) {
+          float rv[8], dv[8], gv[8], h[8];
+          unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), rv);
+          unpack8(*reinterpret_cast<const uint4*>(s1 + 8 * c), dv);
+          unpack8(__ldg(reinterpret_cast<const uint4*>(gg + 8 * c)), gv);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) ss = __fadd_rn(ss, __fmul_rn(hf[j], hf[j]));
+          for (int j = 0; j < 8; ++j) h[j] = __fadd_rn(rv[j], __fmul_rn(gv[j], dv[j]));
+          const uint4 hb = pack8_bf16(h);
+          if (ok) *reinterpret_cast<uint4*>(rr + 8 * c) = hb;
+          unpack8(hb, xv[i]);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss = __fadd_rn(ss, __fmul_rn(xv[i][j], xv[i][j]));
+        }
       }
-      ss = block_sum(ss, red);
+      ss = block_sum_into(ss, red1, ok);   // every thread is done with the stage
+      if (!ok) { aborted = true; break; }
+      if (tid == 0) {
+        const long rn = r + kStages * stride;
+        if (rn < a.rows) issue(rn, st);
+      }
       const float ms = __fdiv_rn(ss, float(D));
       const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
       const uint16_t* sty = a.style + r * a.style_stride;
-      for (int c = tid; c < C; c += kStagedThreads) {
-        float hf[8], wv[8], sc[8], sh[8], q[8];
-        unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), hf);
-        if (a.weight) unpack8(__ldg(reinterpret_cast<const uint4*>(a.weight + 8 * c)), wv);
-        else {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) wv[j] = 1.0f;
-        }
-        unpack8(__ldg(reinterpret_cast<const uint4*>(sty + 8 * c)), sc);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(sty + D + 8 * c)), sh);
+      for (int i = 0; i < CPT; ++i) {
+        const int c = tid + i * T;
+        if (has[i]) {
+          float sc[8], sh[8], q[8];
+          unpack8(__ldg(reinterpret_cast<const uint4*>(sty + 8 * c)), sc);
+          unpack8(__ldg(reinterpret_cast<const uint4*>(sty + D + 8 * c)), sh);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float v = __fmul_rn(hf[j], inv);
-          v = __fmul_rn(v, wv[j]);
-          v = __fmul_rn(v, __fadd_rn(1.0f, sc[j]));
-          const float y = __fadd_rn(v, sh[j]);
-          mx = fmaxf(mx, fabsf(y));
-          q[j] = __fmul_rn(y, inv_as);
+          for (int j = 0; j < 8; ++j) {
+            float v = __fmul_rn(xv[i][j], inv);
+            v = __fmul_rn(v, k0[i][j]);
+            v = __fmul_rn(v, __fadd_rn(1.0f, sc[j]));
+            const float y = __fadd_rn(v, sh[j]);
+            mx = fmaxf(mx, fabsf(y));
+            q[j] = __fmul_rn(y, inv_as);
+          }
+          *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
+          if (a.gate_out)
+            *reinterpret_cast<uint4*>(a.gate_out + r * D + 8 * c) =
+                __ldg(reinterpret_cast<const uint4*>(sty + 2 * D + 8 * c));
         }
-        *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
-        if (a.gate_out)
-          *reinterpret_cast<uint4*>(a.gate_out + r * D + 8 * c) =
-              __ldg(reinterpret_cast<const uint4*>(sty + 2 * D + 8 * c));
       }
     } else {
       // s0: x row, s1: shift chunk of temb, s2: scale chunk of temb
       const uint16_t* s2 = s1 + D;
+      uint4 esh4[CPT], esc4[CPT];
       float sum = 0.0f;
-      for (int c = tid; c < C; c += kStagedThreads) {
-        float xv[8];
-        unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), xv);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) sum = __fadd_rn(sum, xv[j]);
+      for (int i = 0; i < CPT; ++i) {
+        const int c = tid + i * T;
+        if (has[i]) {
+          unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), xv[i]);
+          esh4[i] = *reinterpret_cast<const uint4*>(s1 + 8 * c);
+          esc4[i] = *reinterpret_cast<const uint4*>(s2 + 8 * c);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sum = __fadd_rn(sum, xv[i][j]);
+        }
       }
-      sum = block_sum(sum, red);
+      sum = block_sum_into(sum, red1, ok);  // every thread is done with the stage
+      if (!ok) { aborted = true; break; }
+      if (tid == 0) {
+        const long rn = r + kStages * stride;
+        if (rn < a.rows) issue(rn, st);
+      }
       const float mu = __fdiv_rn(sum, float(D));
       float sq = 0.0f;
-      for (int c = tid; c < C; c += kStagedThreads) {
-        float xv[8];
-        unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), xv);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float d = __fsub_rn(xv[j], mu);
-          sq = __fadd_rn(sq, __fmul_rn(d, d));
+      for (int i = 0; i < CPT; ++i) {
+        if (has[i]) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float d = __fsub_rn(xv[i][j], mu);
+            sq = __fadd_rn(sq, __fmul_rn(d, d));
+          }
         }
       }
-      sq = block_sum(sq, red);
+      bool ok2 = true;
+      sq = block_sum_into(sq, red2, ok2);
       const float var = __fdiv_rn(sq, float(D));
       const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
-      const float* bsh = a.table + long(a.shift_idx) * D;
-      const float* bsc = a.table + long(a.scale_idx) * D;
-      for (int c = tid; c < C; c += kStagedThreads) {
-        float xv[8], esh[8], esc[8], q[8];
-        unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), xv);
-        unpack8(*reinterpret_cast<const uint4*>(s1 + 8 * c), esh);
-        unpack8(*reinterpret_cast<const uint4*>(s2 + 8 * c), esc);
-        const float4 h0 = __ldg(reinterpret_cast<const float4*>(bsh + 8 * c));
-        const float4 h1 = __ldg(reinterpret_cast<const float4*>(bsh + 8 * c + 4));
-        const float4 c0 = __ldg(reinterpret_cast<const float4*>(bsc + 8 * c));
-        const float4 c1 = __ldg(reinterpret_cast<const float4*>(bsc + 8 * c + 4));
-        const float tsh8[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-        const float tsc8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float shift = __fadd_rn(tsh8[j], esh[j]);
-          const float scale = __fadd_rn(tsc8[j], esc[j]);
-          float v = __fmul_rn(__fsub_rn(xv[j], mu), inv);
-          v = __fmul_rn(v, __fadd_rn(1.0f, scale));
-          const float y = __fadd_rn(v, shift);
-          mx = fmaxf(mx, fabsf(y));
-          q[j] = __fmul_rn(y, inv_as);
+      for (int i = 0; i < CPT; ++i) {
+        const int c = tid + i * T;
+        if (has[i]) {
+          float esh[8], esc[8], q[8];
+          unpack8(esh4[i], esh);
+          unpack8(esc4[i], esc);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float shift = __fadd_rn(k0[i][j], esh[j]);
+            const float scale = __fadd_rn(k1[i][j], esc[j]);
+            float v = __fmul_rn(__fsub_rn(xv[i][j], mu), inv);
+            v = __fmul_rn(v, __fadd_rn(1.0f, scale));
+            const float y = __fadd_rn(v, shift);
+            mx = fmaxf(mx, fabsf(y));
+            q[j] = __fmul_rn(y, inv_as);
+          }
+          *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
         }
-        *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
       }
-    }
-    __syncthreads();  // every thread is done with this stage
-    if (tid == 0) {
-      const long rn = r + kStages * stride;
-      if (rn < a.rows) issue(rn, st);
     }
   }
   if (aborted && tid == 0) {
@@ -461,7 +500,6 @@ __global__ void __launch_bounds__(kStagedThreads) producer_staged_kernel(Produce
     if ((threadIdx.x & 31) == 0) atomic_max_nonneg(a.amax, mx);
   }
 }
-
 }  // namespace
 
 int producer_call(int mode, int rows, int D, float eps, uint16_t* res, const uint16_t* delta,
@@ -516,24 +554,33 @@ int producer_call(int mode, int rows, int D, float eps, uint16_t* res, const uin
   a.status = device_status_ptr();
   const int sms = num_sms();
   const int ns = mode == FRT_NORM_LAYERNORM_TABLE ? 3 : 2;
-  const size_t staged_smem = size_t(3) * ns * 2 * D + 64;
-  if (rows > 2 * sms && staged_smem <= 72 * 1024) {
-    // bandwidth regime: persistent CTAs with a bulk-copy row ring
-    auto kern = mode == FRT_NORM_ADARMS ? producer_staged_kernel<FRT_NORM_ADARMS>
-                                        : producer_staged_kernel<FRT_NORM_LAYERNORM_TABLE>;
+  const size_t staged_smem = size_t(kStages) * ns * 2 * D + 64;
+  const int cpt = (a.C + 255) / 256;
+  if (rows > 2 * sms && staged_smem <= 72 * 1024 && cpt <= kMaxCpt) {
+    // bandwidth regime: persistent CTAs with a bulk-copy row ring; each
+    // thread owns cpt chunks of 8 columns
+    using Kern = void (*)(ProducerArgs);
+    static const Kern kerns[2][kMaxCpt] = {
+        {producer_staged_kernel<FRT_NORM_ADARMS, 1>, producer_staged_kernel<FRT_NORM_ADARMS, 2>,
+         producer_staged_kernel<FRT_NORM_ADARMS, 3>, producer_staged_kernel<FRT_NORM_ADARMS, 4>},
+        {producer_staged_kernel<FRT_NORM_LAYERNORM_TABLE, 1>,
+         producer_staged_kernel<FRT_NORM_LAYERNORM_TABLE, 2>,
+         producer_staged_kernel<FRT_NORM_LAYERNORM_TABLE, 3>,
+         producer_staged_kernel<FRT_NORM_LAYERNORM_TABLE, 4>}};
+    const Kern kern = kerns[mode == FRT_NORM_ADARMS ? 0 : 1][cpt - 1];
+    const int block = ((a.C + cpt - 1) / cpt + 31) / 32 * 32;
     if (first_use(reinterpret_cast<const void*>(kern)) &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              72 * 1024 + 64) != cudaSuccess)
       return fail(FRT_ECUDA, "cudaFuncSetAttribute(producer smem)");
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kStagedThreads,
-                                                      staged_smem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, staged_smem) !=
+            cudaSuccess ||
         per_sm < 1) {
       cudaGetLastError();
       per_sm = 1;
     }
     a.row_blocks = rows < sms * per_sm ? rows : sms * per_sm;
-    const int block = kStagedThreads;
     int pre_blocks = 0;
     if (pre_units > 0) {
       const long need = (pre_units + block - 1) / block;
