@@ -97,6 +97,62 @@ __device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
       __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
+// ---- paired fp32 arithmetic (sm_100 f32x2 instructions) --------------------
+// A uint64_t holds two fp32 lanes (lo, hi).  add2 / sub2 / mul2 round each
+// lane to nearest even exactly like the scalar __fadd_rn / __fsub_rn /
+// __fmul_rn, so swapping a scalar pair for one paired instruction leaves
+// every result bit unchanged while halving the instructions issued.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(uint32_t(v)); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(uint32_t(v >> 32)); }
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// Two bf16 in one 32-bit word (lo in the low half) -> an fp32 pair.
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+  return (uint64_t(w & 0xFFFF0000u) << 32) | uint64_t(w << 16);
+}
+// 8 bf16 in a uint4 -> 4 fp32 pairs.
+__device__ __forceinline__ void unpack8_f2(const uint4& v, uint64_t (&f)[4]) {
+  f[0] = bf16x2_to_f2(v.x);
+  f[1] = bf16x2_to_f2(v.y);
+  f[2] = bf16x2_to_f2(v.z);
+  f[3] = bf16x2_to_f2(v.w);
+}
+// 4 fp32 pairs -> 8 bf16 (round to nearest even) in a uint4.
+__device__ __forceinline__ uint4 pack8_bf16_f2(const uint64_t (&f)[4]) {
+  return make_uint4(pack_bf16x2(f2_lo(f[0]), f2_hi(f[0])), pack_bf16x2(f2_lo(f[1]), f2_hi(f[1])),
+                    pack_bf16x2(f2_lo(f[2]), f2_hi(f[2])), pack_bf16x2(f2_lo(f[3]), f2_hi(f[3])));
+}
+// 4 fp32 pairs -> 8 e4m3fn codes in a uint2.
+__device__ __forceinline__ uint2 pack8_e4m3_f2(const uint64_t (&q)[4]) {
+  const uint32_t lo = pack_e4m3x2(f2_lo(q[0]), f2_hi(q[0])) |
+                      (uint32_t(pack_e4m3x2(f2_lo(q[1]), f2_hi(q[1]))) << 16);
+  const uint32_t hi = pack_e4m3x2(f2_lo(q[2]), f2_hi(q[2])) |
+                      (uint32_t(pack_e4m3x2(f2_lo(q[3]), f2_hi(q[3]))) << 16);
+  return make_uint2(lo, hi);
+}
+// max(m, |lo|, |hi|)
+__device__ __forceinline__ float absmax2(float m, uint64_t v) {
+  return fmaxf(fmaxf(m, fabsf(f2_lo(v))), fabsf(f2_hi(v)));
+}
+
 // 8 bf16 packed in a uint4 -> 8 floats.
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};

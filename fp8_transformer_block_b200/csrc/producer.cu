@@ -279,8 +279,18 @@ __global__ void __launch_bounds__(512) ln_table_kernel(ProducerArgs a) {
 // reduction, and the per-column constants (table rows, norm weight) stay in
 // registers for the CTA's lifetime.  Two block barriers per row, one per
 // row statistic; the first also carries the consensus on a timed-out wait.
-// Same arithmetic, in the same order, as the register kernels.
-constexpr int kStages = 3;
+// Same operations as the register kernels, issued two lanes at a time
+// (f32x2: identical rounding per lane, half the instructions); the row sums
+// keep two running partials per thread, a different summation order that
+// moves the statistics by a few ulps at most.
+#ifndef FRT_PRODUCER_STAGES
+#define FRT_PRODUCER_STAGES 3
+#endif
+#ifndef FRT_PRODUCER_MAX_THREADS
+#define FRT_PRODUCER_MAX_THREADS 128
+#endif
+constexpr int kStages = FRT_PRODUCER_STAGES;        // rows in flight per CTA
+constexpr int kMaxThreads = FRT_PRODUCER_MAX_THREADS;  // threads per row (CTA)
 constexpr int kMaxCpt = 4;
 constexpr uint64_t kRowWaitNs = 2000000000ull;   // 2 s per wait
 constexpr uint64_t kRowDrainNs = 200000000ull;
@@ -297,7 +307,8 @@ __device__ __forceinline__ float block_sum_into(float v, float* red, bool& ok) {
 }
 
 template <int MODE, int CPT>
-__global__ void __launch_bounds__(256) producer_staged_kernel(ProducerArgs a) {
+__global__ void __launch_bounds__(256)
+producer_staged_kernel(ProducerArgs a) {
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ float red1[8], red2[8];
   constexpr int NS = MODE == FRT_NORM_LAYERNORM_TABLE ? 3 : 2;  // streamed inputs per row
@@ -332,9 +343,10 @@ __global__ void __launch_bounds__(256) producer_staged_kernel(ProducerArgs a) {
   }
   __syncthreads();
 
-  // per-column constants of this thread's chunks
+  // per-column constants of this thread's chunks, as fp32 pairs
   bool has[CPT];
-  float k0[CPT][8], k1[CPT][8];  // table: shift / scale rows; AdaRMS: weight
+  uint64_t k0[CPT][4], k1[CPT][4];  // table: shift / scale rows; AdaRMS: weight
+  const uint64_t one2 = f2_pack(1.0f, 1.0f);
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {
     const int c = tid + i * T;
@@ -343,26 +355,29 @@ __global__ void __launch_bounds__(256) producer_staged_kernel(ProducerArgs a) {
       if (has[i]) {
         const float* bsh = a.table + long(a.shift_idx) * D + 8 * c;
         const float* bsc = a.table + long(a.scale_idx) * D + 8 * c;
-        const float4 h0 = __ldg(reinterpret_cast<const float4*>(bsh));
-        const float4 h1 = __ldg(reinterpret_cast<const float4*>(bsh + 4));
-        const float4 c0 = __ldg(reinterpret_cast<const float4*>(bsc));
-        const float4 c1 = __ldg(reinterpret_cast<const float4*>(bsc + 4));
-        k0[i][0] = h0.x; k0[i][1] = h0.y; k0[i][2] = h0.z; k0[i][3] = h0.w;
-        k0[i][4] = h1.x; k0[i][5] = h1.y; k0[i][6] = h1.z; k0[i][7] = h1.w;
-        k1[i][0] = c0.x; k1[i][1] = c0.y; k1[i][2] = c0.z; k1[i][3] = c0.w;
-        k1[i][4] = c1.x; k1[i][5] = c1.y; k1[i][6] = c1.z; k1[i][7] = c1.w;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float4 t0 = __ldg(reinterpret_cast<const float4*>(bsh + 4 * h));
+          const float4 t1 = __ldg(reinterpret_cast<const float4*>(bsc + 4 * h));
+          k0[i][2 * h] = f2_pack(t0.x, t0.y);
+          k0[i][2 * h + 1] = f2_pack(t0.z, t0.w);
+          k1[i][2 * h] = f2_pack(t1.x, t1.y);
+          k1[i][2 * h + 1] = f2_pack(t1.z, t1.w);
+        }
       }
     } else {
       if (has[i] && a.weight) {
-        unpack8(__ldg(reinterpret_cast<const uint4*>(a.weight + 8 * c)), k0[i]);
+        unpack8_f2(__ldg(reinterpret_cast<const uint4*>(a.weight + 8 * c)), k0[i]);
       } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) k0[i][j] = 1.0f;
+        for (int j = 0; j < 4; ++j) k0[i][j] = one2;
       }
     }
   }
 
   const float inv_as = __frcp_rn(__ldg(a.act_scale));  // quantize: y * (1 / scale)
+  const uint64_t inv_as2 = f2_pack(inv_as, inv_as);
+  const uint64_t zero2 = f2_pack(0.0f, 0.0f);
   float mx = 0.0f;
   int k = 0;
   bool aborted = false;
@@ -371,29 +386,30 @@ __global__ void __launch_bounds__(256) producer_staged_kernel(ProducerArgs a) {
     bool ok = mbar_wait_bounded(&full[st], uint32_t((k / kStages) & 1), kRowWaitNs, nullptr);
     const uint16_t* s0 = reinterpret_cast<const uint16_t*>(ring + st * NS * row_bytes);
     const uint16_t* s1 = s0 + D;
-    float xv[CPT][8];
+    uint64_t xv[CPT][4];
     if (MODE == FRT_NORM_ADARMS) {
       // s0: residual row, s1: delta row; h = res + gate * delta, written back
       const uint16_t* gg = a.gate + r * a.gate_stride;
       uint16_t* rr = a.res + r * D;
-      float ss = 0.0f;
+      uint64_t ss2 = zero2;
 #pragma unroll
       for (int i = 0; i < CPT; ++i) {
         const int c = tid + i * T;
         if (has[i]) {
-          float rv[8], dv[8], gv[8], h[8];
-          unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), rv);
-          unpack8(*reinterpret_cast<const uint4*>(s1 + 8 * c), dv);
-          unpack8(__ldg(reinterpret_cast<const uint4*>(gg + 8 * c)), gv);
+          uint64_t rv[4], dv[4], gv[4], h[4];
+          unpack8_f2(*reinterpret_cast<const uint4*>(s0 + 8 * c), rv);
+          unpack8_f2(*reinterpret_cast<const uint4*>(s1 + 8 * c), dv);
+          unpack8_f2(__ldg(reinterpret_cast<const uint4*>(gg + 8 * c)), gv);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) h[j] = __fadd_rn(rv[j], __fmul_rn(gv[j], dv[j]));
-          const uint4 hb = pack8_bf16(h);
+          for (int j = 0; j < 4; ++j) h[j] = add2(rv[j], mul2(gv[j], dv[j]));
+          const uint4 hb = pack8_bf16_f2(h);
           if (ok) *reinterpret_cast<uint4*>(rr + 8 * c) = hb;
-          unpack8(hb, xv[i]);
+          unpack8_f2(hb, xv[i]);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) ss = __fadd_rn(ss, __fmul_rn(xv[i][j], xv[i][j]));
+          for (int j = 0; j < 4; ++j) ss2 = add2(ss2, mul2(xv[i][j], xv[i][j]));
         }
       }
+      float ss = __fadd_rn(f2_lo(ss2), f2_hi(ss2));
       ss = block_sum_into(ss, red1, ok);   // every thread is done with the stage
       if (!ok) { aborted = true; break; }
       if (tid == 0) {
@@ -402,24 +418,25 @@ __global__ void __launch_bounds__(256) producer_staged_kernel(ProducerArgs a) {
       }
       const float ms = __fdiv_rn(ss, float(D));
       const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
+      const uint64_t inv2 = f2_pack(inv, inv);
       const uint16_t* sty = a.style + r * a.style_stride;
 #pragma unroll
       for (int i = 0; i < CPT; ++i) {
         const int c = tid + i * T;
         if (has[i]) {
-          float sc[8], sh[8], q[8];
-          unpack8(__ldg(reinterpret_cast<const uint4*>(sty + 8 * c)), sc);
-          unpack8(__ldg(reinterpret_cast<const uint4*>(sty + D + 8 * c)), sh);
+          uint64_t sc[4], sh[4], q[4];
+          unpack8_f2(__ldg(reinterpret_cast<const uint4*>(sty + 8 * c)), sc);
+          unpack8_f2(__ldg(reinterpret_cast<const uint4*>(sty + D + 8 * c)), sh);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float v = __fmul_rn(xv[i][j], inv);
-            v = __fmul_rn(v, k0[i][j]);
-            v = __fmul_rn(v, __fadd_rn(1.0f, sc[j]));
-            const float y = __fadd_rn(v, sh[j]);
-            mx = fmaxf(mx, fabsf(y));
-            q[j] = __fmul_rn(y, inv_as);
+          for (int j = 0; j < 4; ++j) {
+            uint64_t v = mul2(xv[i][j], inv2);
+            v = mul2(v, k0[i][j]);
+            v = mul2(v, add2(one2, sc[j]));
+            const uint64_t y = add2(v, sh[j]);
+            mx = absmax2(mx, y);
+            q[j] = mul2(y, inv_as2);
           }
-          *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
+          *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3_f2(q);
           if (a.gate_out)
             *reinterpret_cast<uint4*>(a.gate_out + r * D + 8 * c) =
                 __ldg(reinterpret_cast<const uint4*>(sty + 2 * D + 8 * c));
@@ -429,18 +446,19 @@ __global__ void __launch_bounds__(256) producer_staged_kernel(ProducerArgs a) {
       // s0: x row, s1: shift chunk of temb, s2: scale chunk of temb
       const uint16_t* s2 = s1 + D;
       uint4 esh4[CPT], esc4[CPT];
-      float sum = 0.0f;
+      uint64_t sum2 = zero2;
 #pragma unroll
       for (int i = 0; i < CPT; ++i) {
         const int c = tid + i * T;
         if (has[i]) {
-          unpack8(*reinterpret_cast<const uint4*>(s0 + 8 * c), xv[i]);
+          unpack8_f2(*reinterpret_cast<const uint4*>(s0 + 8 * c), xv[i]);
           esh4[i] = *reinterpret_cast<const uint4*>(s1 + 8 * c);
           esc4[i] = *reinterpret_cast<const uint4*>(s2 + 8 * c);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) sum = __fadd_rn(sum, xv[i][j]);
+          for (int j = 0; j < 4; ++j) sum2 = add2(sum2, xv[i][j]);
         }
       }
+      float sum = __fadd_rn(f2_lo(sum2), f2_hi(sum2));
       sum = block_sum_into(sum, red1, ok);  // every thread is done with the stage
       if (!ok) { aborted = true; break; }
       if (tid == 0) {
@@ -448,39 +466,42 @@ __global__ void __launch_bounds__(256) producer_staged_kernel(ProducerArgs a) {
         if (rn < a.rows) issue(rn, st);
       }
       const float mu = __fdiv_rn(sum, float(D));
-      float sq = 0.0f;
+      const uint64_t mu2 = f2_pack(mu, mu);
+      uint64_t sq2 = zero2;
 #pragma unroll
       for (int i = 0; i < CPT; ++i) {
         if (has[i]) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float d = __fsub_rn(xv[i][j], mu);
-            sq = __fadd_rn(sq, __fmul_rn(d, d));
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t d = sub2(xv[i][j], mu2);
+            sq2 = add2(sq2, mul2(d, d));
           }
         }
       }
+      float sq = __fadd_rn(f2_lo(sq2), f2_hi(sq2));
       bool ok2 = true;
       sq = block_sum_into(sq, red2, ok2);
       const float var = __fdiv_rn(sq, float(D));
       const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
+      const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
       for (int i = 0; i < CPT; ++i) {
         const int c = tid + i * T;
         if (has[i]) {
-          float esh[8], esc[8], q[8];
-          unpack8(esh4[i], esh);
-          unpack8(esc4[i], esc);
+          uint64_t esh[4], esc[4], q[4];
+          unpack8_f2(esh4[i], esh);
+          unpack8_f2(esc4[i], esc);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float shift = __fadd_rn(k0[i][j], esh[j]);
-            const float scale = __fadd_rn(k1[i][j], esc[j]);
-            float v = __fmul_rn(__fsub_rn(xv[i][j], mu), inv);
-            v = __fmul_rn(v, __fadd_rn(1.0f, scale));
-            const float y = __fadd_rn(v, shift);
-            mx = fmaxf(mx, fabsf(y));
-            q[j] = __fmul_rn(y, inv_as);
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t shift = add2(k0[i][j], esh[j]);
+            const uint64_t scale = add2(k1[i][j], esc[j]);
+            uint64_t v = mul2(sub2(xv[i][j], mu2), inv2);
+            v = mul2(v, add2(one2, scale));
+            const uint64_t y = add2(v, shift);
+            mx = absmax2(mx, y);
+            q[j] = mul2(y, inv_as2);
           }
-          *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
+          *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3_f2(q);
         }
       }
     }
@@ -555,8 +576,9 @@ int producer_call(int mode, int rows, int D, float eps, uint16_t* res, const uin
   const int sms = num_sms();
   const int ns = mode == FRT_NORM_LAYERNORM_TABLE ? 3 : 2;
   const size_t staged_smem = size_t(kStages) * ns * 2 * D + 64;
-  const int cpt = (a.C + 255) / 256;
-  if (rows > 2 * sms && staged_smem <= 72 * 1024 && cpt <= kMaxCpt) {
+  const int cpt = (a.C + kMaxThreads - 1) / kMaxThreads;
+  constexpr size_t kStagedSmemMax = size_t(kStages) * 24 * 1024 + 64;
+  if (rows > 2 * sms && staged_smem <= kStagedSmemMax && cpt <= kMaxCpt) {
     // bandwidth regime: persistent CTAs with a bulk-copy row ring; each
     // thread owns cpt chunks of 8 columns
     using Kern = void (*)(ProducerArgs);
@@ -571,7 +593,7 @@ int producer_call(int mode, int rows, int D, float eps, uint16_t* res, const uin
     const int block = ((a.C + cpt - 1) / cpt + 31) / 32 * 32;
     if (first_use(reinterpret_cast<const void*>(kern)) &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             72 * 1024 + 64) != cudaSuccess)
+                             int(kStagedSmemMax)) != cudaSuccess)
       return fail(FRT_ECUDA, "cudaFuncSetAttribute(producer smem)");
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, staged_smem) !=
