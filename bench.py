@@ -47,16 +47,27 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP8_PER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
-# DRAM bytes per launch of the dominant kernel from the committed ncu capture
-# (profiles/), keyed by workload; valid only while the kernel's source hash
-# matches the one the counters were taken on.
-NCU_TRAFFIC = {}
+# DRAM bytes (read + write) per launch of the dominant kernel from the ncu
+# captures summarised under profiles/, keyed by (workload, kernel); a value
+# counts only while the hash of the kernel's sources matches the one the
+# counters were taken on (else the line reports traffic null).
+KERNEL_SOURCES = {
+    "gemm": ("gemm.cu", "frt_sm100.cuh"),
+    "producer": ("producer.cu", "frt_common.cuh", "frt_sm100.cuh", "frt_prefix.cuh"),
+    "prefix_copy": ("rope.cu", "frt_prefix.cuh"),
+}
+NCU_TRAFFIC = {
+    ("vla_action_expert", "gemm_rope_kv"): (5_426_176, "892268e76741ebb5"),
+    ("video_dit", "gemm_rope_kv"): (154_795_264, "892268e76741ebb5"),
+    ("gateup_mlp", "gemm_gateup_geglu"): (73_113_856, "892268e76741ebb5"),
+}
 
 
-def _src_hash():
+def _src_hash(kernel_name):
+    kind = ("gemm" if kernel_name.startswith("gemm") else
+            "producer" if kernel_name == "producer" else "prefix_copy")
     h = hashlib.sha256()
-    for f in ("gemm.cu", "producer.cu", "rope.cu", "frt_sm100.cuh",
-              "frt_common.cuh"):
+    for f in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, "fp8_transformer_block_b200", "csrc", f),
                   "rb") as fh:
             h.update(fh.read())
@@ -912,7 +923,7 @@ def run_gpu(args):
         peak = hbm
         unit = "GB/s"
     tr = NCU_TRAFFIC.get((args.config, kd.name))
-    traffic = tr[0] if tr and tr[1] == _src_hash() else None
+    traffic = tr[0] if tr and tr[1] == _src_hash(kd.name) else None
     kern_list = []
     for ms, k in zip(kern_ms, kinds):
         e = {"kernel": k.name, "us": round(ms * 1e3, 3),

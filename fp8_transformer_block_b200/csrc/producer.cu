@@ -97,6 +97,9 @@ __global__ void __launch_bounds__(512) adarms_kernel(ProducerArgs a) {
 
   float hr[VPT][8];
   float ss = 0.0f;
+  // every input of the row is requested up front (one memory round trip)
+  uint4 sc4[VPT], sh4[VPT], w4[VPT], go4[VPT];
+  const uint16_t* st = a.style + r * a.style_stride;
   if (ok) {
     uint16_t* rr = a.res + r * D;
     const uint16_t* dd = a.delta + r * D;
@@ -109,6 +112,10 @@ __global__ void __launch_bounds__(512) adarms_kernel(ProducerArgs a) {
         rv4[i] = *reinterpret_cast<const uint4*>(rr + 8 * c);
         dv4[i] = ldg16(dd + 8 * c);
         gv4[i] = ldg16(gg + 8 * c);
+        sc4[i] = ldg16(st + 8 * c);
+        sh4[i] = ldg16(st + D + 8 * c);
+        if (a.weight) w4[i] = ldg16(a.weight + 8 * c);
+        if (a.gate_out) go4[i] = ldg16(st + 2 * D + 8 * c);
       }
     }
 #pragma unroll
@@ -134,20 +141,19 @@ __global__ void __launch_bounds__(512) adarms_kernel(ProducerArgs a) {
   const float ms = __fdiv_rn(ss, float(D));
   const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
   const float inv_as = __frcp_rn(__ldg(a.act_scale));  // quantize: y * (1 / scale)
-  const uint16_t* st = a.style + r * a.style_stride;
   float mx = 0.0f;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int c = t + i * G;
     if (c < C) {
       float wv[8], sc[8], sh[8];
-      if (a.weight) unpack8(ldg16(a.weight + 8 * c), wv);
+      if (a.weight) unpack8(w4[i], wv);
       else {
 #pragma unroll
         for (int j = 0; j < 8; ++j) wv[j] = 1.0f;
       }
-      unpack8(ldg16(st + 8 * c), sc);
-      unpack8(ldg16(st + D + 8 * c), sh);
+      unpack8(sc4[i], sc);
+      unpack8(sh4[i], sh);
       float q[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -160,7 +166,7 @@ __global__ void __launch_bounds__(512) adarms_kernel(ProducerArgs a) {
       }
       *reinterpret_cast<uint2*>(a.x8 + r * D + 8 * c) = pack8_e4m3(q);
       if (a.gate_out)
-        *reinterpret_cast<uint4*>(a.gate_out + r * D + 8 * c) = ldg16(st + 2 * D + 8 * c);
+        *reinterpret_cast<uint4*>(a.gate_out + r * D + 8 * c) = go4[i];
     }
   }
   if (a.amax) {
