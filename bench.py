@@ -385,43 +385,78 @@ class ChainRunner:
 
     # ---------------------------------------------------------------- e2e --
     def e2e_setup(self):
-        torch = self.torch
-        self.pin_in = {k: torch.from_numpy(v.view(np.int16)).pin_memory()
-                       for k, v in self.host_in.items()}
-        self.dev_in = ({"x": self.x, "temb": self.temb} if self.dit else
-                       {"res": self.res, "delta": self.delta,
-                        "prev_gate": self.gate, "style": self.style1})
+        """Host-buffer form of the step: the step's inputs sit back to back
+        in one pinned host buffer and one device arena (the chain's input
+        tensors become views of it), so a step copies them in with one
+        host->device copy; the residual, the last layer's q and gate outputs
+        follow them in the arena and come back with one device->host copy,
+        the new K/V cache rows with one copy each."""
+        torch, w, L = self.torch, self.w, self.L
+        lq = (L - 1) % 2
+        # (name, device tensor, host array or None, setter)
+        ins = []
+        if self.dit:
+            ins.append(("x", self.x, self.host_in["x"],
+                        lambda t: setattr(self, "x", t)))
+            ins.append(("temb", self.temb, self.host_in["temb"],
+                        lambda t: setattr(self, "temb", t)))
+        else:
+            ins.append(("delta", self.delta, self.host_in["delta"],
+                        lambda t: setattr(self, "delta", t)))
+            ins.append(("prev_gate", self.gate, self.host_in["prev_gate"],
+                        lambda t: setattr(self, "gate", t)))
+            ins.append(("style", self.style1, self.host_in["style"],
+                        lambda t: setattr(self, "style1", t)))
         for l, lay in enumerate(self.layers):
             if lay["pk_host"] is not None:
-                self.pin_in[f"pk{l}"] = torch.from_numpy(
-                    lay["pk_host"].view(np.int16)).pin_memory()
-                self.pin_in[f"pv{l}"] = torch.from_numpy(
-                    lay["pv_host"].view(np.int16)).pin_memory()
-                self.dev_in[f"pk{l}"] = lay["pkd"]
-                self.dev_in[f"pv{l}"] = lay["pvd"]
-        w = self.w
-        outs = {"q": self.q[(self.L - 1) % 2]}
-        for l, lay in enumerate(self.layers):
-            outs[f"k{l}"] = lay["kc"][:, w.P:w.P + w.M]
-            outs[f"v{l}"] = lay["vc"][:, w.P:w.P + w.M]
+                ins.append((f"pk{l}", lay["pkd"], lay["pk_host"],
+                            lambda t, lay=lay: lay.__setitem__("pkd", t)))
+                ins.append((f"pv{l}", lay["pvd"], lay["pv_host"],
+                            lambda t, lay=lay: lay.__setitem__("pvd", t)))
+        outs = []
+        if not self.dit:   # the residual is both an input and an output
+            ins.append(("res", self.res, self.host_in["res"],
+                        lambda t: setattr(self, "res", t)))
+        outs.append(("q", self.q[lq], lambda t: self.q.__setitem__(lq, t)))
         if not self.dit:
-            outs["res"] = self.res
-            outs["gate"] = self.gate_out[(self.L - 1) % 2]
-        self.dev_out = outs
-        self.pin_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory()
-                        for k, v in outs.items()}
-        self.h2d_bytes = sum(t.numel() * t.element_size()
-                             for t in self.pin_in.values())
-        self.d2h_bytes = sum(t.numel() * t.element_size()
-                             for t in self.pin_out.values())
+            outs.append(("gate", self.gate_out[lq],
+                         lambda t: self.gate_out.__setitem__(lq, t)))
+        offs, n = {}, 0
+        for name, t, *_ in ins + outs:
+            offs[name] = n
+            n += (t.numel() + 127) // 128 * 128   # 256-byte aligned slices
+        arena = torch.empty(n, dtype=torch.int16, device="cuda")
+        pin = torch.empty(n, dtype=torch.int16).pin_memory()
+        for name, t, host, setter in ins:
+            v = arena[offs[name]:offs[name] + t.numel()].view(t.dtype).view(t.shape)
+            v.copy_(t)
+            pin[offs[name]:offs[name] + t.numel()].copy_(
+                torch.from_numpy(np.ascontiguousarray(host).view(np.int16).reshape(-1)))
+            setter(v)
+        for name, t, setter in outs:
+            v = arena[offs[name]:offs[name] + t.numel()].view(t.dtype).view(t.shape)
+            setter(v)
+        self._build_descs()
+        self.arena, self.pin_arena = arena, pin
+        self.in_elems = offs["res"] + self.res.numel() if not self.dit else offs["q"]
+        self.out_lo = offs["res"] if not self.dit else offs["q"]
+        self.out_hi = n
+        self.pin_back = torch.empty(n - self.out_lo, dtype=torch.int16).pin_memory()
+        self.kv_out = []
+        for lay in self.layers:
+            for c in ("kc", "vc"):
+                src = lay[c][:, w.P:w.P + w.M]
+                self.kv_out.append((src, torch.empty(src.shape, dtype=src.dtype).pin_memory()))
+        self.h2d_bytes = 2 * self.in_elems
+        self.d2h_bytes = (2 * (self.out_hi - self.out_lo) +
+                          sum(t.numel() * t.element_size() for _, t in self.kv_out))
 
     def e2e_step(self):
-        for k, t in self.pin_in.items():
-            d = self.dev_in[k]
-            d.view(self.torch.int16).copy_(t.view(d.shape), non_blocking=True)
+        self.arena[:self.in_elems].copy_(self.pin_arena[:self.in_elems], non_blocking=True)
         self.step()
-        for k, t in self.pin_out.items():
-            t.copy_(self.dev_out[k], non_blocking=True)
+        self.pin_back.copy_(self.arena[self.out_lo:self.out_hi], non_blocking=True)
+        for src, dst in self.kv_out:
+            dst.copy_(src, non_blocking=True)
 
 
 class MlpRunner:
