@@ -74,6 +74,42 @@ def _src_hash(kernel_name):
     return h.hexdigest()[:16]
 
 
+def own_peaks(torch, frt):
+    """The library's own probes (frt_peak_fp8_mma, frt_peak_copy): best of
+    three timed launches each, CUDA events on the current stream."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    iters = 20000
+    flops = 2.0 * 128 * 256 * 128 * iters * sms
+
+    def best(fn, n=3):
+        fn()
+        torch.cuda.synchronize()
+        out = []
+        for _ in range(n):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            out.append(a.elapsed_time(b) * 1e-3)
+        return min(out)
+    t_mma = best(lambda: frt.frt_peak_fp8_mma(sms, iters))
+    nbytes = 1 << 30
+    src = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    dst = torch.empty_like(src)
+    src.fill_(1)
+    t_cp = best(lambda: frt.frt_peak_copy(src, dst, nbytes))
+    del src, dst
+    assert frt.frt_device_status(True) == frt.FRT_OK
+    return {"fp8_dense_tflops": round(flops / t_mma / 1e12, 1),
+            "hbm_copy_gbs": round(2.0 * nbytes / t_cp / 1e9, 1),
+            "method": f"tcgen05 e4m3 MMA loop, {sms} CTAs x {4 * iters} "
+                      "M128xN256xK32 MMAs from shared memory; 1 GiB "
+                      "device copy (read + write bytes); best of 3",
+            "datasheet": {"fp8_dense_tflops": 4500.0, "hbm_gbs": 7700.0}}
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -959,6 +995,7 @@ def run_gpu(args):
         unit = "GB/s"
     tr = NCU_TRAFFIC.get((args.config, kd.name))
     traffic = tr[0] if tr and tr[1] == _src_hash(kd.name) else None
+    own = own_peaks(torch, frt)
     kern_list = []
     for ms, k in zip(kern_ms, kinds):
         e = {"kernel": k.name, "us": round(ms * 1e3, 3),
@@ -970,6 +1007,8 @@ def run_gpu(args):
             e["TFLOP_s"] = round(k.flops / (ms * 1e-3) / 1e12, 2)
             e["fp8_frac"] = round(k.flops / (ms * 1e-3) / 1e12 /
                                   (bf16_burst * FP8_PER_BF16), 4)
+            e["fp8_frac_own"] = round(e["TFLOP_s"] / own["fp8_dense_tflops"], 4)
+        e["hbm_frac_own"] = round(e["GB_s"] / own["hbm_copy_gbs"], 4)
         kern_list.append(e)
 
     if rank != 0:
@@ -1005,6 +1044,7 @@ def run_gpu(args):
                      "algo_per_launch": kd.flops if unit == "TFLOP/s"
                      else kd.algo_bytes},
         "kernels": kern_list,
+        "peaks_own": own,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": int(first.h2d_bytes),

@@ -96,6 +96,8 @@ _SIGS = {
     "frt_chain_workspace_size": (_z, [C.POINTER(frt_chain_desc)]),
     "frt_chain_layer": (_i, [C.POINTER(frt_chain_desc), _p]),
     "frt_selftest_bounded_wait": (_i, [_i, _p]),
+    "frt_peak_fp8_mma": (_i, [_i, _i, _p]),
+    "frt_peak_copy": (_i, [_p, _p, C.c_size_t, _p]),
 }
 
 for _name, (_res, _args) in _SIGS.items():
@@ -243,6 +245,17 @@ def frt_chain_workspace_size(desc: frt_chain_desc) -> int:
 def frt_chain_layer(desc: frt_chain_desc, stream=None):
     return _check(_lib.frt_chain_layer(C.byref(desc), _stream(stream)),
                   "frt_chain_layer")
+
+
+def frt_peak_fp8_mma(ctas: int, iters: int, stream=None) -> None:
+    """Launch the dense FP8 tensor-core loop (the library's peak probe)."""
+    _check(_lib.frt_peak_fp8_mma(ctas, iters, _stream(stream)), "frt_peak_fp8_mma")
+
+
+def frt_peak_copy(src, dst, nbytes: int, stream=None) -> None:
+    """Launch the device-to-device copy probe over `nbytes`."""
+    _check(_lib.frt_peak_copy(ptr(src), ptr(dst), nbytes, _stream(stream)),
+           "frt_peak_copy")
 
 
 def frt_selftest_bounded_wait(timeout_us: int, stream=None) -> int:

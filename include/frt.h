@@ -338,6 +338,27 @@ int frt_chain_layer(const frt_chain_desc* d, void* stream);
  */
 int frt_selftest_bounded_wait(int timeout_us, void* stream);
 
+/* ----------------------------------------------------------------------- */
+/* The library's own peak probes (no counterpart on the pages).             */
+/* ----------------------------------------------------------------------- */
+
+/*
+ * Dense FP8 tensor-core loop: `ctas` CTAs (one per SM is the intended use)
+ * each issue 4 * iters tcgen05.mma.kind::f8f6f4 (M 128, N 256, K 32,
+ * e4m3 x e4m3 -> fp32 in TMEM) back to back from operands already in shared
+ * memory: 2 * 128 * 256 * 128 * iters flops per CTA and no memory traffic.
+ * The caller times the launch on `stream` (asynchronous).  FRT_EINVAL for
+ * ctas outside [1, 4096] or iters < 1.
+ */
+int frt_peak_fp8_mma(int ctas, int iters, void* stream);
+
+/*
+ * Device-to-device copy of `bytes` (16-byte aligned pointers, a multiple
+ * of 16) with streaming loads and stores: 2 * bytes of DRAM traffic when
+ * the buffers are far larger than L2.  Asynchronous on `stream`.
+ */
+int frt_peak_copy(const void* src, void* dst, size_t bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
