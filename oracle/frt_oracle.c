@@ -477,6 +477,69 @@ void or_geglu_quant(int M, int H, const uint16_t *gu, float out_scale,
     free(row_amax);
 }
 
+/* ------------------------------------------------------------------ */
+/* Static quantize of the attention output ([fp8_chain] `out_project`: */
+/* quantize_fp8_static_bf16(att2, t_sc_o) before the o_proj GEMM).      */
+/* ------------------------------------------------------------------ */
+/*
+ *   x8[r, j] = q8(x[r, j]; scale)        x bf16 [rows, D], row stride ldx
+ *   amax     = max |x|                   (the calibration statistic)
+ */
+void or_quant_fp8_static(int rows, int D, const uint16_t *x, long ldx, float scale,
+                         uint8_t *x8, float *amax_out)
+{
+    float mx = 0.0f;
+    for (int r = 0; r < rows; ++r) {
+        for (int j = 0; j < D; ++j) {
+            float v = or_bf16_to_f32(x[(long)r * ldx + j]);
+            x8[(long)r * D + j] = q8(v, scale);
+            if (fabsf(v) > mx) mx = fabsf(v);
+        }
+    }
+    if (amax_out) *amax_out = mx;
+}
+
+/* ------------------------------------------------------------------ */
+/* Final AdaRMS tail of the stack ([fp8_chain] `_make_run`, the         */
+/* "ad:tail" range after the layer loop).                               */
+/* ------------------------------------------------------------------ */
+/*
+ * Per row r, all fp32 (the page lifts res, gate and delta to fp32 and does
+ * not round the sum to bf16 before the norm):
+ *   h_j   = res_j + gate_j * delta_j
+ *   ms    = (sum_j h_j^2) / D
+ *   out_j = bf16((h_j * (1 / sqrt(ms + eps))) * (1 + fin[0, j]) + fin[1, j])
+ * fin: fp32 rows (scale, shift) of the last norm, fin_stride elements apart
+ * (the page keeps them fp32: they are sliced from the fp32 projection
+ * before the bf16 cast of the styles).  gate_stride 0 broadcasts one gate
+ * row.  The page writes torch.rsqrt; the reading here is 1 / sqrt, the
+ * same as the producer's.
+ */
+void or_ada_rms_tail(int rows, int D, float eps, const uint16_t *res,
+                     const uint16_t *delta, const uint16_t *gate, long gate_stride,
+                     const float *fin, long fin_stride, uint16_t *out)
+{
+    float *h = (float *)malloc((size_t)(D > 0 ? D : 1) * sizeof(float));
+    for (int r = 0; r < rows; ++r) {
+        const uint16_t *rr = res + (long)r * D;
+        const uint16_t *dd = delta + (long)r * D;
+        const uint16_t *gg = gate + (long)r * gate_stride;
+        float ss = 0.0f;
+        for (int j = 0; j < D; ++j) {
+            h[j] = or_bf16_to_f32(rr[j]) + or_bf16_to_f32(gg[j]) * or_bf16_to_f32(dd[j]);
+            ss = ss + h[j] * h[j];
+        }
+        float ms = ss / (float)D;
+        float inv = 1.0f / sqrtf(ms + eps);
+        for (int j = 0; j < D; ++j) {
+            float t = h[j] * inv;
+            t = t * (1.0f + fin[j]);
+            out[(long)r * D + j] = or_bf16_from_f32(t + fin[fin_stride + j]);
+        }
+    }
+    free(h);
+}
+
 /* OpenMP thread count the oracle runs with (1 without OpenMP). */
 int or_num_threads(void)
 {

@@ -25,7 +25,7 @@ __all__ = [
     "bf16_to_f32", "f32_to_bf16", "f64_to_bf16", "e4m3_to_f32", "f32_to_e4m3",
     "ada_rms_norm_quant", "ada_layer_norm_quant_table", "pack_weights_fp8",
     "fp8_gemm", "rope_table", "split_rope_kvcache", "prefix_copy",
-    "geglu_quant",
+    "geglu_quant", "quant_fp8_static", "ada_rms_tail",
 ]
 
 
@@ -70,6 +70,8 @@ def _L():
                                              p]),
             "or_prefix_copy": (None, [i, i, i, i, i, i, p, p, i, p, p]),
             "or_geglu_quant": (None, [i, i, p, f, p, p]),
+            "or_quant_fp8_static": (None, [i, i, p, l, f, p, p]),
+            "or_ada_rms_tail": (None, [i, i, f, p, p, p, l, p, l, p]),
             "or_num_threads": (i, []),
         }
         for name, (res, args) in sig.items():
@@ -244,6 +246,33 @@ def prefix_copy(prefix_k, prefix_v, P, k_cache, v_cache, interleave=True):
                         _ptr(prefix_v), int(bool(interleave)), _ptr(k_cache),
                         _ptr(v_cache))
     return k_cache, v_cache
+
+
+def quant_fp8_static(x, scale):
+    """[fp8_chain] out_project's static quantize: x8 = q8(x; scale) for a
+    bf16-bits array x [rows, D]; returns (x8, amax of |x|)."""
+    x = _c(x, np.uint16)
+    rows, D = x.shape
+    x8 = np.empty((rows, D), np.uint8)
+    amax = np.zeros(1, np.float32)
+    _L().or_quant_fp8_static(rows, D, _ptr(x), D, float(scale), _ptr(x8), _ptr(amax))
+    return x8, float(amax[0])
+
+
+def ada_rms_tail(res, delta, gate, fin, eps):
+    """[fp8_chain] _make_run's final tail: bf16 bits [rows, D] of
+    RMSnorm(res + gate*delta) * (1 + fin[0]) + fin[1] (fp32 throughout).
+    gate is [1, D] (broadcast) or [rows, D]; fin is fp32 [2 or 3, D]."""
+    res = _c(res, np.uint16)
+    delta = _c(delta, np.uint16)
+    gate = _c(gate, np.uint16)
+    fin = _c(fin, np.float32)
+    rows, D = res.shape
+    out = np.empty((rows, D), np.uint16)
+    gs = 0 if gate.shape[0] == 1 else D
+    _L().or_ada_rms_tail(rows, D, float(eps), _ptr(res), _ptr(delta), _ptr(gate), gs,
+                         _ptr(fin), fin.shape[1], _ptr(out))
+    return out
 
 
 def geglu_quant(gu, out_scale):

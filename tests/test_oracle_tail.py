@@ -1,0 +1,87 @@
+"""Pins of the oracle's output-side pieces of the AdaRMS layer: the static
+quantize in front of the output projection and the stack's final AdaRMS
+tail (impls/adarms_stack/fp8_chain.py: `out_project`, and the "ad:tail"
+range of `_make_run`).  Each check is a value the definitions fix."""
+
+import numpy as np
+
+import oracle
+
+
+def _bf16(x):
+    return oracle.f32_to_bf16(np.asarray(x, dtype=np.float32))
+
+
+def test_quant_roundtrips_every_finite_code():
+    # dec(c) * 2^-3 is exact in bf16 for every finite e4m3 code c, so the
+    # quantizer must return c itself (signed zero included)
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    vals = oracle.e4m3_to_f32(codes) * np.float32(0.125)
+    x = _bf16(vals).reshape(1, -1)
+    assert np.array_equal(oracle.bf16_to_f32(x[0]), vals)
+    x8, amax = oracle.quant_fp8_static(x, 0.125)
+    assert np.array_equal(x8[0], codes)
+    assert amax == 448.0 * 0.125
+
+
+def test_quant_saturates_and_keeps_sign():
+    s = 0.25
+    x = _bf16([[449 * s, -449 * s, 1000 * s, -1000 * s, 0.0, -0.0, 3e-7, -3e-7]])
+    x8, amax = oracle.quant_fp8_static(x, s)
+    assert list(x8[0]) == [0x7E, 0xFE, 0x7E, 0xFE, 0x00, 0x80, 0x00, 0x80]
+    assert amax == float(oracle.bf16_to_f32(x[0, 2]))
+
+
+def _tail(res, delta, gate, scale, shift, eps=1e-6):
+    res, delta, gate = (np.atleast_2d(np.asarray(a, np.uint16)) for a in (res, delta, gate))
+    D = res.shape[1]
+    fin = np.stack([np.broadcast_to(np.float32(scale), (D,)),
+                    np.broadcast_to(np.float32(shift), (D,))]).astype(np.float32)
+    return oracle.ada_rms_tail(res, delta, gate, fin, eps)
+
+
+def test_tail_unit_rms_row_maps_to_plus_minus_one():
+    h = _bf16([1, -1, 1, -1, 1, -1, 1, -1]).reshape(1, 8)
+    z = np.zeros((1, 8), np.uint16)
+    out = _tail(h, z, z, 0.0, 0.0)
+    # ms = 1, 1/sqrt(1 + 1e-6) rounds, after the product, to +-1 in bf16
+    assert list(out[0]) == [0x3F80, 0xBF80] * 4
+
+
+def test_tail_gated_delta_equals_the_same_residual():
+    rng = np.random.default_rng(3)
+    x = _bf16(rng.normal(size=(4, 64)))
+    half = _bf16(oracle.bf16_to_f32(x) * np.float32(0.5))   # exact: a power of two
+    two = _bf16(np.full((1, 64), 2.0))
+    z = np.zeros((4, 64), np.uint16)
+    a = _tail(x, z, np.zeros((1, 64), np.uint16), 0.3, -0.2)
+    b = _tail(z, half, two, 0.3, -0.2)
+    assert np.array_equal(a, b)
+
+
+def test_tail_scale_minus_one_leaves_the_shift():
+    rng = np.random.default_rng(4)
+    x = _bf16(rng.normal(size=(3, 32)))
+    z = np.zeros((3, 32), np.uint16)
+    out = _tail(x, z, np.zeros((1, 32), np.uint16), -1.0, 0.375)
+    assert np.all(out == _bf16(0.375))
+
+
+def test_tail_output_has_unit_rms():
+    rng = np.random.default_rng(5)
+    x = _bf16(rng.normal(size=(16, 512)) * 3.0)
+    z = np.zeros((16, 512), np.uint16)
+    y = oracle.bf16_to_f32(_tail(x, z, np.zeros((1, 512), np.uint16), 0.0, 0.0))
+    ms = (y.astype(np.float64) ** 2).mean(axis=1)
+    assert np.all(np.abs(ms - 1.0) < 1e-2)
+
+
+def test_tail_norm_sees_the_unrounded_sum():
+    # h = (1 + 2^-9, 1) is not a bf16 pair: rms(h) = 1 + 2^-10 (to first
+    # order), so h / rms(h) - 1 = (+2^-10, -2^-10); rounding h to bf16 first
+    # would give (1, 1) and an output of ~0 in both columns
+    res = _bf16([[1.0, 1.0]])
+    delta = _bf16([[2.0 ** -9, 0.0]])
+    gate = _bf16([[1.0, 1.0]])
+    out = oracle.bf16_to_f32(_tail(res, delta, gate, 0.0, -1.0))
+    assert abs(out[0, 0] - 2.0 ** -10) < 1e-4 and abs(out[0, 1] + 2.0 ** -10) < 1e-4
