@@ -96,6 +96,8 @@ _SIGS = {
     "frt_chain_workspace_size": (_z, [C.POINTER(frt_chain_desc)]),
     "frt_chain_layer": (_i, [C.POINTER(frt_chain_desc), _p]),
     "frt_selftest_bounded_wait": (_i, [_i, _p]),
+    "frt_quantize_fp8_static": (_i, [_i, _i, _p, _l, _p, _p, _p, _p]),
+    "frt_ada_rms_tail": (_i, [_i, _i, _f, _p, _p, _p, _l, _p, _l, _p, _p]),
     "frt_peak_fp8_mma": (_i, [_i, _i, _p]),
     "frt_peak_copy": (_i, [_p, _p, C.c_size_t, _p]),
 }
@@ -245,6 +247,24 @@ def frt_chain_workspace_size(desc: frt_chain_desc) -> int:
 def frt_chain_layer(desc: frt_chain_desc, stream=None):
     return _check(_lib.frt_chain_layer(C.byref(desc), _stream(stream)),
                   "frt_chain_layer")
+
+
+def frt_quantize_fp8_static(rows, D, x, ldx, act_scale, x8_out, amax_out=None,
+                            stream=None) -> None:
+    """Static e4m3 quantize of a bf16 activation (the o_proj input)."""
+    _check(_lib.frt_quantize_fp8_static(rows, D, ptr(x), ldx, ptr(act_scale), ptr(x8_out),
+                                        ptr(amax_out), _stream(stream)),
+           "frt_quantize_fp8_static")
+
+
+def frt_ada_rms_tail(rows, D, eps, res, delta, gate, gate_row_stride, fin, fin_row_stride,
+                     out, stream=None) -> None:
+    """The stack's final AdaRMS tail: bf16(RMSnorm(res + gate*delta) *
+    (1 + fin[0]) + fin[1])."""
+    _check(_lib.frt_ada_rms_tail(rows, D, eps, ptr(res), ptr(delta), ptr(gate),
+                                 gate_row_stride, ptr(fin), fin_row_stride, ptr(out),
+                                 _stream(stream)),
+           "frt_ada_rms_tail")
 
 
 def frt_peak_fp8_mma(ctas: int, iters: int, stream=None) -> None:

@@ -327,6 +327,38 @@ size_t frt_chain_workspace_size(const frt_chain_desc* d);
 int frt_chain_layer(const frt_chain_desc* d, void* stream);
 
 /* ----------------------------------------------------------------------- */
+/* Output side of the AdaRMS layer (fp8_chain.py `out_project`, "ad:tail").  */
+/* ----------------------------------------------------------------------- */
+
+/*
+ * frt_quantize_fp8_static (fp8_chain.py `out_project`: the attention output
+ * quantized with the site's static scale, t_sc_o, before the o_proj GEMM):
+ *   x8[r, j] = e4m3_rne_sat(x[r, j] / act_scale[0])   (IEEE fp32 division)
+ * x: bf16 [rows, ldx] (device, 16-byte aligned, ldx >= D,
+ * ldx % 8 == 0); act_scale: device fp32 [1]; x8_out: [rows, D] e4m3, 8-byte
+ * aligned.  amax_out (nullable, device fp32 [1], caller-zeroed) receives
+ * max |x| via atomic max.  D % 8 == 0.  rows == 0 is a no-op.
+ */
+int frt_quantize_fp8_static(int rows, int D, const frt_bf16* x, long ldx,
+                            const float* act_scale, frt_e4m3* x8_out,
+                            float* amax_out, void* stream);
+
+/*
+ * frt_ada_rms_tail (fp8_chain.py `_make_run`, the "ad:tail" range after
+ * the layer loop), per row r, fp32 throughout:
+ *   h_j   = res[r, j] + gate[r|0, j] * delta[r, j]     (not rounded to bf16)
+ *   out_j = bf16((h_j / sqrt(mean_j h^2 + eps)) * (1 + fin[j]) + fin[fin_row_stride + j])
+ * res, delta, out: bf16 [rows, D]; gate: bf16 rows gate_row_stride apart
+ * (0 = one broadcast row); fin: device fp32, the last norm's scale row and,
+ * fin_row_stride elements later, its shift row (one row each, broadcast
+ * over tokens).  All 16-byte aligned; D % 8 == 0, 8 <= D <= 8192.
+ */
+int frt_ada_rms_tail(int rows, int D, float eps, const frt_bf16* res,
+                     const frt_bf16* delta, const frt_bf16* gate,
+                     long gate_row_stride, const float* fin, long fin_row_stride,
+                     frt_bf16* out, void* stream);
+
+/* ----------------------------------------------------------------------- */
 /* Self-test of the bounded device wait.                                    */
 /* ----------------------------------------------------------------------- */
 
