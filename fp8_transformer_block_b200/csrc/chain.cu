@@ -65,3 +65,40 @@ extern "C" int frt_chain_layer(const frt_chain_desc* d, void* stream) {
                                 d->q_out, d->k_cache, d->v_cache, d->prefix_k, d->prefix_v,
                                 d->prefix_T_src, d->prefix_interleave, stream);
 }
+
+// ---------------------------------------------------------------- FFN half --
+//
+// fp8_chain.py `_make_run`, the second half of the layer loop:
+// norm_project(styles, 2l + 1, dn, g1, e, "gu", gu, g2) -- the AdaRMS
+// producer at the FFN site feeding the packed gate/up GEMM -- then
+// `down_project`: the merged GEGLU + static requant (here the gate/up GEMM's
+// epilogue) and the FP8 down projection.  Three launches, each with
+// programmatic dependent launch.
+
+extern "C" size_t frt_ffn_workspace_size(const frt_ffn_desc* d) {
+  if (!d || d->rows <= 0 || d->D <= 0 || d->H <= 0) return 0;
+  const size_t a = frt_gemm_workspace_size(d->rows, 2 * d->H, d->D, FRT_EPI_GEGLU_E4M3);
+  const size_t b = frt_gemm_workspace_size(d->rows, d->D, d->H, FRT_EPI_BF16);
+  return a > b ? a : b;
+}
+
+extern "C" int frt_ffn_layer(const frt_ffn_desc* d, void* stream) {
+  frt::clear_error();
+  FRT_REQUIRE(d, FRT_EINVAL, "descriptor is NULL");
+  FRT_REQUIRE(d->rows >= 0 && d->D > 0 && d->H > 0, FRT_ESHAPE, "bad rows/D/H");
+  FRT_REQUIRE(d->x8 && d->hid8 && d->out, FRT_EINVAL, "x8, hid8 and out are required");
+  if (d->rows == 0) return FRT_OK;
+  int rc = frt::producer_call(FRT_NORM_ADARMS, d->rows, d->D, d->eps, d->res, d->delta,
+                              d->prev_gate, d->gate_row_stride, d->norm_weight, d->style,
+                              d->style_row_stride, nullptr, nullptr, 0, nullptr, 0, 0,
+                              d->act_scale, d->x8, d->gate_out, nullptr, nullptr,
+                              static_cast<cudaStream_t>(stream));
+  if (rc) return rc;
+  rc = frt_packed_fp8_gemm(d->rows, 2 * d->H, d->D, d->x8, d->w8_gu, d->act_scale, d->w_scale_gu,
+                           d->bias_gu, FRT_EPI_GEGLU_E4M3, d->hid8, d->H, d->hid_scale,
+                           d->workspace, d->workspace_bytes, stream);
+  if (rc) return rc;
+  return frt_packed_fp8_gemm(d->rows, d->D, d->H, d->hid8, d->w8_dn, d->hid_scale,
+                             d->w_scale_dn, d->bias_dn, FRT_EPI_BF16, d->out, d->D, nullptr,
+                             d->workspace, d->workspace_bytes, stream);
+}

@@ -71,6 +71,19 @@ class frt_chain_desc(C.Structure):
     ]
 
 
+class frt_ffn_desc(C.Structure):
+    """Mirror of ``frt_ffn_desc`` in include/frt.h (same field order)."""
+    _fields_ = [
+        ("rows", _i), ("D", _i), ("H", _i), ("eps", _f),
+        ("res", _p), ("delta", _p), ("prev_gate", _p), ("gate_row_stride", _l),
+        ("norm_weight", _p), ("style", _p), ("style_row_stride", _l),
+        ("gate_out", _p), ("act_scale", _p), ("x8", _p),
+        ("w8_gu", _p), ("w_scale_gu", _p), ("bias_gu", _p), ("hid_scale", _p),
+        ("hid8", _p), ("w8_dn", _p), ("w_scale_dn", _p), ("bias_dn", _p),
+        ("out", _p), ("workspace", _p), ("workspace_bytes", _z),
+    ]
+
+
 _SIGS = {
     "frt_last_error": (C.c_char_p, []),
     "frt_version": (_i, []),
@@ -95,6 +108,8 @@ _SIGS = {
     "frt_geglu_quant_fp8": (_i, [_i, _i, _p, _l, _p, _p, _p, _p]),
     "frt_chain_workspace_size": (_z, [C.POINTER(frt_chain_desc)]),
     "frt_chain_layer": (_i, [C.POINTER(frt_chain_desc), _p]),
+    "frt_ffn_workspace_size": (_z, [C.POINTER(frt_ffn_desc)]),
+    "frt_ffn_layer": (_i, [C.POINTER(frt_ffn_desc), _p]),
     "frt_selftest_bounded_wait": (_i, [_i, _p]),
     "frt_quantize_fp8_static": (_i, [_i, _i, _p, _l, _p, _p, _p, _p]),
     "frt_ada_rms_tail": (_i, [_i, _i, _f, _p, _p, _p, _l, _p, _l, _p, _p]),
@@ -247,6 +262,14 @@ def frt_chain_workspace_size(desc: frt_chain_desc) -> int:
 def frt_chain_layer(desc: frt_chain_desc, stream=None):
     return _check(_lib.frt_chain_layer(C.byref(desc), _stream(stream)),
                   "frt_chain_layer")
+
+
+def frt_ffn_workspace_size(desc: frt_ffn_desc) -> int:
+    return int(_lib.frt_ffn_workspace_size(C.byref(desc)))
+
+
+def frt_ffn_layer(desc: frt_ffn_desc, stream=None):
+    return _check(_lib.frt_ffn_layer(C.byref(desc), _stream(stream)), "frt_ffn_layer")
 
 
 def frt_quantize_fp8_static(rows, D, x, ldx, act_scale, x8_out, amax_out=None,

@@ -104,3 +104,12 @@ def chain_desc(**kw) -> frt.frt_chain_desc:
         else:
             setattr(d, k, v)
     return d
+
+
+def ffn_desc(**kw) -> frt.frt_ffn_desc:
+    """Build an frt_ffn_desc; tensor fields accept tensors/ints/None."""
+    d = frt.frt_ffn_desc()
+    ptr_fields = {name for name, typ in frt.frt_ffn_desc._fields_ if typ is frt._p}
+    for k, v in kw.items():
+        setattr(d, k, frt.ptr(v) if k in ptr_fields else v)
+    return d

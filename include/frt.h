@@ -327,6 +327,51 @@ size_t frt_chain_workspace_size(const frt_chain_desc* d);
 int frt_chain_layer(const frt_chain_desc* d, void* stream);
 
 /* ----------------------------------------------------------------------- */
+/* The FFN half of the AdaRMS layer (fp8_chain.py `_make_run`:               */
+/* norm_project(styles, 2l + 1, dn, g1, e, "gu", gu, g2), then               */
+/* `down_project`).                                                          */
+/* ----------------------------------------------------------------------- */
+
+typedef struct frt_ffn_desc {
+  int rows, D, H;         /* tokens, model width, FFN hidden width         */
+  float eps;
+  /* AdaRMS producer at the FFN site (see frt_ada_norm_quant_fp8, mode 0)   */
+  frt_bf16* res;          /* [rows, D] residual, updated in place          */
+  const frt_bf16* delta;  /* [rows, D] the output projection's result      */
+  const frt_bf16* prev_gate; long gate_row_stride; /* the attention norm's gate */
+  const frt_bf16* norm_weight;                      /* nullable = ones      */
+  const frt_bf16* style; long style_row_stride;     /* this norm's (scale, shift, gate) */
+  frt_bf16* gate_out;     /* nullable: [rows, D], this norm's gate         */
+  const float* act_scale; /* device [1]: static scale of the producer      */
+  frt_e4m3* x8;           /* [rows, D] staging                             */
+  /* gate/up projection with the GEGLU requant epilogue                     */
+  const frt_e4m3* w8_gu;  /* [2H, D], FRT_PACK_GATE_UP_BLOCKS layout       */
+  const float* w_scale_gu;
+  const frt_bf16* bias_gu;    /* nullable, [2H] in the same layout         */
+  const float* hid_scale; /* device [1]: static scale of the GEGLU output  */
+  frt_e4m3* hid8;         /* [rows, H] staging                             */
+  /* down projection                                                         */
+  const frt_e4m3* w8_dn;  /* [D, H] */
+  const float* w_scale_dn;
+  const frt_bf16* bias_dn;    /* nullable, [D] */
+  frt_bf16* out;          /* [rows, D] bf16: the next layer's delta        */
+  void* workspace; size_t workspace_bytes;  /* both GEMMs, used in turn   */
+} frt_ffn_desc;
+
+/* Workspace bytes frt_ffn_layer needs (the larger of its two GEMMs'). */
+size_t frt_ffn_workspace_size(const frt_ffn_desc* d);
+
+/*
+ * frt_ffn_layer: the producer at the FFN site (res += prev_gate * delta,
+ * AdaRMS, static quantize into x8, gate out), the packed gate/up GEMM with
+ * the GEGLU + static requant epilogue into hid8, and the down projection
+ * into out: three launches on `stream`, each starting while its
+ * predecessor drains.  Shapes: D and H multiples of 16, 2H a multiple of
+ * 256; errors as the underlying entry points report them.
+ */
+int frt_ffn_layer(const frt_ffn_desc* d, void* stream);
+
+/* ----------------------------------------------------------------------- */
 /* Output side of the AdaRMS layer (fp8_chain.py `out_project`, "ad:tail").  */
 /* ----------------------------------------------------------------------- */
 

@@ -144,3 +144,12 @@ def test_chain_desc_layout_matches_header(frt):
     body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
     names = re.findall(r"\**\s*([A-Za-z_][A-Za-z0-9_]*)\s*(?=[,;])", body)
     assert names == [f for f, _ in frt.frt_chain_desc._fields_]
+
+
+def test_ffn_desc_layout_matches_header(frt):
+    src = open(os.path.join(ROOT, "include", "frt.h")).read()
+    body = src[src.index("typedef struct frt_ffn_desc"):]
+    body = body[:body.index("} frt_ffn_desc;")]
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    names = re.findall(r"\**\s*([A-Za-z_][A-Za-z0-9_]*)\s*(?=[,;])", body)
+    assert names == [f for f, _ in frt.frt_ffn_desc._fields_]

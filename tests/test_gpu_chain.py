@@ -329,3 +329,85 @@ def test_gateup_mlp_chain(rt):
     rel_o = np.linalg.norm(og - orf) / np.linalg.norm(orf)
     print(f"gate/up MLP down output: rel-L2 {rel_o:.3e}")
     assert rel_o <= 2e-2, "down projection end to end"
+
+
+def test_ffn_layer_entry(rt):
+    """frt_ffn_layer (the FFN half: producer at the FFN site -> gate/up GEMM
+    with the fused GEGLU requant -> down GEMM) equals the three entry points
+    called one by one, bit for bit, and the oracle within the chain's bars."""
+    frt, runtime, torch = rt
+    w = synth.WORKLOADS["gateup_mlp"]
+    M, D, H = 96, 1024, 4096
+    mw = synth.mlp_weights(D, H, w.seed + 1)
+    inp = synth.adarms_inputs(M, D, w.seed + 1)
+    rng = np.random.default_rng(11)
+    gate_rows = synth.normal_bf16(rng, (M, D), 0.5)   # per-row gate of the previous norm
+    pr0 = oracle.ada_rms_norm_quant(inp["res"], inp["delta"], gate_rows, inp["style"], 1.0)
+    a_gu = max(pr0["amax"] / 448.0, 1e-8)
+    pr = oracle.ada_rms_norm_quant(inp["res"], inp["delta"], gate_rows, inp["style"], a_gu)
+    gu_ref = oracle.pack_weights_fp8([mw["gate"], mw["up"]])
+    dn_ref = oracle.pack_weights_fp8([mw["down"]])
+    gu = oracle.fp8_gemm(pr["x8"], gu_ref["w8"], a_gu, gu_ref["w_scale"])
+    _, amax = oracle.geglu_quant(gu, 1.0)
+    a_dn = amax / 448.0
+    hid_ref, _ = oracle.geglu_quant(gu, a_dn)
+    out_ref = oracle.fp8_gemm(hid_ref, dn_ref["w8"], a_dn, dn_ref["w_scale"])
+
+    blk = runtime.pack([mw["gate"], mw["up"]], layout=frt.FRT_PACK_GATE_UP_BLOCKS)
+    dn = runtime.pack([mw["down"]])
+    s_gu, s_dn = runtime.scale_dev(a_gu), runtime.scale_dev(a_dn)
+    delta, gate = runtime.bf16_dev(inp["delta"]), runtime.bf16_dev(gate_rows)
+    style = runtime.bf16_dev(inp["style"])
+
+    def run_entry():
+        res = runtime.bf16_dev(inp["res"])
+        x8, hid = runtime.empty_u8(M, D), runtime.empty_u8(M, H)
+        out, g_out = runtime.empty_bf16(M, D), runtime.empty_bf16(M, D)
+        d = runtime.ffn_desc(rows=M, D=D, H=H, eps=w.eps, res=res, delta=delta,
+                             prev_gate=gate, gate_row_stride=D, norm_weight=None,
+                             style=style, style_row_stride=0, gate_out=g_out,
+                             act_scale=s_gu, x8=x8, w8_gu=blk.w8, w_scale_gu=blk.w_scale,
+                             bias_gu=None, hid_scale=s_dn, hid8=hid, w8_dn=dn.w8,
+                             w_scale_dn=dn.w_scale, bias_dn=None, out=out)
+        wsb = frt.frt_ffn_workspace_size(d)
+        ws = runtime.workspace(wsb)
+        d.workspace, d.workspace_bytes = frt.ptr(ws), wsb
+        frt.frt_ffn_layer(d)
+        torch.cuda.synchronize()
+        return res, x8, hid, out, g_out
+
+    def run_calls():
+        res = runtime.bf16_dev(inp["res"])
+        x8, hid = runtime.empty_u8(M, D), runtime.empty_u8(M, H)
+        out, g_out = runtime.empty_bf16(M, D), runtime.empty_bf16(M, D)
+        frt.frt_ada_norm_quant_fp8(frt.FRT_NORM_ADARMS, M, D, w.eps, res, delta, gate, D,
+                                   None, style, 0, None, None, 0, None, 0, 0, s_gu, x8,
+                                   g_out, None)
+        ws1 = frt.frt_gemm_workspace_size(M, 2 * H, D, frt.FRT_EPI_GEGLU_E4M3)
+        frt.frt_packed_fp8_gemm(M, 2 * H, D, x8, blk.w8, s_gu, blk.w_scale, None,
+                                frt.FRT_EPI_GEGLU_E4M3, hid, H, s_dn,
+                                runtime.workspace(ws1), ws1)
+        ws2 = frt.frt_gemm_workspace_size(M, D, H)
+        frt.frt_packed_fp8_gemm(M, D, H, hid, dn.w8, s_dn, dn.w_scale, None,
+                                frt.FRT_EPI_BF16, out, D, None, runtime.workspace(ws2), ws2)
+        torch.cuda.synchronize()
+        return res, x8, hid, out, g_out
+
+    a, b = run_entry(), run_calls()
+    for name, ta, tb in zip(("res", "x8", "hid8", "out", "gate_out"), a, b):
+        assert torch.equal(ta.view(torch.uint8), tb.view(torch.uint8)), name
+    res, x8, hid, out, g_out = (runtime.bf16_host(a[0]), runtime.u8_host(a[1]),
+                                runtime.u8_host(a[2]), runtime.bf16_host(a[3]),
+                                runtime.bf16_host(a[4]))
+    assert np.array_equal(res, pr["res"])
+    assert np.array_equal(g_out, pr["gate_out"])
+    assert_codes(x8, pr["x8"], what="x8")
+    d8 = e4m3_step_distance(hid, hid_ref)
+    dq_g = oracle.e4m3_to_f32(hid).astype(np.float64)
+    dq_r = oracle.e4m3_to_f32(hid_ref).astype(np.float64)
+    assert (d8 == 0).mean() >= 0.99
+    assert np.linalg.norm(dq_g - dq_r) / np.linalg.norm(dq_r) <= 2e-2
+    og = bf16_value(out).astype(np.float64)
+    orf = bf16_value(out_ref).astype(np.float64)
+    assert np.linalg.norm(og - orf) / np.linalg.norm(orf) <= 2e-2
+    assert frt.frt_device_status(True) == frt.FRT_OK
