@@ -60,8 +60,10 @@ def outlier_rows(rng: np.random.Generator, rows: int, frac: float = 0.01):
 class Workload:
     """One of the five shapes.  ``kind`` is "adarms" (AdaRMS producer +
     q/k/v chain), "dit" (per-token-table LayerNorm + biased q/k/v),
-    "mlp" (AdaRMS producer + gate/up GEMM + GEGLU + down GEMM) or
-    "stack" (``layers`` AdaRMS chain layers, residual carried)."""
+    "mlp" (AdaRMS producer + gate/up GEMM + GEGLU + down GEMM),
+    "stack" (``layers`` AdaRMS chain layers, residual carried) or "full"
+    (``layers`` whole AdaRMS layers except attention: the q/k/v chain, the
+    output projection, the FFN half; then the final tail)."""
     name: str
     cid: int
     kind: str
@@ -97,7 +99,7 @@ class Workload:
         return (self.hq + 2 * self.hkv) * self.hd
 
     def with_M(self, M: int) -> "Workload":
-        T = self.P + M if self.kind == "stack" else self.T
+        T = self.P + M if self.kind in ("stack", "full") else self.T
         return Workload(**{**self.__dict__, "M": M, "T": T})
 
 
@@ -116,6 +118,12 @@ WORKLOADS = {
                                hq=8, hkv=1, hd=64, P=816, T=866, layers=18,
                                cal_rows=64,
                                m_sweep=(1, 16, 50, 256, 1024, 4096)),
+    # not one of the five configurations: the stack's layers made whole
+    # except attention (FFN hidden 4 * D, a reading: the pages give none
+    # for this shape)
+    "adarms_layer18": Workload("adarms_layer18", 5, "full", B=1, M=50, D=512,
+                               hq=8, hkv=1, hd=64, P=816, T=866, H=2048,
+                               layers=18, cal_rows=64),
 }
 
 
@@ -179,3 +187,25 @@ def stack_layer_inputs(w: Workload, layer: int):
     style = normal_bf16(rng, (1, 3 * w.D), 0.02 * np.sqrt(w.D))
     pk, pv = prefix_cache(w.B, w.hkv, w.P, w.hd, s)
     return {"w": ws, "b": bs, "style": style, "prefix_k": pk, "prefix_v": pv}
+
+
+def full_layer_inputs(w: Workload, layer: int):
+    """Per-layer fresh weights of a whole AdaRMS layer (q/k/v, o, gate/up,
+    down), the two norms' styles (attention site, FFN site) and the prefix."""
+    s = w.seed + 1000 * (layer + 1)
+    ws, bs = qkv_weights(w.hq, w.hkv, w.hd, w.D, s)
+    rng = np.random.Generator(np.random.PCG64(s))
+    styles = normal_bf16(rng, (2, 3 * w.D), 0.02 * np.sqrt(w.D))
+    o = normal_bf16(np.random.Generator(np.random.PCG64(s + 17)), (w.D, w.hq * w.hd), 0.02)
+    mw = mlp_weights(w.D, w.H, s)
+    pk, pv = prefix_cache(w.B, w.hkv, w.P, w.hd, s)
+    return {"w": ws, "b": bs, "o": o, "mlp": mw, "styles": styles,
+            "prefix_k": pk, "prefix_v": pv}
+
+
+def final_norm_rows(w: Workload):
+    """fp32 (scale, shift, gate) rows of the final norm, the modulation
+    projection's distribution."""
+    rng = np.random.Generator(np.random.PCG64(w.seed + 31337))
+    return (rng.standard_normal(size=(3, w.D), dtype=np.float32)
+            * np.float32(0.02 * np.sqrt(w.D)))

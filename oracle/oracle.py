@@ -25,7 +25,7 @@ __all__ = [
     "bf16_to_f32", "f32_to_bf16", "f64_to_bf16", "e4m3_to_f32", "f32_to_e4m3",
     "ada_rms_norm_quant", "ada_layer_norm_quant_table", "pack_weights_fp8",
     "fp8_gemm", "rope_table", "split_rope_kvcache", "prefix_copy",
-    "geglu_quant", "quant_fp8_static", "ada_rms_tail",
+    "geglu_quant", "quant_fp8_static", "ada_rms_tail", "adarms_layer_stack",
 ]
 
 
@@ -284,3 +284,76 @@ def geglu_quant(gu, out_scale):
     _L().or_geglu_quant(M, H, _ptr(gu), float(out_scale), _ptr(hid8),
                         _ptr(amax))
     return hid8, float(amax[0])
+
+
+def adarms_layer_stack(x, layers, fin, dims, scales=None, eps=1e-6):
+    """Every step of the AdaRMS layer loop except attention, in the order of
+    [fp8_chain] `_make_run`, then the final tail.  Per layer l:
+      norm_project(slot 2l, "qkv"): producer (res += gate * delta, AdaRMS,
+        quantize) into the packed q/k/v GEMM; the prefix copy and the split +
+        RoPE + KV write;
+      attention stand-in: att2 = q_out viewed as [rows, hq * hd] (attention
+        itself is outside the path);
+      out_project: static quantize of att2, o GEMM -> dn;
+      norm_project(slot 2l + 1, "gu"): producer (delta = dn, gate = the qkv
+        norm's gate) into the packed gate/up GEMM;
+      down_project: GEGLU requant, down GEMM -> dn;
+      delta, gate = dn, the gu norm's gate.
+    Then ada_rms_tail(res, delta, gate, fin).
+
+    layers[l]: dict(qkv, o, gu, dn: pack_weights_fp8 results (qkv with the
+    q/k interleave, gu in concatenated [gate; up] order), styles [2, 3D]
+    (attention site, FFN site), prefix_k, prefix_v host caches).
+    dims: dict(B, M, D, hq, hkv, hd, P, T, H, theta).  scales: per layer
+    dict(a_qkv, a_o, a_gu, a_dn); None calibrates them on this batch, each
+    site's scale = amax / 448 of its quantizer input, in order.
+    Returns (out, records, scales)."""
+    B, M, D = dims["B"], dims["M"], dims["D"]
+    rows = B * M
+    table = rope_table(M, dims["hd"], dims["P"], dims.get("theta", 10000.0))
+    res = _c(x, np.uint16).copy()
+    delta = np.zeros((rows, D), np.uint16)
+    gate = np.zeros((1, D), np.uint16)
+    recs, used = [], []
+
+    def scale_of(site, l, amax):
+        if scales is not None:
+            return scales[l][site]
+        return max(amax / 448.0, 1e-8)
+
+    for l, ly in enumerate(layers):
+        sc = {}
+        st_attn, st_ffn = ly["styles"][0:1], ly["styles"][1:2]
+        a = scale_of("a_qkv", l, None if scales else
+                     ada_rms_norm_quant(res, delta, gate, st_attn, 1.0, eps)["amax"])
+        sc["a_qkv"] = a
+        pr = ada_rms_norm_quant(res, delta, gate, st_attn, a, eps)
+        qkv = fp8_gemm(pr["x8"], ly["qkv"]["w8"], a, ly["qkv"]["w_scale"])
+        kc = np.zeros((B, dims["T"], dims["hkv"], dims["hd"]), np.uint16)
+        vc = kc
+        if ly.get("prefix_k") is not None:
+            kc, vc = prefix_copy(ly["prefix_k"], ly["prefix_v"], dims["P"], kc, vc, True)
+        q, kc, vc = split_rope_kvcache(qkv, table, B, M, dims["hq"], dims["hkv"],
+                                       dims["hd"], dims["P"], kc, vc)
+        att2 = q.reshape(rows, dims["hq"] * dims["hd"])
+        a_o = scale_of("a_o", l, None if scales else quant_fp8_static(att2, 1.0)[1])
+        sc["a_o"] = a_o
+        o8, _ = quant_fp8_static(att2, a_o)
+        dn_o = fp8_gemm(o8, ly["o"]["w8"], a_o, ly["o"]["w_scale"])
+        a_gu = scale_of("a_gu", l, None if scales else
+                        ada_rms_norm_quant(pr["res"], dn_o, pr["gate_out"], st_ffn, 1.0,
+                                           eps)["amax"])
+        sc["a_gu"] = a_gu
+        pf = ada_rms_norm_quant(pr["res"], dn_o, pr["gate_out"], st_ffn, a_gu, eps)
+        gu = fp8_gemm(pf["x8"], ly["gu"]["w8"], a_gu, ly["gu"]["w_scale"])
+        a_dn = scale_of("a_dn", l, None if scales else geglu_quant(gu, 1.0)[1])
+        sc["a_dn"] = a_dn
+        hid8, _ = geglu_quant(gu, a_dn)
+        dn = fp8_gemm(hid8, ly["dn"]["w8"], a_dn, ly["dn"]["w_scale"])
+        recs.append({"x8": pr["x8"], "q": q, "k": kc, "v": vc, "o8": o8, "dn_o": dn_o,
+                     "x8_ffn": pf["x8"], "hid8": hid8, "dn": dn, "res": pf["res"],
+                     "g1": pr["gate_out"], "g2": pf["gate_out"]})
+        used.append(sc)
+        res, delta, gate = pf["res"], dn, pf["gate_out"]
+    out = ada_rms_tail(res, delta, gate, fin, eps)
+    return out, recs, used

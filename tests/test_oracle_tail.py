@@ -85,3 +85,35 @@ def test_tail_norm_sees_the_unrounded_sum():
     gate = _bf16([[1.0, 1.0]])
     out = oracle.bf16_to_f32(_tail(res, delta, gate, 0.0, -1.0))
     assert abs(out[0, 0] - 2.0 ** -10) < 1e-4 and abs(out[0, 1] + 2.0 ** -10) < 1e-4
+
+
+def test_layer_stack_wiring_with_silent_projections():
+    # with zero o and down weights the FFN half adds nothing: the residual
+    # leaving the layer is the one the q/k/v norm stored, and the tail sees
+    # a zero delta (checks the loop's order and which tensor feeds which)
+    rng = np.random.default_rng(8)
+    D, M, H = 64, 4, 128
+    dims = {"B": 1, "M": M, "D": D, "hq": 1, "hkv": 1, "hd": 64, "P": 0, "T": M, "H": H}
+    wq = [oracle.f32_to_bf16(rng.normal(0, 0.05, size=(64, D)).astype(np.float32))
+          for _ in range(3)]
+    zero_o = np.zeros((D, D), np.uint16)
+    mlp = [oracle.f32_to_bf16(rng.normal(0, 0.05, size=(H, D)).astype(np.float32))
+           for _ in range(2)]
+    layer = {"qkv": oracle.pack_weights_fp8(wq, layout=1, hd=64),
+             "o": oracle.pack_weights_fp8([zero_o]),
+             "gu": oracle.pack_weights_fp8(mlp),
+             "dn": oracle.pack_weights_fp8([np.zeros((D, H), np.uint16)]),
+             "styles": oracle.f32_to_bf16(rng.normal(0, 0.2, size=(2, 3 * D))
+                                          .astype(np.float32))}
+    x = oracle.f32_to_bf16(rng.normal(size=(M, D)).astype(np.float32))
+    fin = rng.normal(0, 0.1, size=(3, D)).astype(np.float32)
+    out, recs, scales = oracle.adarms_layer_stack(x, [layer], fin, dims)
+    r = recs[0]
+    assert not np.any(r["dn_o"]) and not np.any(r["dn"])
+    first = oracle.ada_rms_norm_quant(x, np.zeros((M, D), np.uint16),
+                                      np.zeros((1, D), np.uint16), layer["styles"][0:1],
+                                      scales[0]["a_qkv"])
+    assert np.array_equal(r["res"], first["res"])
+    assert np.array_equal(r["x8"], first["x8"])
+    want = oracle.ada_rms_tail(first["res"], np.zeros((M, D), np.uint16), r["g2"], fin, 1e-6)
+    assert np.array_equal(out, want)
