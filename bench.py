@@ -616,6 +616,154 @@ class MlpRunner:
             t.copy_(self.dev_out[k], non_blocking=True)
 
 
+class FullRunner:
+    """Whole AdaRMS layers except attention (fp8_transformer_block_b200.stack):
+    per layer the q/k/v chain layer, the output projection's static quantize
+    and GEMM on the attention stand-in, the FFN half; then the final tail."""
+
+    def __init__(self, w, torch, frt, rt, synth):
+        from fp8_transformer_block_b200 import stack
+        self.w, self.torch, self.frt, self.rt = w, torch, frt, rt
+        L, rows, D, H = w.layers, w.rows, w.D, w.H
+        self.L = L
+        lays = [synth.full_layer_inputs(w, l) for l in range(L)]
+        fin = synth.final_norm_rows(w)
+        cal = synth.adarms_inputs(rows, D, w.seed + synth.CAL_OFFSET)["res"]
+        self.st = stack.AdaRmsLayerStack(w, lays, fin, x=cal)
+        self.x_host = synth.adarms_inputs(rows, D, w.seed)["res"]
+        self.x0 = rt.bf16_dev(self.x_host)
+        self.st.res.copy_(self.x0)
+        self.pk_host = [(li["prefix_k"], li["prefix_v"]) for li in lays]
+        N = (w.hq + 2 * w.hkv) * w.hd
+        gb = N * D + rows * D + w.M * w.hd * 2 + rows * N * 2
+        gf = 2.0 * rows * N * D
+        self.kerns = [
+            Kern("prefix_copy", "hbm", 4.0 * w.B * w.P * w.hkv * w.hd * 2, per_step=L),
+            Kern("producer", "hbm", rows * D * 11 + 6 * D, per_step=2 * L),
+            Kern("gemm_rope_kv", "tensor" if gf / gb > 560 else "hbm", gb, gf, per_step=L),
+            Kern("quantize_o", "hbm", rows * D * 3, per_step=L),
+            Kern("gemm_o", "tensor" if rows > 560 else "hbm", D * D + rows * D * 3,
+                 2.0 * rows * D * D, per_step=L),
+            Kern("gemm_gateup_geglu", "tensor" if rows > 560 else "hbm",
+                 2 * H * D + rows * D + rows * H, 2.0 * rows * 2 * H * D, per_step=L),
+            Kern("gemm_down", "tensor" if rows > 560 else "hbm",
+                 D * H + rows * H + rows * D * 2, 2.0 * rows * D * H, per_step=L),
+            Kern("tail", "hbm", rows * D * 8 + 8 * D, per_step=1),
+        ]
+        self.tokens = rows
+        self.launches = 7 * L + 1
+
+    def footprint(self):
+        st, seen, total = self.st, set(), 0
+        ts = [v for v in vars(st).values() if isinstance(v, self.torch.Tensor)]
+        for v in vars(st).values():
+            if isinstance(v, list):
+                ts += [x for x in v if isinstance(x, self.torch.Tensor)]
+        for ly in st.lay:
+            for v in ly.values():
+                if isinstance(v, self.torch.Tensor):
+                    ts.append(v)
+                elif hasattr(v, "w8"):
+                    ts.append(v.w8)
+        for t in ts:
+            if t.data_ptr() not in seen:
+                seen.add(t.data_ptr())
+                total += t.numel() * t.element_size()
+        return total
+
+    def reset(self):
+        self.st.res.copy_(self.x0)
+
+    def step(self):
+        self.st.step()
+
+    def kernel_calls(self):
+        st, w, frt = self.st, self.w, self.frt
+        ly, sc = st.lay[0], st.sdev[0]
+        D, H, rows = w.D, w.H, st.rows
+
+        def prefix():
+            frt.frt_prefix_copy_kv(w.B, w.hkv, w.hd, w.P, w.T, w.P, ly["pk"], ly["pv"], 1,
+                                   ly["kc"], ly["vc"])
+
+        def producer():
+            frt.frt_ada_norm_quant_fp8(frt.FRT_NORM_ADARMS, rows, D, w.eps, st.res, st.dn_o,
+                                       st.g1, D, None, ly["st_ffn"], 0, None, None, 0, None,
+                                       0, 0, sc["a_gu"], st.x8f, st.g2[0], None)
+
+        def gemm_rope():
+            frt.frt_packed_fp8_gemm_rope_kvcache(
+                w.B, w.M, D, w.hq, w.hkv, w.hd, w.P, w.T, st.x8, ly["qkv"].w8, sc["a_qkv"],
+                ly["qkv"].w_scale, None, st.rope, st.q, ly["kc"], ly["vc"], st.ws, st.ws_bytes)
+
+        def quant():
+            frt.frt_quantize_fp8_static(rows, D, st.q, D, sc["a_o"], st.o8)
+
+        def gemm_o():
+            frt.frt_packed_fp8_gemm(rows, D, D, st.o8, ly["o"].w8, sc["a_o"], ly["o"].w_scale,
+                                    None, frt.FRT_EPI_BF16, st.dn_o, D, None, st.ws,
+                                    st.ws_bytes)
+
+        def gemm_gu():
+            frt.frt_packed_fp8_gemm(rows, 2 * H, D, st.x8f, ly["gu"].w8, sc["a_gu"],
+                                    ly["gu"].w_scale, None, frt.FRT_EPI_GEGLU_E4M3, st.hid8, H,
+                                    sc["a_dn"], st.ws, st.ws_bytes)
+
+        def gemm_dn():
+            frt.frt_packed_fp8_gemm(rows, D, H, st.hid8, ly["dn"].w8, sc["a_dn"],
+                                    ly["dn"].w_scale, None, frt.FRT_EPI_BF16, st.dn[0], D,
+                                    None, st.ws, st.ws_bytes)
+
+        def tail():
+            frt.frt_ada_rms_tail(rows, D, w.eps, st.res, st.dn[0], st.g2[0], D, st.fin, D,
+                                 st.out)
+        return list(zip(self.kerns, (prefix, producer, gemm_rope, quant, gemm_o, gemm_gu,
+                                     gemm_dn, tail)))
+
+    # ---------------------------------------------------------------- e2e --
+    def e2e_setup(self):
+        """The step's inputs (the rows entering the stack and every layer's
+        host prefix cache) back to back in one pinned buffer and one device
+        arena the stack reads directly (one host->device copy); the output
+        rows and each layer's new K/V rows come back with one copy each."""
+        torch, st, w = self.torch, self.st, self.w
+        ins = [("x", st.res, self.x_host)]
+        for l, ly in enumerate(st.lay):
+            ins.append((f"pk{l}", ly["pk"], self.pk_host[l][0]))
+            ins.append((f"pv{l}", ly["pv"], self.pk_host[l][1]))
+        offs, n = {}, 0
+        for name, t, _ in ins:
+            offs[name] = n
+            n += (t.numel() + 127) // 128 * 128
+        arena = torch.empty(n, dtype=torch.int16, device="cuda")
+        pin = torch.empty(n, dtype=torch.int16).pin_memory()
+        views = {}
+        for name, t, host in ins:
+            v = arena[offs[name]:offs[name] + t.numel()].view(t.dtype).view(t.shape)
+            v.copy_(t)
+            pin[offs[name]:offs[name] + t.numel()].copy_(
+                torch.from_numpy(np.ascontiguousarray(host).view(np.int16).reshape(-1)))
+            views[name] = v
+        st.res = views["x"]
+        for l, ly in enumerate(st.lay):
+            ly["pk"], ly["pv"] = views[f"pk{l}"], views[f"pv{l}"]
+        st._build()
+        self.arena, self.pin_arena, self.n_in = arena, pin, n
+        self.outs = [(st.out, torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory())]
+        for ly in st.lay:
+            for c in ("kc", "vc"):
+                src = ly[c][:, w.P:w.P + w.M]
+                self.outs.append((src, torch.empty(src.shape, dtype=src.dtype).pin_memory()))
+        self.h2d_bytes = 2 * n
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t, _ in self.outs)
+
+    def e2e_step(self):
+        self.arena.copy_(self.pin_arena, non_blocking=True)
+        self.step()
+        for src, dst in self.outs:
+            dst.copy_(src, non_blocking=True)
+
+
 def make_runner(name, torch, frt, rt, synth):
     base, _, m = name.partition(":")
     w = synth.WORKLOADS[base]
@@ -623,10 +771,17 @@ def make_runner(name, torch, frt, rt, synth):
         w = w.with_M(int(m))
     if w.kind == "mlp":
         return MlpRunner(w, torch, frt, rt, synth)
+    if w.kind == "full":
+        return FullRunner(w, torch, frt, rt, synth)
     return ChainRunner(w, torch, frt, rt, synth)
 
 
 def workload_text(w):
+    if w.kind == "full":
+        return (f"{w.name}: B={w.B} M={w.M} D={w.D} Hq={w.hq}x{w.hd} Hkv={w.hkv}x{w.hd} "
+                f"P={w.P} T={w.T} FFN {w.H}, {w.layers} whole layers except attention "
+                "(q/k/v chain, output projection on the attention stand-in q_out, "
+                "FFN half) + final tail")
     if w.kind == "mlp":
         return (f"{w.name}: M={w.M} D={w.D} gate/up {w.H} each (packed "
                 f"N={2 * w.H}) + GEGLU requant + down [{w.D},{w.H}]")
@@ -666,6 +821,30 @@ def oracle_sampler(name, synth, rows_cap=None):
             hid, _ = oracle.geglu_quant(gu, 0.05)
             oracle.fp8_gemm(hid, dn_p["w8"], 0.05, dn_p["w_scale"])
         return fn, len(sel), f"{len(sel)} of {w.M} rows, full MLP per row"
+
+    if w.kind == "full":
+        # rows stay independent through the whole loop (the attention
+        # stand-in is the row's own q): a leading block of rows, the stack
+        # at its own positions, static scales fixed
+        n = w.rows if rows_cap is None else max(1, min(w.rows, rows_cap))
+        wl = w.with_M(n)
+        lays = [synth.full_layer_inputs(w, l) for l in range(w.layers)]
+        ol = [{"qkv": oracle.pack_weights_fp8(li["w"], layout=1, hd=w.hd),
+               "o": oracle.pack_weights_fp8([li["o"]]),
+               "gu": oracle.pack_weights_fp8([li["mlp"]["gate"], li["mlp"]["up"]]),
+               "dn": oracle.pack_weights_fp8([li["mlp"]["down"]]),
+               "styles": li["styles"], "prefix_k": li["prefix_k"],
+               "prefix_v": li["prefix_v"]} for li in lays]
+        fin = synth.final_norm_rows(w)
+        x = synth.adarms_inputs(w.rows, w.D, w.seed)["res"][:n]
+        dims = {"B": 1, "M": n, "D": w.D, "hq": w.hq, "hkv": w.hkv, "hd": w.hd,
+                "P": w.P, "T": wl.T, "H": w.H, "theta": w.theta}
+        fixed = [{"a_qkv": 0.01, "a_o": 0.01, "a_gu": 0.01, "a_dn": 0.05}] * w.layers
+
+        def fn():
+            oracle.adarms_layer_stack(x, ol, fin, dims, scales=fixed, eps=w.eps)
+        return fn, n, (f"{n} of {w.rows} rows, {w.layers} whole layers except attention "
+                       "+ tail")
 
     L = w.layers
     rows = w.rows
@@ -801,6 +980,8 @@ L2_BYTES = 126 << 20
 
 def _footprint(runner, torch):
     """Device bytes a step of this runner reads or writes (its own tensors)."""
+    if hasattr(runner, "footprint"):
+        return runner.footprint()
     seen, total = set(), 0
     for v in vars(runner).values():
         ts = []
