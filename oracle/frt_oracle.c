@@ -540,6 +540,44 @@ void or_ada_rms_tail(int rows, int D, float eps, const uint16_t *res,
     free(h);
 }
 
+/* ------------------------------------------------------------------ */
+/* GELU + static requant between the DiT FFN's two GEMMs ([ptok_table] */
+/* PerTokenModChainBlock.forward: the fp8_gelu_mlp call on the FFN      */
+/* site's FP8 activation, with the ffn_hid static scale).               */
+/* ------------------------------------------------------------------ */
+/*
+ * u [M, H] bf16 (the up projection's bf16 output, bias included):
+ *   hid8[m, j] = q8(gelu_tanh(u[m, j]); out_scale)
+ * gelu_tanh as in or_geglu_quant (the kernel's GELU variant is not shown on
+ * the pages; the tanh form is the reading), fp32, tanhf from the C library.
+ */
+void or_gelu_quant(int M, int H, const uint16_t *u, long ldu, float out_scale,
+                   uint8_t *hid8, float *amax_out)
+{
+    const float k0 = 0.7978845608028654f;   /* sqrt(2/pi) */
+    const float k1 = 0.044715f;
+    float *row_amax = (float *)calloc((size_t)(M > 0 ? M : 1), sizeof(float));
+    #pragma omp parallel for schedule(static)
+    for (int m = 0; m < M; ++m) {
+        float mx = 0.0f;
+        for (int j = 0; j < H; ++j) {
+            float g = or_bf16_to_f32(u[(long)m * ldu + j]);
+            float g3 = (g * g) * g;
+            float inner = k0 * (g + k1 * g3);
+            float h = (0.5f * g) * (1.0f + tanhf(inner));
+            hid8[(long)m * H + j] = q8(h, out_scale);
+            if (fabsf(h) > mx) mx = fabsf(h);
+        }
+        row_amax[m] = mx;
+    }
+    if (amax_out) {
+        float mx = 0.0f;
+        for (int m = 0; m < M; ++m) if (row_amax[m] > mx) mx = row_amax[m];
+        *amax_out = mx;
+    }
+    free(row_amax);
+}
+
 /* OpenMP thread count the oracle runs with (1 without OpenMP). */
 int or_num_threads(void)
 {

@@ -26,6 +26,7 @@ __all__ = [
     "ada_rms_norm_quant", "ada_layer_norm_quant_table", "pack_weights_fp8",
     "fp8_gemm", "rope_table", "split_rope_kvcache", "prefix_copy",
     "geglu_quant", "quant_fp8_static", "ada_rms_tail", "adarms_layer_stack",
+    "gelu_quant",
 ]
 
 
@@ -71,6 +72,7 @@ def _L():
             "or_prefix_copy": (None, [i, i, i, i, i, i, p, p, i, p, p]),
             "or_geglu_quant": (None, [i, i, p, f, p, p]),
             "or_quant_fp8_static": (None, [i, i, p, l, f, p, p]),
+            "or_gelu_quant": (None, [i, i, p, l, f, p, p]),
             "or_ada_rms_tail": (None, [i, i, f, p, p, p, l, p, l, p]),
             "or_num_threads": (i, []),
         }
@@ -246,6 +248,17 @@ def prefix_copy(prefix_k, prefix_v, P, k_cache, v_cache, interleave=True):
                         _ptr(prefix_v), int(bool(interleave)), _ptr(k_cache),
                         _ptr(v_cache))
     return k_cache, v_cache
+
+
+def gelu_quant(u, out_scale):
+    """[ptok_table] fp8_gelu_mlp's middle step: hid8 = q8(gelu_tanh(u);
+    out_scale) for bf16 bits u [M, H]; returns (hid8, amax)."""
+    u = _c(u, np.uint16)
+    M, H = u.shape
+    hid8 = np.empty((M, H), np.uint8)
+    amax = np.zeros(1, np.float32)
+    _L().or_gelu_quant(M, H, _ptr(u), H, float(out_scale), _ptr(hid8), _ptr(amax))
+    return hid8, float(amax[0])
 
 
 def quant_fp8_static(x, scale):

@@ -117,3 +117,30 @@ def test_layer_stack_wiring_with_silent_projections():
     assert np.array_equal(r["x8"], first["x8"])
     want = oracle.ada_rms_tail(first["res"], np.zeros((M, D), np.uint16), r["g2"], fin, 1e-6)
     assert np.array_equal(out, want)
+
+
+def _gelu_vals(x, scale=1.0 / 32):
+    u = _bf16(np.asarray(x, np.float32).reshape(1, -1))
+    hid, amax = oracle.gelu_quant(u, scale)
+    return oracle.e4m3_to_f32(hid[0]) * np.float32(scale), amax
+
+
+def test_gelu_quant_fixed_points():
+    # gelu(0) = 0; gelu(x) -> x for large x and -> 0 for large -x; the
+    # odd-part identity gelu(x) - gelu(-x) = x (the tanh factor is odd)
+    v, _ = _gelu_vals([0.0, 6.0, -6.0, 10.0, -10.0])
+    assert v[0] == 0.0 and v[2] == 0.0 and v[4] == 0.0
+    assert abs(v[1] - 6.0) <= 6.0 / 8 and abs(v[3] - 10.0) <= 10.0 / 8  # one e4m3 step
+    xs = np.array([0.25, 0.5, 1.0, 1.5, 2.0, 3.0], np.float32)
+    u = _bf16(np.concatenate([xs, -xs]).reshape(1, -1))
+    hid, _ = oracle.gelu_quant(u, 1.0 / 256)
+    g = oracle.e4m3_to_f32(hid[0]).astype(np.float64) / 256
+    diff = g[:6] - g[6:]
+    assert np.all(np.abs(diff - xs) <= 0.07 * xs + 2e-3)   # within e4m3 rounding
+
+
+def test_gelu_quant_amax_is_the_largest_output():
+    u = _bf16(np.array([[-3.0, -0.5, 0.0, 0.7, 2.5]], np.float32))
+    _, amax = oracle.gelu_quant(u, 1.0)
+    # gelu is increasing for x > -0.75: the largest value is gelu(2.5) ~ 2.48
+    assert 2.45 < amax < 2.5
