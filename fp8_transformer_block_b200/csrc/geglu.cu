@@ -1,4 +1,5 @@
-// geglu.cu -- a5 (standalone form): merged GEGLU + static FP8 requant.
+// geglu.cu -- a5 (standalone form): merged GEGLU + static FP8 requant, and
+// the plain GELU + requant of the DiT FFN (fp8_ptok_table.py).
 //
 // flashrt-structures 0.2.0, impls/adarms_stack/fp8_chain.py `down_project`
 // (the merged gate/up output gu [S, 2H] becomes hid8 [S, H] in one kernel,
@@ -42,6 +43,37 @@ __global__ void geglu_kernel(int M, int H, const uint16_t* gu, long ld, const fl
   }
 }
 
+// GELU + static requant of a bf16 [M, H] tensor (the DiT FFN's
+// fp8_gelu_mlp middle step, unfused form; the GEMM's GELU epilogue gives the
+// same codes).
+__global__ void gelu_kernel(int M, int H, const uint16_t* u, long ld, const float* out_scale,
+                            uint8_t* hid8, float* amax) {
+  const int h8 = H / 8;
+  const long total = long(M) * h8;
+  pdl_trigger();
+  pdl_wait();
+  const float inv_os = __frcp_rn(__ldg(out_scale));
+  float mx = 0.0f;
+  for (long g = blockIdx.x * long(blockDim.x) + threadIdx.x; g < total;
+       g += long(gridDim.x) * blockDim.x) {
+    const long m = g / h8;
+    const int c = int(g % h8);
+    float uv[8], q[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(u + m * ld + 8 * c)), uv);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float h = gelu_tanh_mul(uv[j], 1.0f);
+      mx = fmaxf(mx, fabsf(h));
+      q[j] = __fmul_rn(h, inv_os);
+    }
+    *reinterpret_cast<uint2*>(hid8 + m * H + 8 * c) = pack8_e4m3(q);
+  }
+  if (amax) {
+    mx = warp_max(mx);
+    if ((threadIdx.x & 31) == 0) atomic_max_nonneg(amax, mx);
+  }
+}
+
 }  // namespace
 }  // namespace frt
 
@@ -60,5 +92,23 @@ extern "C" int frt_geglu_quant_fp8(int M, int H, const frt_bf16* gu, long ld_gu,
   const int grid = int(need < frt::num_sms() * 16L ? need : frt::num_sms() * 16L);
   return frt::launch_pdl("geglu_kernel", frt::geglu_kernel, dim3(grid), dim3(256), 0,
                          static_cast<cudaStream_t>(stream), M, H, gu, ld_gu, out_scale, hid8,
+                         amax_out);
+}
+
+extern "C" int frt_gelu_quant_fp8(int M, int H, const frt_bf16* u, long ld_u,
+                                  const float* out_scale, frt_e4m3* hid8, float* amax_out,
+                                  void* stream) {
+  using frt::aligned;
+  frt::clear_error();
+  FRT_REQUIRE(M >= 0 && H > 0 && H % 8 == 0, FRT_ESHAPE, "H must be a positive multiple of 8");
+  FRT_REQUIRE(ld_u >= H && ld_u % 8 == 0, FRT_ESHAPE, "ld_u must be >= H and a multiple of 8");
+  FRT_REQUIRE(u && out_scale && hid8, FRT_EINVAL, "u, out_scale and hid8 are required");
+  FRT_REQUIRE(aligned(u, 16) && aligned(hid8, 8), FRT_EALIGN, "u 16-byte, hid8 8-byte aligned");
+  if (M == 0) return FRT_OK;
+  const long total = long(M) * (H / 8);
+  const long need = (total + 255) / 256;
+  const int grid = int(need < frt::num_sms() * 16L ? need : frt::num_sms() * 16L);
+  return frt::launch_pdl("gelu_kernel", frt::gelu_kernel, dim3(grid), dim3(256), 0,
+                         static_cast<cudaStream_t>(stream), M, H, u, ld_u, out_scale, hid8,
                          amax_out);
 }

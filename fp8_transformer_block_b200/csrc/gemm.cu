@@ -43,7 +43,7 @@ constexpr int kMaxCluster = 8;      // portable thread-block cluster size
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per wait
 constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s to drain after an abort
 
-enum { EPI_BF16 = 0, EPI_GEGLU = 1, EPI_ROPE = 2 };
+enum { EPI_BF16 = 0, EPI_GEGLU = 1, EPI_ROPE = 2, EPI_GELU = 3 };
 
 #ifndef FRT_MIN_KB_PER_SPLIT
 #define FRT_MIN_KB_PER_SPLIT 16  // K-blocks (of 128) per split at least
@@ -249,6 +249,28 @@ __device__ __forceinline__ void epi_geglu_chunk(const GemmParams& p, const float
   }
 }
 
+// GELU + static requant of one row's 32 columns (the DiT FFN's fp8_gelu_mlp
+// middle step): h = gelu_tanh(bf16(acc * alpha + bias)), out = e4m3(h / s)
+// computed as h * fp32(1 / s), as the GEGLU epilogue does.
+__device__ __forceinline__ void epi_gelu_chunk(const GemmParams& p, const float (&v)[32], int m,
+                                               int n0, float alpha) {
+  if (m >= p.M) return;
+  const float inv_os = __frcp_rn(__ldg(p.out_scale));
+  float q[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    q[j] = __fmul_rn(gelu_tanh_mul(scale_bias_bf16(v[j], alpha, p.bias, n0 + j), 1.0f), inv_os);
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + long(m) * p.ldo + n0);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    float a[8], b[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { a[j] = q[16 * k + j]; b[j] = q[16 * k + 8 + j]; }
+    const uint2 lo = pack8_e4m3(a), hi = pack8_e4m3(b);
+    dst[k] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+  }
+}
+
 // TMEM lane holding accumulator row r of an MMA with M = BMT rows: all 128
 // lanes for M = 128; for M = 64 the rows fill the first 16 lanes of each
 // 32-lane quarter (rows 16q .. 16q+15 in lanes 32q .. 32q+15).  The epilogue
@@ -320,7 +342,8 @@ __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int t
       float v[32];
       load(c, v);
       if (c == c_last) done();
-      epi_rows_chunk(p, v, m, tb * BN + 32 * c, alpha);
+      if (p.epi == EPI_GELU) epi_gelu_chunk(p, v, m, tb * BN + 32 * c, alpha);
+      else epi_rows_chunk(p, v, m, tb * BN + 32 * c, alpha);
     }
     return;
   }
@@ -990,7 +1013,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           float v[32];
           load(c, v);
           if (c == BN / 32 - 1) release();
-          epi_rows_chunk(p, v, m, tn * BN + 32 * c, alpha);
+          if (p.epi == EPI_GELU) epi_gelu_chunk(p, v, m, tn * BN + 32 * c, alpha);
+          else epi_rows_chunk(p, v, m, tn * BN + 32 * c, alpha);
         }
       }
     }
@@ -1056,7 +1080,12 @@ Plan make_plan(int M, int N, int K, int epi) {
   Plan pl{};
   pl.k_blocks = (K + BK - 1) / BK;
   pl.bmt = 128;
-  if (epi != EPI_GEGLU && M <= 128) { pl.swap = true; pl.bmt = 64; pl.bn = M <= 64 ? 64 : 128; }
+  // the e4m3 epilogues write token rows: the normal orientation serves them
+  if (epi != EPI_GEGLU && epi != EPI_GELU && M <= 128) {
+    pl.swap = true;
+    pl.bmt = 64;
+    pl.bn = M <= 64 ? 64 : 128;
+  }
   else {
     pl.swap = false;
     pl.bn = (N % 256 == 0) ? 256 : 128;
@@ -1301,6 +1330,13 @@ int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void
   return launch_swap<64, 128, 7>(pl, ta, tb, p, s);
 }
 
+// The C ABI's epilogue code -> the kernels' epilogue.
+int epi_of(int epilogue) {
+  return epilogue == FRT_EPI_GEGLU_E4M3   ? EPI_GEGLU
+         : epilogue == FRT_EPI_GELU_E4M3 ? EPI_GELU
+                                         : EPI_BF16;
+}
+
 int validate_common(int M, int N, int K, const void* x8, const void* w8, const float* act_scale,
                     const float* w_scale) {
   FRT_REQUIRE(M >= 0, FRT_ESHAPE, "M must be >= 0, got %d", M);
@@ -1317,7 +1353,7 @@ int validate_common(int M, int N, int K, const void* x8, const void* w8, const f
 
 extern "C" size_t frt_gemm_workspace_size(int M, int N, int K, int epilogue) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
-  return frt::make_plan(M, N, K, epilogue == FRT_EPI_GEGLU_E4M3 ? frt::EPI_GEGLU : frt::EPI_BF16)
+  return frt::make_plan(M, N, K, frt::epi_of(epilogue))
       .ws_bytes;
 }
 
@@ -1330,13 +1366,18 @@ extern "C" int frt_packed_fp8_gemm(int M, int N, int K, const frt_e4m3* x8, cons
   frt::clear_error();
   int rc = frt::validate_common(M, N, K, x8, w8, act_scale, w_scale);
   if (rc) return rc;
-  FRT_REQUIRE(epilogue == FRT_EPI_BF16 || epilogue == FRT_EPI_GEGLU_E4M3, FRT_EINVAL,
-              "unknown epilogue %d", epilogue);
+  FRT_REQUIRE(epilogue == FRT_EPI_BF16 || epilogue == FRT_EPI_GEGLU_E4M3 ||
+                  epilogue == FRT_EPI_GELU_E4M3,
+              FRT_EINVAL, "unknown epilogue %d", epilogue);
   FRT_REQUIRE(out, FRT_EINVAL, "out is required");
   FRT_REQUIRE(!bias || aligned(bias, 16), FRT_EALIGN, "bias must be 16-byte aligned");
   FRT_REQUIRE(aligned(out, 16), FRT_EALIGN, "out must be 16-byte aligned");
   if (epilogue == FRT_EPI_BF16) {
     FRT_REQUIRE(ldo >= N && ldo % 8 == 0, FRT_EALIGN, "ldo must be >= N and a multiple of 8");
+  } else if (epilogue == FRT_EPI_GELU_E4M3) {
+    FRT_REQUIRE(out_scale, FRT_EINVAL, "the GELU epilogue needs out_scale");
+    FRT_REQUIRE(ldo >= N && ldo % 16 == 0, FRT_EALIGN,
+                "ldo must be >= N and a multiple of 16 bytes");
   } else {
     FRT_REQUIRE(N % 256 == 0, FRT_ESHAPE, "the GEGLU epilogue needs N %% 256 == 0, got %d", N);
     FRT_REQUIRE(out_scale, FRT_EINVAL, "the GEGLU epilogue needs out_scale");
@@ -1344,7 +1385,7 @@ extern "C" int frt_packed_fp8_gemm(int M, int N, int K, const frt_e4m3* x8, cons
                 "ldo must be >= N/2 and a multiple of 16 bytes");
   }
   if (M == 0) return FRT_OK;
-  const int epi = epilogue == FRT_EPI_BF16 ? frt::EPI_BF16 : frt::EPI_GEGLU;
+  const int epi = frt::epi_of(epilogue);
   frt::Plan pl = frt::make_plan(M, N, K, epi);
   frt::GemmParams p{};
   p.M = M; p.N = N; p.K = K;
@@ -1450,10 +1491,7 @@ extern "C" int frt_packed_fp8_gemm_noalloc(int M, int N, int K, const frt_e4m3* 
       if (rc) return rc;
       // the split counters at the head of the workspace must start at zero;
       // a completed call leaves them zero, an interrupted one might not
-      const size_t counters = (size_t(frt::make_plan(M, N, K, epilogue == FRT_EPI_GEGLU_E4M3
-                                                                   ? frt::EPI_GEGLU
-                                                                   : frt::EPI_BF16)
-                                            .counters_bytes));
+      const size_t counters = size_t(frt::make_plan(M, N, K, frt::epi_of(epilogue)).counters_bytes);
       if (counters > 0 &&
           cudaMemsetAsync(ws, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return frt::fail(FRT_ECUDA, "clearing the static scratch counters");

@@ -24,7 +24,7 @@ FRT_OK, FRT_EINVAL, FRT_ESHAPE, FRT_EALIGN, FRT_ERANGE, FRT_ECUDA, \
     FRT_ETIMEOUT = 0, -1, -2, -3, -4, -5, -6
 FRT_NORM_ADARMS, FRT_NORM_LAYERNORM_TABLE = 0, 1
 FRT_PACK_CONCAT, FRT_PACK_QK_INTERLEAVE, FRT_PACK_GATE_UP_BLOCKS = 0, 1, 2
-FRT_EPI_BF16, FRT_EPI_GEGLU_E4M3 = 0, 1
+FRT_EPI_BF16, FRT_EPI_GEGLU_E4M3, FRT_EPI_GELU_E4M3 = 0, 1, 2
 FRT_CHAIN_FUSED_ROPE, FRT_CHAIN_UNFUSED = 0, 1
 
 STATUS_NAMES = {0: "FRT_OK", -1: "FRT_EINVAL", -2: "FRT_ESHAPE",
@@ -112,6 +112,7 @@ _SIGS = {
     "frt_ffn_layer": (_i, [C.POINTER(frt_ffn_desc), _p]),
     "frt_selftest_bounded_wait": (_i, [_i, _p]),
     "frt_quantize_fp8_static": (_i, [_i, _i, _p, _l, _p, _p, _p, _p]),
+    "frt_gelu_quant_fp8": (_i, [_i, _i, _p, _l, _p, _p, _p, _p]),
     "frt_ada_rms_tail": (_i, [_i, _i, _f, _p, _p, _p, _l, _p, _l, _p, _p]),
     "frt_peak_fp8_mma": (_i, [_i, _i, _p]),
     "frt_peak_copy": (_i, [_p, _p, C.c_size_t, _p]),
@@ -270,6 +271,12 @@ def frt_ffn_workspace_size(desc: frt_ffn_desc) -> int:
 
 def frt_ffn_layer(desc: frt_ffn_desc, stream=None):
     return _check(_lib.frt_ffn_layer(C.byref(desc), _stream(stream)), "frt_ffn_layer")
+
+
+def frt_gelu_quant_fp8(M, H, u, ld_u, out_scale, hid8, amax_out=None, stream=None) -> None:
+    """GELU + static e4m3 requant (the DiT FFN's middle step, unfused)."""
+    _check(_lib.frt_gelu_quant_fp8(M, H, ptr(u), ld_u, ptr(out_scale), ptr(hid8),
+                                   ptr(amax_out), _stream(stream)), "frt_gelu_quant_fp8")
 
 
 def frt_quantize_fp8_static(rows, D, x, ldx, act_scale, x8_out, amax_out=None,

@@ -142,7 +142,7 @@ int frt_pack_weights_fp8(int n_siblings, const frt_bf16* const* w,
 /* ----------------------------------------------------------------------- */
 /* a2 (+ a5)  Packed FP8 GEMM on tcgen05 tensor cores.                      */
 /* ----------------------------------------------------------------------- */
-enum { FRT_EPI_BF16 = 0, FRT_EPI_GEGLU_E4M3 = 1 };
+enum { FRT_EPI_BF16 = 0, FRT_EPI_GEGLU_E4M3 = 1, FRT_EPI_GELU_E4M3 = 2 };
 
 /*
  * Bytes of workspace frt_packed_fp8_gemm / _rope_kvcache need for this
@@ -163,6 +163,10 @@ size_t frt_gemm_workspace_size(int M, int N, int K, int epilogue);
  *   g, u = bf16(acc * alpha + bias) of matching gate/up columns,
  *                  out[m, j] = e4m3(gelu_tanh(g) * u * (1 / out_scale))
  *                  out: [M, ldo] e4m3, ldo >= N / 2; N % 256 == 0.
+ *   FRT_EPI_GELU_E4M3 (fp8_ptok_table.py, the DiT FFN's fp8_gelu_mlp
+ *   middle step): with y = bf16(acc * alpha + bias),
+ *                  out[m, n] = e4m3(gelu_tanh(y) * (1 / out_scale))
+ *                  out: [M, ldo] e4m3, ldo >= N.
  * x8: [M, K] e4m3; w8: [N, K] e4m3; bias: [N] bf16 or NULL.
  * Requires K % 16 == 0, N % 32 == 0, 16-byte aligned x8/w8/out/bias, ldo %
  * 16 == 0 (bytes of a row).  M == 0 is a no-op.  workspace: see
@@ -276,6 +280,18 @@ int frt_prefix_copy_kv(int B, int hkv, int hd, int P, int T, int T_src,
 int frt_geglu_quant_fp8(int M, int H, const frt_bf16* gu, long ld_gu,
                         const float* out_scale, frt_e4m3* hid8,
                         float* amax_out, void* stream);
+
+/*
+ * frt_gelu_quant_fp8 (fp8_ptok_table.py, the DiT FFN's fp8_gelu_mlp middle
+ * step, unfused form): hid8[m, j] = e4m3(gelu_tanh(u[m, j]) / out_scale),
+ * computed as a multiply by the fp32 reciprocal like the GEGLU kernel.
+ * u: bf16 [M, ld_u] (16-byte aligned, ld_u >= H, multiple of 8); hid8:
+ * [M, H] e4m3 (8-byte aligned); amax_out (nullable, caller-zeroed) gets
+ * max |gelu_tanh(u)|.  H % 8 == 0.
+ */
+int frt_gelu_quant_fp8(int M, int H, const frt_bf16* u, long ld_u,
+                       const float* out_scale, frt_e4m3* hid8, float* amax_out,
+                       void* stream);
 
 /* ----------------------------------------------------------------------- */
 /* The attention-input chain layer: producer -> packed GEMM (+ RoPE + KV).  */

@@ -407,3 +407,45 @@ def test_peak_probes_run_and_are_plausible(rt):
     frt.frt_peak_copy(src, dst, n)
     _sync(torch)
     assert torch.equal(src, dst)
+
+
+# -------------------------------------------------------- GELU epilogue --
+@pytest.mark.parametrize("M,D,H", [(64, 512, 1024), (300, 512, 1024), (1100, 512, 2048),
+                                   (200, 4096, 256)])
+def test_gelu_fused_epilogue(rt, M, D, H):
+    """The GEMM's GELU + requant epilogue (the DiT FFN's up projection)
+    against the unfused GEMM -> GELU kernel, and that against the oracle."""
+    frt, runtime, torch = rt
+    rng = np.random.default_rng(M + H)
+    w = normal_bf16(rng, (H, D), 0.02)
+    b = normal_bf16(rng, (H,), 0.01)
+    x8 = runtime.u8_dev(_x8_codes(M, D, 91))
+    sc = runtime.scale_dev(0.02)
+    pk = runtime.pack([w], [b])
+    u = runtime.empty_bf16(M, H)
+    wsb = frt.frt_gemm_workspace_size(M, H, D)
+    frt.frt_packed_fp8_gemm(M, H, D, x8, pk.w8, sc, pk.w_scale, pk.bias, frt.FRT_EPI_BF16,
+                            u, H, None, runtime.workspace(wsb), wsb)
+    am = torch.zeros(1, dtype=torch.float32, device="cuda")
+    h1 = runtime.empty_u8(M, H)
+    frt.frt_gelu_quant_fp8(M, H, u, H, runtime.scale_dev(1.0), h1, am)
+    torch.cuda.synchronize()
+    s_h = float(am.item()) / 448.0
+    out_scale = runtime.scale_dev(s_h)
+    frt.frt_gelu_quant_fp8(M, H, u, H, out_scale, h1)
+    h2 = torch.full((M, H), 0x7F, dtype=torch.uint8, device="cuda")
+    wsb2 = frt.frt_gemm_workspace_size(M, H, D, frt.FRT_EPI_GELU_E4M3)
+    frt.frt_packed_fp8_gemm(M, H, D, x8, pk.w8, sc, pk.w_scale, pk.bias,
+                            frt.FRT_EPI_GELU_E4M3, h2, H, out_scale,
+                            runtime.workspace(wsb2), wsb2)
+    _sync(torch)
+    assert frt.frt_device_status(True) == frt.FRT_OK
+    u_host = runtime.bf16_host(u)
+    ref_u = oracle.fp8_gemm(runtime.u8_host(x8), runtime.u8_host(pk.w8), 0.02,
+                            float(pk.w_scale.item()), runtime.bf16_host(pk.bias))
+    assert_rms(u_host, ref_u, what="up projection")
+    assert_codes(runtime.u8_host(h2), runtime.u8_host(h1), match=0.9999,
+                 what="fused vs unfused GELU")
+    ref, amax = oracle.gelu_quant(u_host, s_h)
+    assert_codes(runtime.u8_host(h1), ref, what="unfused GELU vs oracle")
+    assert abs(float(am.item()) - amax) <= 1e-6 * amax
