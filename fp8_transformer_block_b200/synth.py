@@ -63,7 +63,8 @@ class Workload:
     "mlp" (AdaRMS producer + gate/up GEMM + GEGLU + down GEMM),
     "stack" (``layers`` AdaRMS chain layers, residual carried) or "full"
     (``layers`` whole AdaRMS layers except attention: the q/k/v chain, the
-    output projection, the FFN half; then the final tail)."""
+    output projection, the FFN half; then the final tail) or "ditffn" (the
+    video-DiT block's FFN half)."""
     name: str
     cid: int
     kind: str
@@ -124,6 +125,11 @@ WORKLOADS = {
     "adarms_layer18": Workload("adarms_layer18", 5, "full", B=1, M=50, D=512,
                                hq=8, hkv=1, hd=64, P=816, T=866, H=2048,
                                layers=18, cal_rows=64),
+    # not one of the five configurations: the video-DiT block's FFN half
+    # (producer at the FFN site, chunks 3/4; up projection + GELU requant;
+    # down projection; both with bias), FFN hidden 4 * D (a reading)
+    "video_dit_ffn": Workload("video_dit_ffn", 6, "ditffn", B=2, M=4096, D=3072,
+                              H=12288, bias=True, cal_rows=256),
 }
 
 
@@ -209,3 +215,11 @@ def final_norm_rows(w: Workload):
     rng = np.random.Generator(np.random.PCG64(w.seed + 31337))
     return (rng.standard_normal(size=(3, w.D), dtype=np.float32)
             * np.float32(0.02 * np.sqrt(w.D)))
+
+
+def dit_ffn_weights(D: int, H: int, seed: int):
+    """Up [H, D] and down [D, H] projections N(0, 0.02) with bf16 biases
+    N(0, 0.01) (the DiT block's FFN, biased like its q/k/v)."""
+    rng = np.random.Generator(np.random.PCG64(seed + 7919))
+    return {"up": normal_bf16(rng, (H, D), 0.02), "up_b": normal_bf16(rng, (H,), 0.01),
+            "dn": normal_bf16(rng, (D, H), 0.02), "dn_b": normal_bf16(rng, (D,), 0.01)}

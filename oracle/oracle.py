@@ -26,7 +26,7 @@ __all__ = [
     "ada_rms_norm_quant", "ada_layer_norm_quant_table", "pack_weights_fp8",
     "fp8_gemm", "rope_table", "split_rope_kvcache", "prefix_copy",
     "geglu_quant", "quant_fp8_static", "ada_rms_tail", "adarms_layer_stack",
-    "gelu_quant",
+    "gelu_quant", "dit_ffn",
 ]
 
 
@@ -370,3 +370,19 @@ def adarms_layer_stack(x, layers, fin, dims, scales=None, eps=1e-6):
         res, delta, gate = pf["res"], dn, pf["gate_out"]
     out = ada_rms_tail(res, delta, gate, fin, eps)
     return out, recs, used
+
+
+def dit_ffn(x, temb, table, up, dn, a_in, a_hid=None, eps=1e-6, shift_idx=3, scale_idx=4):
+    """The video-DiT block's FFN half ([ptok_table] PerTokenModChainBlock.
+    forward): the per-token-table producer at the FFN site (chunks 3, 4)
+    into the fp8_gelu_mlp pair: up GEMM (+ bias), GELU + static requant,
+    down GEMM (+ bias).  up / dn: pack_weights_fp8 results with bias.
+    a_hid None calibrates it on this batch (amax of the GELU output / 448).
+    Returns dict(x8, u, hid8, ff, a_hid)."""
+    pr = ada_layer_norm_quant_table(x, temb, table, shift_idx, scale_idx, a_in, eps=eps)
+    u = fp8_gemm(pr["x8"], up["w8"], a_in, up["w_scale"], up["bias"])
+    if a_hid is None:
+        a_hid = max(gelu_quant(u, 1.0)[1] / 448.0, 1e-8)
+    hid8, _ = gelu_quant(u, a_hid)
+    ff = fp8_gemm(hid8, dn["w8"], a_hid, dn["w_scale"], dn["bias"])
+    return {"x8": pr["x8"], "u": u, "hid8": hid8, "ff": ff, "a_hid": a_hid, "amax_in": pr["amax"]}

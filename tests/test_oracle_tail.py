@@ -144,3 +144,18 @@ def test_gelu_quant_amax_is_the_largest_output():
     _, amax = oracle.gelu_quant(u, 1.0)
     # gelu is increasing for x > -0.75: the largest value is gelu(2.5) ~ 2.48
     assert 2.45 < amax < 2.5
+
+
+def test_dit_ffn_wiring_zero_up_projection_gives_the_down_bias():
+    # u = 0 -> gelu(0) = 0 -> hid8 = 0 -> ff = bf16(0 * alpha + bias_dn)
+    from fp8_transformer_block_b200 import synth
+    rng = np.random.default_rng(12)
+    D, H, rows = 64, 128, 5
+    inp = synth.dit_inputs(rows, D, 3)
+    up = oracle.pack_weights_fp8([np.zeros((H, D), np.uint16)], [np.zeros(H, np.uint16)])
+    bias_dn = _bf16(rng.normal(0, 0.3, size=D).astype(np.float32))
+    dn = oracle.pack_weights_fp8([_bf16(rng.normal(0, 0.02, size=(D, H)).astype(np.float32))],
+                                 [bias_dn])
+    r = oracle.dit_ffn(inp["x"], inp["temb"], inp["table"], up, dn, 0.02, a_hid=0.01)
+    assert not np.any(r["hid8"])
+    assert np.array_equal(r["ff"], np.broadcast_to(bias_dn, (rows, D)))
