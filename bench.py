@@ -764,6 +764,115 @@ class FullRunner:
             dst.copy_(src, non_blocking=True)
 
 
+class DitFfnRunner:
+    """The video-DiT block's FFN half: the per-token-table producer at the
+    FFN site (chunks 3/4) -> up projection with the GELU + static requant
+    epilogue -> down projection, both with bias."""
+
+    def __init__(self, w, torch, frt, rt, synth):
+        self.w, self.torch, self.frt, self.rt = w, torch, frt, rt
+        rows, D, H = w.rows, w.D, w.H
+        self.rows = rows
+        fw = synth.dit_ffn_weights(D, H, w.seed)
+        self.up = rt.pack([fw["up"]], [fw["up_b"]])
+        self.dn = rt.pack([fw["dn"]], [fw["dn_b"]])
+        inp = synth.dit_inputs(rows, D, w.seed)
+        self.host_in = {"x": inp["x"], "temb": inp["temb"]}
+        self.x = rt.bf16_dev(inp["x"])
+        self.temb = rt.bf16_dev(inp["temb"])
+        self.table = rt.f32_dev(inp["table"])
+        self.x8 = rt.empty_u8(rows, D)
+        self.hid8 = rt.empty_u8(rows, H)
+        self.ff = rt.empty_bf16(rows, D)
+        self.ws1 = frt.frt_gemm_workspace_size(rows, H, D, frt.FRT_EPI_GELU_E4M3)
+        self.ws2 = frt.frt_gemm_workspace_size(rows, D, H)
+        self.wsp1, self.wsp2 = rt.workspace(self.ws1), rt.workspace(self.ws2)
+        self.calibrate(synth, fw)
+        self.kerns = [
+            Kern("producer", "hbm", rows * D * (2 + 2 * 2 + 1)),
+            Kern("gemm_up_gelu", "tensor", H * D + rows * D + rows * H + 2 * H,
+                 2.0 * rows * H * D),
+            Kern("gemm_down", "tensor", D * H + rows * H + rows * D * 2 + 2 * D,
+                 2.0 * rows * D * H),
+        ]
+        self.tokens = rows
+        self.launches = 3
+
+    def calibrate(self, synth, fw):
+        """a_in from the producer's amax and a_hid from the unfused GELU
+        kernel's amax, on a seeded calibration batch (seed + 500)."""
+        torch, frt, rt, w = self.torch, self.frt, self.rt, self.w
+        C, D, H = w.cal_rows, w.D, w.H
+        cal = synth.dit_inputs(C, D, w.seed + synth.CAL_OFFSET)
+        am = torch.zeros(1, dtype=torch.float32, device="cuda")
+        x8 = rt.empty_u8(C, D)
+        frt.frt_ada_norm_quant_fp8(frt.FRT_NORM_LAYERNORM_TABLE, C, D, w.eps, None, None, None,
+                                   0, None, None, 0, rt.bf16_dev(cal["x"]),
+                                   rt.bf16_dev(cal["temb"]), 6, rt.f32_dev(cal["table"]), 3, 4,
+                                   rt.scale_dev(1.0), x8, None, am)
+        torch.cuda.synchronize()
+        self.a_in = max(float(am.item()) / 448.0, 1e-8)
+        s_in = rt.scale_dev(self.a_in)
+        frt.frt_ada_norm_quant_fp8(frt.FRT_NORM_LAYERNORM_TABLE, C, D, w.eps, None, None, None,
+                                   0, None, None, 0, rt.bf16_dev(cal["x"]),
+                                   rt.bf16_dev(cal["temb"]), 6, rt.f32_dev(cal["table"]), 3, 4,
+                                   s_in, x8, None, None)
+        u = rt.empty_bf16(C, H)
+        wsb = frt.frt_gemm_workspace_size(C, H, D)
+        frt.frt_packed_fp8_gemm(C, H, D, x8, self.up.w8, s_in, self.up.w_scale, self.up.bias,
+                                frt.FRT_EPI_BF16, u, H, None, rt.workspace(wsb), wsb)
+        am.zero_()
+        frt.frt_gelu_quant_fp8(C, H, u, H, rt.scale_dev(1.0), rt.empty_u8(C, H), am)
+        torch.cuda.synchronize()
+        self.a_hid = max(float(am.item()) / 448.0, 1e-8)
+        self.s_in, self.s_hid = s_in, rt.scale_dev(self.a_hid)
+
+    def _producer(self):
+        w, frt = self.w, self.frt
+        frt.frt_ada_norm_quant_fp8(frt.FRT_NORM_LAYERNORM_TABLE, self.rows, w.D, w.eps, None,
+                                   None, None, 0, None, None, 0, self.x, self.temb, 6,
+                                   self.table, 3, 4, self.s_in, self.x8, None, None)
+
+    def _up(self):
+        w, frt = self.w, self.frt
+        frt.frt_packed_fp8_gemm(self.rows, w.H, w.D, self.x8, self.up.w8, self.s_in,
+                                self.up.w_scale, self.up.bias, frt.FRT_EPI_GELU_E4M3,
+                                self.hid8, w.H, self.s_hid, self.wsp1, self.ws1)
+
+    def _down(self):
+        w, frt = self.w, self.frt
+        frt.frt_packed_fp8_gemm(self.rows, w.D, w.H, self.hid8, self.dn.w8, self.s_hid,
+                                self.dn.w_scale, self.dn.bias, frt.FRT_EPI_BF16, self.ff, w.D,
+                                None, self.wsp2, self.ws2)
+
+    def reset(self):
+        pass
+
+    def step(self):
+        self._producer()
+        self._up()
+        self._down()
+
+    def kernel_calls(self):
+        return list(zip(self.kerns, (self._producer, self._up, self._down)))
+
+    def e2e_setup(self):
+        torch = self.torch
+        self.pin_in = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).pin_memory()
+                       for k, v in self.host_in.items()}
+        self.dev_in = {"x": self.x, "temb": self.temb}
+        self.pin_out = torch.empty(self.ff.shape, dtype=self.ff.dtype).pin_memory()
+        self.h2d_bytes = sum(t.numel() * 2 for t in self.pin_in.values())
+        self.d2h_bytes = self.ff.numel() * 2
+
+    def e2e_step(self):
+        for k, t in self.pin_in.items():
+            d = self.dev_in[k]
+            d.view(self.torch.int16).copy_(t.view(d.shape), non_blocking=True)
+        self.step()
+        self.pin_out.copy_(self.ff, non_blocking=True)
+
+
 def make_runner(name, torch, frt, rt, synth):
     base, _, m = name.partition(":")
     w = synth.WORKLOADS[base]
@@ -773,10 +882,15 @@ def make_runner(name, torch, frt, rt, synth):
         return MlpRunner(w, torch, frt, rt, synth)
     if w.kind == "full":
         return FullRunner(w, torch, frt, rt, synth)
+    if w.kind == "ditffn":
+        return DitFfnRunner(w, torch, frt, rt, synth)
     return ChainRunner(w, torch, frt, rt, synth)
 
 
 def workload_text(w):
+    if w.kind == "ditffn":
+        return (f"{w.name}: B={w.B} M={w.M} D={w.D} FFN {w.H}: table producer at the FFN "
+                "site (chunks 3/4) + up GEMM with GELU requant + down GEMM, both biased")
     if w.kind == "full":
         return (f"{w.name}: B={w.B} M={w.M} D={w.D} Hq={w.hq}x{w.hd} Hkv={w.hkv}x{w.hd} "
                 f"P={w.P} T={w.T} FFN {w.H}, {w.layers} whole layers except attention "
@@ -821,6 +935,19 @@ def oracle_sampler(name, synth, rows_cap=None):
             hid, _ = oracle.geglu_quant(gu, 0.05)
             oracle.fp8_gemm(hid, dn_p["w8"], 0.05, dn_p["w_scale"])
         return fn, len(sel), f"{len(sel)} of {w.M} rows, full MLP per row"
+
+    if w.kind == "ditffn":
+        n = rows_cap or 32
+        sel = np.sort(rng.choice(w.rows, size=min(n, w.rows), replace=False))
+        fw = synth.dit_ffn_weights(w.D, w.H, w.seed)
+        up = oracle.pack_weights_fp8([fw["up"]], [fw["up_b"]])
+        dnp = oracle.pack_weights_fp8([fw["dn"]], [fw["dn_b"]])
+        inp = synth.dit_inputs(w.rows, w.D, w.seed)
+        x, temb, table = inp["x"][sel], inp["temb"][sel], inp["table"]
+
+        def fn():
+            oracle.dit_ffn(x, temb, table, up, dnp, 0.02, a_hid=0.01, eps=w.eps)
+        return fn, len(sel), f"{len(sel)} of {w.rows} rows, the FFN half per row"
 
     if w.kind == "full":
         # rows stay independent through the whole loop (the attention
@@ -946,6 +1073,8 @@ def run_reference(args):
         base, _, m = args.config.partition(":")
         w = synth.WORKLOADS[base]
         full = w.M if w.kind == "mlp" else w.rows
+        if w.kind == "ditffn":
+            full = 32
         cap = max(1, int(full * 150.0 / (args.steps * t1) * 0.5))
         fn, tokens, text = oracle_sampler(args.config, synth, rows_cap=cap)
     for _ in range(args.warmup):

@@ -411,3 +411,58 @@ def test_ffn_layer_entry(rt):
     orf = bf16_value(out_ref).astype(np.float64)
     assert np.linalg.norm(og - orf) / np.linalg.norm(orf) <= 2e-2
     assert frt.frt_device_status(True) == frt.FRT_OK
+
+
+def test_dit_ffn_sampled(rt):
+    """The video-DiT block's FFN half at full size on the GPU (8192 rows,
+    D 3072, FFN 12288: table producer at chunks 3/4, up projection with the
+    GELU requant epilogue, biased down projection), checked on seeded sampled
+    rows that the oracle computes from the same inputs (rows are
+    independent through the FFN)."""
+    frt, runtime, torch = rt
+    w = synth.WORKLOADS["video_dit_ffn"]
+    rows, D, H = w.rows, w.D, w.H
+    fw = synth.dit_ffn_weights(D, H, w.seed)
+    up = oracle.pack_weights_fp8([fw["up"]], [fw["up_b"]])
+    dnp = oracle.pack_weights_fp8([fw["dn"]], [fw["dn_b"]])
+    cal = synth.dit_inputs(64, D, w.seed + synth.CAL_OFFSET)
+    c0 = oracle.dit_ffn(cal["x"], cal["temb"], cal["table"], up, dnp, 1.0)
+    a_in = c0["amax_in"] / 448.0
+    a_hid = oracle.dit_ffn(cal["x"], cal["temb"], cal["table"], up, dnp, a_in)["a_hid"]
+    inp = synth.dit_inputs(rows, D, w.seed)
+    sel = np.sort(np.random.default_rng(5).choice(rows, size=48, replace=False))
+    ref = oracle.dit_ffn(inp["x"][sel], inp["temb"][sel], inp["table"], up, dnp, a_in,
+                         a_hid=a_hid)
+
+    upd = runtime.pack([fw["up"]], [fw["up_b"]])
+    dnd = runtime.pack([fw["dn"]], [fw["dn_b"]])
+    s_in, s_hid = runtime.scale_dev(a_in), runtime.scale_dev(a_hid)
+    x8 = runtime.empty_u8(rows, D)
+    hid8 = runtime.empty_u8(rows, H)
+    ff = runtime.empty_bf16(rows, D)
+    frt.frt_ada_norm_quant_fp8(frt.FRT_NORM_LAYERNORM_TABLE, rows, D, w.eps, None, None, None,
+                               0, None, None, 0, runtime.bf16_dev(inp["x"]),
+                               runtime.bf16_dev(inp["temb"]), 6, runtime.f32_dev(inp["table"]),
+                               3, 4, s_in, x8, None, None)
+    ws1 = frt.frt_gemm_workspace_size(rows, H, D, frt.FRT_EPI_GELU_E4M3)
+    frt.frt_packed_fp8_gemm(rows, H, D, x8, upd.w8, s_in, upd.w_scale, upd.bias,
+                            frt.FRT_EPI_GELU_E4M3, hid8, H, s_hid, runtime.workspace(ws1), ws1)
+    ws2 = frt.frt_gemm_workspace_size(rows, D, H)
+    frt.frt_packed_fp8_gemm(rows, D, H, hid8, dnd.w8, s_hid, dnd.w_scale, dnd.bias,
+                            frt.FRT_EPI_BF16, ff, D, None, runtime.workspace(ws2), ws2)
+    torch.cuda.synchronize()
+    assert frt.frt_device_status(True) == frt.FRT_OK
+    g_x8 = runtime.u8_host(x8)[sel]
+    g_hid = runtime.u8_host(hid8)[sel]
+    g_ff = runtime.bf16_host(ff)[sel]
+    assert_codes(g_x8, ref["x8"], what="FFN-site x8")
+    d8 = e4m3_step_distance(g_hid, ref["hid8"])
+    dq_g = oracle.e4m3_to_f32(g_hid).astype(np.float64)
+    dq_r = oracle.e4m3_to_f32(ref["hid8"]).astype(np.float64)
+    rel_h = np.linalg.norm(dq_g - dq_r) / np.linalg.norm(dq_r)
+    og = bf16_value(g_ff).astype(np.float64)
+    orf = bf16_value(ref["ff"]).astype(np.float64)
+    rel_o = np.linalg.norm(og - orf) / np.linalg.norm(orf)
+    print(f"DiT FFN: hid8 identical {(d8 == 0).mean():.6f} rel-L2 {rel_h:.3e}; ff rel-L2 {rel_o:.3e}")
+    assert (d8 == 0).mean() >= 0.99 and rel_h <= 2e-2
+    assert rel_o <= 2e-2
