@@ -153,3 +153,31 @@ def test_ffn_desc_layout_matches_header(frt):
     body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
     names = re.findall(r"\**\s*([A-Za-z_][A-Za-z0-9_]*)\s*(?=[,;])", body)
     assert names == [f for f, _ in frt.frt_ffn_desc._fields_]
+
+
+def test_output_side_validation(frt):
+    q = frt.raw_call
+    # static quantize: D % 8, ldx < D, misaligned input
+    assert q("frt_quantize_fp8_static", 4, 12, A16, 12, A16, A16, None, None) == frt.FRT_ESHAPE
+    assert q("frt_quantize_fp8_static", 4, 64, A16, 32, A16, A16, None, None) == frt.FRT_EALIGN
+    assert q("frt_quantize_fp8_static", 4, 64, A16 + 8, 64, A16, A16, None, None) == \
+        frt.FRT_EALIGN
+    assert q("frt_quantize_fp8_static", 0, 64, A16, 64, A16, A16, None, None) == frt.FRT_OK
+    # final tail: D beyond 8192, a gate stride below D, a missing fin
+    assert q("frt_ada_rms_tail", 4, 8200, C.c_float(1e-6), A16, A16, A16, 0, A16, 8200, A16,
+             None) == frt.FRT_ESHAPE
+    assert q("frt_ada_rms_tail", 4, 64, C.c_float(1e-6), A16, A16, A16, 32, A16, 64, A16,
+             None) == frt.FRT_EALIGN
+    assert q("frt_ada_rms_tail", 4, 64, C.c_float(1e-6), A16, A16, A16, 0, None, 64, A16,
+             None) == frt.FRT_EINVAL
+    # GELU requant: H % 8
+    assert q("frt_gelu_quant_fp8", 4, 12, A16, 16, A16, A16, None, None) == frt.FRT_ESHAPE
+    # GEMM with the GELU epilogue needs out_scale
+    assert q("frt_packed_fp8_gemm", 4, 256, 512, A16, A16, A16, A16, None,
+             frt.FRT_EPI_GELU_E4M3, A16, 256, None, None, 0, None) == frt.FRT_EINVAL
+    assert q("frt_packed_fp8_gemm", 4, 256, 512, A16, A16, A16, A16, None, 9, A16, 256,
+             A16, None, 0, None) == frt.FRT_EINVAL
+    # FFN half: no descriptor; the peak probe: no CTAs
+    assert q("frt_ffn_layer", None, None) == frt.FRT_EINVAL
+    assert q("frt_peak_fp8_mma", 0, 10, None) == frt.FRT_EINVAL
+    assert q("frt_peak_copy", A16 + 4, A16, 64, None) == frt.FRT_EALIGN
