@@ -1093,26 +1093,38 @@ Plan make_plan(int M, int N, int K, int epi) {
     // (a GEGLU tile keeps its gate and up halves together: always 256 wide)
     const long t256 = ((M + 127L) / 128) * ((N + 255L) / 256);
     if (epi != EPI_GEGLU && pl.bn == 256 && t256 < num_sms()) pl.bn = 128;
-    // CTA pairs (256-row tiles, half the B tile per SM) when they keep at
-    // least as many SMs busy as single-CTA tiles would
-    const int sms = num_sms();
+    // CTA pairs (256-row tiles, half the B tile per SM): the tile width and
+    // the schedule (pairs or single CTAs) with the lowest estimated cost,
+    // waves x bytes a CTA moves per K-block (16 KB of x8 plus its weight
+    // rows), which is what bounds both the L2-fed main loop and, for short
+    // K, the number of rounds of prologue and epilogue
+    const int sms = num_sms(), npairs = sms / 2;
     const long tiles1 = ((M + 127L) / 128) * ((N + pl.bn - 1L) / pl.bn);
-    const long ctas1 = tiles1 < sms ? tiles1 : sms;
+    const long cost1 = ((tiles1 + sms - 1) / sms) * (16384L + pl.bn * 128L);
     const long mt2 = (M + 255L) / 256;
-    int bn2 = 0;
-    if (N % 256 == 0 && (epi == EPI_GEGLU || 2 * mt2 * (N / 256) >= ctas1)) bn2 = 256;
-    else if (epi != EPI_GEGLU && N % 128 == 0) bn2 = 128;
-    if (M >= 256 && bn2) {
-      const long units2 = mt2 * (N / bn2);
-      const long pairs = units2 < sms / 2 ? units2 : sms / 2;
-      if (2 * pairs >= ctas1 && units2 >= 16) {
+    if (M >= 256) {
+      static const int kPairBn[] = {256, 192, 160, 128};
+      int best = 0;
+      long best_cost = cost1;
+      for (int bn2 : kPairBn) {
+        if (N % bn2 != 0 || (epi == EPI_GEGLU && bn2 != 256)) continue;
+        const long units2 = mt2 * (N / bn2);
+        if (units2 < 16) continue;
+        const long cost2 = ((units2 + npairs - 1) / npairs) * (16384L + bn2 * 64L);
+        if (cost2 < best_cost || (epi == EPI_GEGLU && !best)) {
+          best = bn2;
+          best_cost = cost2;
+        }
+      }
+      if (best) {
+        const long units2 = mt2 * (N / best);
         pl.pair = true;
-        pl.bn = bn2;
+        pl.bn = best;
         pl.a_tiles = int(mt2);
-        pl.b_tiles = int(N / bn2);
+        pl.b_tiles = int(N / best);
         pl.splits = 1;
         pl.units = int(units2);
-        pl.grid = int(2 * pairs);
+        pl.grid = int(2 * (units2 < npairs ? units2 : npairs));
         return pl;
       }
     }
@@ -1315,6 +1327,8 @@ int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void
     if ((rc = make_map(&ta, x8, p.M, p.K, 128))) return rc;
     if ((rc = make_map(&tb, w8, p.N, p.K, pl.bn / 2))) return rc;
     if (pl.bn == 256) return launch_pair<256, 6>(pl, ta, tb, p, s);
+    if (pl.bn == 192) return launch_pair<192, 7>(pl, ta, tb, p, s);
+    if (pl.bn == 160) return launch_pair<160, 8>(pl, ta, tb, p, s);
     return launch_pair<128, 8>(pl, ta, tb, p, s);
   }
   if (!pl.swap) {

@@ -192,6 +192,9 @@ GEMM_CASES = [
                                    # holds rows past M only; K tail
     (1100, 4096, 1024, True),      # BN = 256, ragged last 256-row tile
     (2048, 4096, 512, False),      # several tiles per pair, K < ring depth
+    (1024, 640, 512, False),       # 160-wide pair tiles (one wave where 128 needs two)
+    (1100, 640, 1024, True),       # 160-wide, ragged 256-row tile
+    (2048, 1536, 512, True),       # 192-wide pair tiles
 ]
 
 
