@@ -57,9 +57,9 @@ KERNEL_SOURCES = {
     "prefix_copy": ("rope.cu", "frt_prefix.cuh"),
 }
 NCU_TRAFFIC = {
-    ("vla_action_expert", "gemm_rope_kv"): (5_426_176, "892268e76741ebb5"),
-    ("video_dit", "gemm_rope_kv"): (154_795_264, "892268e76741ebb5"),
-    ("gateup_mlp", "gemm_gateup_geglu"): (73_113_856, "892268e76741ebb5"),
+    ("vla_action_expert", "gemm_rope_kv"): (5_426_432, "dba3502f8d1a22ca"),
+    ("video_dit", "gemm_rope_kv"): (154_199_296, "dba3502f8d1a22ca"),
+    ("gateup_mlp", "gemm_gateup_geglu"): (72_549_376, "dba3502f8d1a22ca"),
 }
 
 
