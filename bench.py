@@ -74,6 +74,21 @@ def _src_hash(kernel_name):
     return h.hexdigest()[:16]
 
 
+def max_over_ranks(ms, torch, dist, world, device):
+    """The slowest rank's time: every rank's device-timed milliseconds,
+    all-reduced with MAX (the identity on one rank)."""
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, steps, max_ms, world):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time
+    (replicas: each rank runs its own copy of the workload)."""
+    return world * tokens_per_rank * steps / (max_ms / 1e3)
+
+
 def own_peaks(torch, frt):
     """The library's own probes (frt_peak_fp8_mma, frt_peak_copy): best of
     three timed launches each, CUDA events on the current stream."""
@@ -1225,13 +1240,9 @@ def run_gpu(args):
     wall = time.perf_counter() - t_wall
     clk = clocks.stop()
     assert frt.frt_device_status(True) == frt.FRT_OK
-    total_ms = e0.elapsed_time(e1)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_total_ms = float(t.item())
+    max_total_ms = max_over_ranks(e0.elapsed_time(e1), torch, dist, world, dev)
     ms_per_step = max_total_ms / K
-    value = world * first.tokens * K / (max_total_ms / 1e3)
+    value = job_throughput(first.tokens, K, max_total_ms, world)
 
     # ---- each kernel alone, back to back over the same R copies
     kinds, kern_ms = [], []
@@ -1284,11 +1295,8 @@ def run_gpu(args):
         first.e2e_step()
         e_ev[i][1].record()
     torch.cuda.synchronize()
-    e_ms = sum(a.elapsed_time(b) for a, b in e_ev)
-    te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * first.tokens * KE / (float(te.item()) / 1e3)
+    e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), torch, dist, world, dev)
+    e2e_value = job_throughput(first.tokens, KE, e_ms, world)
 
     # ---- roofline of the dominant kernel (largest share of a step)
     hbm, bf16_burst, bf16_sust, src = _peaks()
