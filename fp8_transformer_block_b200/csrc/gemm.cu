@@ -1072,6 +1072,9 @@ struct Plan {
   size_t counters_bytes, ws_bytes;
 };
 
+#ifndef FRT_MAX_CLUSTER_SPLITS  // more ranks shorten the main loop but lengthen the gather
+#define FRT_MAX_CLUSTER_SPLITS 4
+#endif
 #ifndef FRT_MIN_KB_PER_CLUSTER_SPLIT
 #define FRT_MIN_KB_PER_CLUSTER_SPLIT 2  // K-blocks per split of a cluster tile
 #endif
@@ -1143,7 +1146,7 @@ Plan make_plan(int M, int N, int K, int epi) {
       s_max = sms / tiles;
       const int by_k = pl.k_blocks / FRT_MIN_KB_PER_CLUSTER_SPLIT;
       if (s_max > by_k) s_max = by_k;
-      if (s_max > kMaxCluster) s_max = kMaxCluster;
+      if (s_max > FRT_MAX_CLUSTER_SPLITS) s_max = FRT_MAX_CLUSTER_SPLITS;
       if (s_max < 1) s_max = 1;
     }
     pl.cluster = s_max > 1;

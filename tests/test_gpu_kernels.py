@@ -183,9 +183,10 @@ GEMM_CASES = [
     (256, 9216, 3072, True),       # video-DiT projection width
     (1200, 4096, 1024, False),     # 256-wide tiles, persistent
     (64, 2048, 16384, False),      # long K: K split in a 4-CTA cluster
-    (100, 1024, 4096, True),       # 128-token tiles: 5-CTA clusters, ragged
-    (32, 1024, 4096, True),        # 8-CTA clusters
-    (50, 1056, 2048, True),        # 8-CTA clusters, ragged last weight tile
+    (100, 1024, 4096, True),       # 128-token tiles: 4-CTA clusters, ragged
+    (32, 1024, 4096, True),        # clusters at the split cap (4)
+    (50, 1056, 2048, True),        # 4-CTA clusters, ragged last weight tile
+    (16, 512, 1024, False),        # 2-CTA clusters, 8 weight tiles
     (200, 256, 16384, True),       # 128-row tiles, K split via workspace
     # CTA pairs (256-row tiles over two SMs)
     (300, 4096, 528, True),        # BN = 128; the odd CTA of the last pair
