@@ -262,12 +262,6 @@ __device__ __forceinline__ uint32_t map_cluster(uint32_t smem_addr, uint32_t ran
   return r;
 }
 
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
-  return v;
-}
 
 // ------------------------------------------------- CTA-pair (2-SM) forms ----
 // A pair of CTAs in one cluster runs one M=256 MMA: each CTA holds half of
