@@ -57,9 +57,9 @@ KERNEL_SOURCES = {
     "prefix_copy": ("rope.cu", "frt_prefix.cuh"),
 }
 NCU_TRAFFIC = {
-    ("vla_action_expert", "gemm_rope_kv"): (5_426_432, "ba0d7c2f10e7e88d"),
-    ("video_dit", "gemm_rope_kv"): (154_199_296, "ba0d7c2f10e7e88d"),
-    ("gateup_mlp", "gemm_gateup_geglu"): (72_549_376, "ba0d7c2f10e7e88d"),
+    ("vla_action_expert", "gemm_rope_kv"): (5_426_432, "6d41c1fed564231c"),
+    ("video_dit", "gemm_rope_kv"): (154_199_296, "6d41c1fed564231c"),
+    ("gateup_mlp", "gemm_gateup_geglu"): (72_549_376, "6d41c1fed564231c"),
 }
 
 

@@ -1029,6 +1029,256 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   }
 }
 
+// --------------------------------------------- CTA-pair kernel, K in halves --
+//
+// One tile per cluster of 4 CTAs: two CTA pairs (cluster ranks 0-1 and 2-3)
+// run the same 256 x BN tile over the two halves of K, each pair as in
+// gemm_pair_kernel (cta_group::2 MMAs issued by its even CTA).  When its MMAs
+// are done, each CTA of the second pair stages its fp32 accumulator rows in
+// its own (now idle) operand ring and bulk-copies them into the ring of the
+// CTA holding the same rows in the first pair (rank - 2), which adds them to
+// its own accumulator chunk by chunk and runs the tile's epilogue.  For
+// shapes whose tiles leave half the SMs idle over a long K (the MLP's down
+// projection): twice the SMs pull operands, and the partial sums stay on chip.
+//   full[s]   (pair's even CTA) 2 arrivals, both CTAs' TMA bytes
+//   empty[s]  (each CTA) the pair's MMA commit, multicast to the pair
+//   tfull     (each CTA) the accumulator is complete
+//   go        (second pair) the receiving CTA's ring is free
+//   red_full  (first pair) the partial rows have landed (transaction bytes)
+//   done      (second pair) the receiver has them: the ring may be released
+// Every wait is bounded; a final cluster barrier keeps all four CTAs alive
+// until the cluster is done.
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_pair_split_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+  constexpr int A_BYTES = 128 * BK;
+  constexpr int B_BYTES = (BN / 2) * BK;
+  constexpr int RS = BN + 4;                       // staged row stride (floats)
+  constexpr uint32_t PART = uint32_t(128 * RS * 4);  // one CTA's staged rows
+  static_assert(PART <= uint32_t(STAGES * (A_BYTES + B_BYTES)), "the ring holds the partial");
+  constexpr uint32_t TMEM_COLS = tmem_cols_for(BN);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* drain = tfull + 1;
+  uint64_t* go = drain + 1;
+  uint64_t* red_full = drain + 2;
+  uint64_t* done = drain + 3;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* epi_ok = abort_flag + 2;  // [4]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int half = int(rank >> 1);          // which half of K this pair runs
+  const bool lead = (rank & 1u) == 0;       // the pair's MMA issuer
+  const uint32_t lead_rank = rank & ~1u;
+  const uint16_t pair_mask = uint16_t(0x3u << (2 * half));
+  const int tile = int(blockIdx.x >> 2);
+  const bool has_tile = tile < p.units;
+  const int tm = tile % p.a_tiles, tn = tile / p.a_tiles;
+  const int kb0 = half * p.k_blocks / 2, kb1 = (half + 1) * p.k_blocks / 2;
+  pdl_trigger();
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 2);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(drain, 1);
+    mbar_init(go, 1);
+    mbar_init(red_full, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    if (half == 0) mbar_arrive_expect_tx(red_full, PART);
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // every CTA's barriers exist before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint32_t full_lead = map_cluster(smem_u32(full), lead_rank);
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0 && has_tile) {
+      const int nk = kb1 - kb0;
+      const int n_pre = nk < STAGES ? nk : STAGES;
+      for (int i = 0; i < n_pre; ++i) {  // weights first, before the dependency wait
+        mbar_arrive_expect_tx_cluster(full_lead + 8u * i, A_BYTES + B_BYTES);
+        tma_load_2d_pair(sB + i * B_BYTES, &tmB, full_lead + 8u * i, (kb0 + i) * BK,
+                         tn * BN + int(rank & 1u) * (BN / 2));
+      }
+      pdl_wait();
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; i < nk; ++i) {
+        const int kb = kb0 + i;
+        if (i >= n_pre) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitNs, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx_cluster(full_lead + 8u * stage, A_BYTES + B_BYTES);
+          tma_load_2d_pair(sB + stage * B_BYTES, &tmB, full_lead + 8u * stage, kb * BK,
+                           tn * BN + int(rank & 1u) * (BN / 2));
+        }
+        tma_load_2d_pair(sA + stage * A_BYTES, &tmA, full_lead + 8u * stage, kb * BK,
+                         tm * 256 + int(rank & 1u) * 128);
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) {
+        record_timeout(p.status);
+        *abort_flag = 1;
+        if (lead) {
+          int st = stage;
+          uint32_t ph = phase;
+          for (int i = 0; i < issued && i < STAGES; ++i) {
+            if (--st < 0) { st = STAGES - 1; ph ^= 1u; }
+            mbar_wait_bounded(&full[st], ph, kDrainNs, nullptr);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // -------------------------------------------- MMA issuer (even CTA) --
+    if (lane == 0 && lead && has_tile) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(256, BN);
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; i < kb1 - kb0; ++i) {
+        if (!mbar_wait_bounded(&full[stage], phase, kWaitNs, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t ad = sdesc_k_sw128(a_base + stage * A_BYTES);
+        const uint64_t bd = sdesc_k_sw128(b_base + stage * B_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 32; ++k)
+          umma_pair_e4m3(tmem_base, ad + 2 * k, bd + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
+        umma_pair_commit(&empty[stage], pair_mask);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (ok) {
+        umma_pair_commit(tfull, pair_mask);
+      } else {
+        record_timeout(p.status);
+        *abort_flag = 1;
+        umma_pair_commit(drain, uint16_t(1u << rank));
+        mbar_wait_bounded(drain, 0, kDrainNs, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (has_tile) {
+    // ----------------------------------------------------------- epilogue --
+    pdl_wait();
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
+    const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(tfull, 0, kWaitNs, abort_flag));
+    if (lane == 0) epi_ok[q] = got ? 1 : 0;
+    named_bar_sync(1, 128);
+    const bool all_ok = epi_ok[0] && epi_ok[1] && epi_ok[2] && epi_ok[3];
+    tc_fence_after();
+    float* part = reinterpret_cast<float*>(smem);  // the idle ring: staged rows
+    if (!all_ok) {
+      if (threadIdx.x == 64) record_timeout(p.status);
+    } else if (half == 1) {
+      // hand this CTA's accumulator rows to the CTA with the same rows in
+      // the first pair, then wait until it has them
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem_base + 32 * c + (uint32_t(32 * q) << 16), v);
+        float4* d4 = reinterpret_cast<float4*>(part + row * RS + 32 * c);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 64) {
+        if (mbar_wait_bounded_cluster(go, 0, kWaitNs)) {
+          bulk_copy_to_peer(map_cluster(smem_u32(smem), rank - 2u), part, PART,
+                            map_cluster(smem_u32(red_full), rank - 2u));
+          if (!mbar_wait_bounded_cluster(done, 0, kWaitNs)) record_timeout(p.status);
+        } else {
+          record_timeout(p.status);
+        }
+      }
+      __syncwarp();
+    } else {
+      // this CTA's MMAs are done: its ring may receive the other half's rows
+      if (threadIdx.x == 64) mbar_arrive_release_cluster(map_cluster(smem_u32(go), rank + 2u));
+      const bool in = mbar_wait_bounded_cluster(red_full, 0, kWaitNs);
+      if (threadIdx.x == 64) {
+        if (in) mbar_arrive_release_cluster(map_cluster(smem_u32(done), rank + 2u));
+        else record_timeout(p.status);
+      }
+      if (in) {
+        const int m = tm * 256 + int(rank & 1u) * 128 + row;
+        const float* pr = part + row * RS;
+        auto load = [&](int c, float (&v)[32]) {
+          tmem_ld32(tmem_base + 32 * c + (uint32_t(32 * q) << 16), v);
+          const float4* s4 = reinterpret_cast<const float4*>(pr + 32 * c);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float4 f = s4[k];
+            v[4 * k] = __fadd_rn(v[4 * k], f.x);
+            v[4 * k + 1] = __fadd_rn(v[4 * k + 1], f.y);
+            v[4 * k + 2] = __fadd_rn(v[4 * k + 2], f.z);
+            v[4 * k + 3] = __fadd_rn(v[4 * k + 3], f.w);
+          }
+        };
+        if (p.epi == EPI_GEGLU) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float g[32], uu[32];
+            load(c, g);
+            load(c + 4, uu);
+            epi_geglu_chunk(p, g, uu, m, tn * BN + 32 * c, tn * BN + 128 + 32 * c,
+                            tn * 128 + 32 * c, alpha);
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            load(c, v);
+            if (p.epi == EPI_GELU) epi_gelu_chunk(p, v, m, tn * BN + 32 * c, alpha);
+            else epi_rows_chunk(p, v, m, tn * BN + 32 * c, alpha);
+          }
+        }
+      }
+    }
+  }
+
+  cluster_sync_all();  // the cluster is done with every CTA's memory
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // -------------------------------------------------------------------- host --
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -1067,7 +1317,7 @@ int make_map(CUtensorMap* m, const void* ptr, long rows, int K, int box_rows) {
 }
 
 struct Plan {
-  bool swap, cluster, pair;
+  bool swap, cluster, pair, split2;
   int bmt, bn, a_tiles, b_tiles, k_blocks, splits, units, grid;
   size_t counters_bytes, ws_bytes;
 };
@@ -1103,31 +1353,46 @@ Plan make_plan(int M, int N, int K, int epi) {
     // K, the number of rounds of prologue and epilogue
     const int sms = num_sms(), npairs = sms / 2;
     const long tiles1 = ((M + 127L) / 128) * ((N + pl.bn - 1L) / pl.bn);
-    const long cost1 = ((tiles1 + sms - 1) / sms) * (16384L + pl.bn * 128L);
+    const long kb = pl.k_blocks;
+    const long cost1 = ((tiles1 + sms - 1) / sms) * (16384L + pl.bn * 128L) * kb;
     const long mt2 = (M + 255L) / 256;
     if (M >= 256) {
       static const int kPairBn[] = {256, 192, 160, 128};
       int best = 0;
+      bool best_split = false;
       long best_cost = cost1;
       for (int bn2 : kPairBn) {
         if (N % bn2 != 0 || (epi == EPI_GEGLU && bn2 != 256)) continue;
         const long units2 = mt2 * (N / bn2);
         if (units2 < 16) continue;
-        const long cost2 = ((units2 + npairs - 1) / npairs) * (16384L + bn2 * 64L);
+        const long cost2 = ((units2 + npairs - 1) / npairs) * (16384L + bn2 * 64L) * kb;
         if (cost2 < best_cost || (epi == EPI_GEGLU && !best)) {
           best = bn2;
           best_cost = cost2;
+          best_split = false;
+        }
+        // K in halves over two pairs per tile (one tile per cluster of 4,
+        // one wave), for tiles that leave half the SMs idle over a long K;
+        // the on-chip hand-over of the partial costs about 8 K-blocks
+        if ((bn2 == 256 || bn2 == 128) && kb >= 32 && units2 * 4 <= sms) {
+          const long cost3 = (16384L + bn2 * 64L) * (kb / 2 + 8);
+          if (cost3 < best_cost) {
+            best = bn2;
+            best_cost = cost3;
+            best_split = true;
+          }
         }
       }
       if (best) {
         const long units2 = mt2 * (N / best);
         pl.pair = true;
+        pl.split2 = best_split;
         pl.bn = best;
         pl.a_tiles = int(mt2);
         pl.b_tiles = int(N / best);
         pl.splits = 1;
         pl.units = int(units2);
-        pl.grid = int(2 * (units2 < npairs ? units2 : npairs));
+        pl.grid = best_split ? int(4 * units2) : int(2 * (units2 < npairs ? units2 : npairs));
         return pl;
       }
     }
@@ -1309,6 +1574,41 @@ int launch_pair(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, co
   return FRT_OK;
 }
 
+template <int BN, int STAGES>
+int launch_pair_split(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb,
+                      const GemmParams& p, cudaStream_t s) {
+  constexpr int smem = STAGES * (128 * BK + (BN / 2) * BK) + 1024 + 256;
+  static_assert(smem <= 232448, "shared memory budget");
+  auto kern = gemm_pair_split_kernel<BN, STAGES>;
+  if (first_use(reinterpret_cast<const void*>(kern))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return fail(FRT_ECUDA, "cudaFuncSetAttribute(max dynamic smem %d)", smem);
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 4;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FRT_ECUDA, "gemm_pair_split_kernel: %s", cudaGetErrorString(e));
+  }
+  return FRT_OK;
+}
+
 int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void* workspace,
              size_t workspace_bytes, cudaStream_t s) {
   if (pl.ws_bytes > 0) {
@@ -1329,6 +1629,10 @@ int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void
   if (pl.pair) {  // each CTA loads 128 rows of x8 and BN/2 rows of w8
     if ((rc = make_map(&ta, x8, p.M, p.K, 128))) return rc;
     if ((rc = make_map(&tb, w8, p.N, p.K, pl.bn / 2))) return rc;
+    if (pl.split2) {
+      if (pl.bn == 256) return launch_pair_split<256, 6>(pl, ta, tb, p, s);
+      return launch_pair_split<128, 8>(pl, ta, tb, p, s);
+    }
     if (pl.bn == 256) return launch_pair<256, 6>(pl, ta, tb, p, s);
     if (pl.bn == 192) return launch_pair<192, 7>(pl, ta, tb, p, s);
     if (pl.bn == 160) return launch_pair<160, 8>(pl, ta, tb, p, s);

@@ -196,6 +196,9 @@ GEMM_CASES = [
     (1024, 640, 512, False),       # 160-wide pair tiles (one wave where 128 needs two)
     (1100, 640, 1024, True),       # 160-wide, ragged 256-row tile
     (2048, 1536, 512, True),       # 192-wide pair tiles
+    (1024, 1024, 4096, True),      # K in halves over two 128-wide pairs (clusters of 4)
+    (1024, 2048, 4096, False),     # K in halves over two 256-wide pairs
+    (1100, 1024, 4096, True),      # K in halves, ragged 256-row tile
 ]
 
 
