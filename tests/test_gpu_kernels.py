@@ -74,6 +74,8 @@ def _gpu_adarms(rt, inp, act_scale, eps=1e-6, weight=None, amax=False):
     (5, 16384, False, False),     # widest D
     (3, 8, False, False),         # narrowest D
     (1024, 2048, True, True),     # gate/up MLP producer site
+    (4096, 512, False, True),     # many narrow rows: register groups, not the staged ring
+    (700, 512, False, False),     # narrow rows, staged ring
 ])
 def test_producer_adarms_parity(rt, rows, D, outliers, per_row):
     inp = synth.adarms_inputs(rows, D, 4242 + D, outliers=outliers)
@@ -96,6 +98,7 @@ def test_producer_adarms_parity(rt, rows, D, outliers, per_row):
 @pytest.mark.parametrize("rows,D,chunks,sidx,cidx", [
     (256, 3072, 6, 0, 1),         # video-DiT attention site
     (33, 1000, 6, 3, 4),          # ragged, FFN-site chunks
+    (4096, 1000, 6, 3, 4),        # many narrow rows (register groups)
     (2, 16384, 6, 0, 1),
 ])
 def test_producer_layernorm_parity(rt, rows, D, chunks, sidx, cidx):
