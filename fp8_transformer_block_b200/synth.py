@@ -18,6 +18,10 @@ order listed, rounded to bf16 by round-to-nearest-even on the bit pattern):
 * Per-token-table LayerNorm inputs: ``x`` N(0,1), ``temb`` N(0,1),
   ``table`` fp32 N(0, 0.1).
 * Prefix K/V of the host cache N(0,1).
+* Modulation projection (every norm's (scale, shift, gate) from one
+  conditioning row): ``cond`` N(0,1) kept as fp32 values on the bf16 grid,
+  the stacked dense weights [(2L+1)*3D, D] N(0, 0.02) bf16, their fp32
+  bias N(0, 0.01) on the bf16 grid.
 * The calibration batch of a workload uses seed + 500.
 """
 
@@ -61,6 +65,8 @@ class Workload:
     """One of the five shapes.  ``kind`` is "adarms" (AdaRMS producer +
     q/k/v chain), "dit" (per-token-table LayerNorm + biased q/k/v),
     "mlp" (AdaRMS producer + gate/up GEMM + GEGLU + down GEMM),
+    "style" (the modulation projection of ``M`` conditioning rows into the
+    (scale, shift, gate) rows of all 2 * ``layers`` + 1 norms),
     "stack" (``layers`` AdaRMS chain layers, residual carried) or "full"
     (``layers`` whole AdaRMS layers except attention: the q/k/v chain, the
     output projection, the FFN half; then the final tail) or "ditffn" (the
@@ -97,6 +103,8 @@ class Workload:
     def N(self) -> int:
         if self.kind == "mlp":
             return 2 * self.H
+        if self.kind == "style":
+            return (2 * self.layers + 1) * 3 * self.D
         return (self.hq + 2 * self.hkv) * self.hd
 
     def with_M(self, M: int) -> "Workload":
@@ -130,6 +138,13 @@ WORKLOADS = {
     # down projection; both with bias), FFN hidden 4 * D (a reading)
     "video_dit_ffn": Workload("video_dit_ffn", 6, "ditffn", B=2, M=4096, D=3072,
                               H=12288, bias=True, cal_rows=256),
+    # not one of the five configurations: the modulation projection on
+    # device, one conditioning row into the rows of all 2 * 18 + 1 norms, at
+    # the stack's width and at the action expert's width
+    "style_stack18": Workload("style_stack18", 7, "style", B=1, M=1, D=512,
+                              layers=18, bias=True),
+    "style_vla18": Workload("style_vla18", 8, "style", B=1, M=1, D=2048,
+                            layers=18, bias=True),
 }
 
 
@@ -215,6 +230,17 @@ def final_norm_rows(w: Workload):
     rng = np.random.Generator(np.random.PCG64(w.seed + 31337))
     return (rng.standard_normal(size=(3, w.D), dtype=np.float32)
             * np.float32(0.02 * np.sqrt(w.D)))
+
+
+def modulation_inputs(rows: int, D: int, n_norms: int, seed: int):
+    """Conditioning rows, stacked modulation weights [n_norms * 3D, D] and
+    their bias (see the module recipe); norm i's (scale, shift, gate) are
+    output columns 3*D*i + {0, D, 2*D}."""
+    rng = np.random.Generator(np.random.PCG64(seed + 4241))
+    cond = bf16_value(normal_bf16(rng, (rows, D)))
+    w = normal_bf16(rng, (n_norms * 3 * D, D), 0.02)
+    bias = bf16_value(normal_bf16(rng, (n_norms * 3 * D,), 0.01))
+    return {"cond": cond, "w": w, "bias": bias}
 
 
 def dit_ffn_weights(D: int, H: int, seed: int):

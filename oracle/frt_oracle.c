@@ -578,6 +578,41 @@ void or_gelu_quant(int M, int H, const uint16_t *u, long ldu, float out_scale,
     free(row_amax);
 }
 
+/* ------------------------------------------------------------------ */
+/* Modulation projection ([fp8_chain] _style_stack, and the per-step    */
+/* table bake in the binder: one stacked dense projection of the        */
+/* conditioning vector gives every norm its (scale, shift, gate)).      */
+/* ------------------------------------------------------------------ */
+/*
+ * st[r, n] = sum_k cond[r, k] * w[n, k] + bias[n]
+ * in fp32 (the binder runs addmm on `.float()` tensors): products and sums
+ * rounded one at a time in k order, the bias added last (addmm's input
+ * term).  style[r, n] = bf16(st[r, n]) (the table's bf16 cast);
+ * fin[r, n - fin_col0] = st[r, n] for n >= fin_col0 (the final norm's
+ * rows, kept fp32; fin NULL skips them).  w is bf16 [N, K] row-major (the
+ * norms' dense weights concatenated along their outputs, norm i's chunks at
+ * columns 3*D*i + {0, D, 2*D}); cond fp32 [rows, K]; bias fp32 [N] or NULL.
+ * Reading: the weights are the modules' own bf16 values, which `.float()`
+ * widens exactly.
+ */
+void or_style_project(int rows, int K, int N, const float *cond,
+                      const uint16_t *w, const float *bias, uint16_t *style,
+                      float *fin, int fin_col0)
+{
+    #pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        const uint16_t *wr = w + (long)n * K;
+        for (int r = 0; r < rows; ++r) {
+            const float *cr = cond + (long)r * K;
+            float acc = 0.0f;
+            for (int k = 0; k < K; ++k) acc = acc + cr[k] * or_bf16_to_f32(wr[k]);
+            float st = bias ? acc + bias[n] : acc;
+            style[(long)r * N + n] = or_bf16_from_f32(st);
+            if (fin && n >= fin_col0) fin[(long)r * (N - fin_col0) + (n - fin_col0)] = st;
+        }
+    }
+}
+
 /* OpenMP thread count the oracle runs with (1 without OpenMP). */
 int or_num_threads(void)
 {

@@ -26,7 +26,7 @@ __all__ = [
     "ada_rms_norm_quant", "ada_layer_norm_quant_table", "pack_weights_fp8",
     "fp8_gemm", "rope_table", "split_rope_kvcache", "prefix_copy",
     "geglu_quant", "quant_fp8_static", "ada_rms_tail", "adarms_layer_stack",
-    "gelu_quant", "dit_ffn",
+    "gelu_quant", "dit_ffn", "style_project",
 ]
 
 
@@ -74,6 +74,7 @@ def _L():
             "or_quant_fp8_static": (None, [i, i, p, l, f, p, p]),
             "or_gelu_quant": (None, [i, i, p, l, f, p, p]),
             "or_ada_rms_tail": (None, [i, i, f, p, p, p, l, p, l, p]),
+            "or_style_project": (None, [i, i, i, p, p, p, p, p, i]),
             "or_num_threads": (i, []),
         }
         for name, (res, args) in sig.items():
@@ -286,6 +287,27 @@ def ada_rms_tail(res, delta, gate, fin, eps):
     _L().or_ada_rms_tail(rows, D, float(eps), _ptr(res), _ptr(delta), _ptr(gate), gs,
                          _ptr(fin), fin.shape[1], _ptr(out))
     return out
+
+
+def style_project(cond, w, bias=None, fin_col0=None):
+    """[fp8_chain] _style_stack and the binder's per-step bake: the stacked
+    modulation projection st = cond @ w.T + bias in fp32 (k order, bias
+    last).  cond fp32 [rows, K]; w bf16 bits [N, K]; bias fp32 [N] or None.
+    Returns (style bf16 bits [rows, N], fin fp32 [rows, N - fin_col0] or
+    None when fin_col0 is None)."""
+    cond = _c(np.atleast_2d(cond), np.float32)
+    w = _c(w, np.uint16)
+    rows, K = cond.shape
+    N = w.shape[0]
+    assert w.shape[1] == K
+    b = None if bias is None else _c(bias, np.float32)
+    style = np.empty((rows, N), np.uint16)
+    fin = None if fin_col0 is None else np.empty((rows, N - fin_col0), np.float32)
+    _L().or_style_project(rows, K, N, _ptr(cond), _ptr(w),
+                          None if b is None else _ptr(b), _ptr(style),
+                          None if fin is None else _ptr(fin),
+                          0 if fin_col0 is None else int(fin_col0))
+    return style, fin
 
 
 def geglu_quant(gu, out_scale):
