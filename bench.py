@@ -55,17 +55,20 @@ KERNEL_SOURCES = {
     "gemm": ("gemm.cu", "frt_sm100.cuh"),
     "producer": ("producer.cu", "frt_common.cuh", "frt_sm100.cuh", "frt_prefix.cuh"),
     "prefix_copy": ("rope.cu", "frt_prefix.cuh"),
+    "style": ("style.cu", "frt_common.cuh"),
 }
 NCU_TRAFFIC = {
     ("vla_action_expert", "gemm_rope_kv"): (5_426_432, "6d41c1fed564231c"),
     ("video_dit", "gemm_rope_kv"): (154_199_296, "6d41c1fed564231c"),
     ("gateup_mlp", "gemm_gateup_geglu"): (72_549_376, "6d41c1fed564231c"),
+    ("style_stack18", "style_project"): (58_503_936, "23ebdd084bfac401"),
 }
 
 
 def _src_hash(kernel_name):
     kind = ("gemm" if kernel_name.startswith("gemm") else
-            "producer" if kernel_name == "producer" else "prefix_copy")
+            "producer" if kernel_name == "producer" else
+            "style" if kernel_name == "style_project" else "prefix_copy")
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, "fp8_transformer_block_b200", "csrc", f),
@@ -888,6 +891,63 @@ class DitFfnRunner:
         self.pin_out.copy_(self.ff, non_blocking=True)
 
 
+class StyleRunner:
+    """Modulation projection: the conditioning rows into the (scale, shift,
+    gate) rows of all 2L + 1 norms (bf16), the final norm's rows also in
+    fp32: one launch, bound by reading the stacked bf16 weights."""
+
+    dtype = "bf16 weights/fp32 accumulate"
+
+    def __init__(self, w, torch, frt, rt, synth):
+        self.w, self.torch, self.frt, self.rt = w, torch, frt, rt
+        self.n_norms = 2 * w.layers + 1
+        rows, K, N = w.rows, w.D, w.N
+        inp = synth.modulation_inputs(rows, K, self.n_norms, w.seed)
+        self.host_in = {"cond": inp["cond"]}
+        self.cond = rt.f32_dev(inp["cond"])
+        self.wm = rt.bf16_dev(inp["w"])
+        self.bias = rt.f32_dev(inp["bias"])
+        del inp
+        self.fin_col0 = 3 * K * (self.n_norms - 1)
+        self.style = rt.empty_bf16(rows, N)
+        self.fin = torch.empty((rows, N - self.fin_col0), dtype=torch.float32,
+                               device="cuda")
+        self.kerns = [Kern("style_project", "hbm",
+                           N * K * 2 + N * 4 + rows * K * 4 + rows * N * 2
+                           + rows * (N - self.fin_col0) * 4)]
+        self.tokens = rows
+        self.launches = 1
+
+    def reset(self):
+        pass
+
+    def _project(self):
+        w = self.w
+        self.frt.frt_style_project(w.rows, w.D, w.N, self.cond, w.D, self.wm, w.D,
+                                   self.bias, self.style, w.N, self.fin,
+                                   w.N - self.fin_col0, self.fin_col0)
+
+    def step(self):
+        self._project()
+
+    def kernel_calls(self):
+        return list(zip(self.kerns, (self._project,)))
+
+    def e2e_setup(self):
+        torch = self.torch
+        self.pin_cond = torch.from_numpy(self.host_in["cond"]).pin_memory()
+        self.pin_style = torch.empty(self.style.shape, dtype=self.style.dtype).pin_memory()
+        self.pin_fin = torch.empty(self.fin.shape, dtype=self.fin.dtype).pin_memory()
+        self.h2d_bytes = self.pin_cond.numel() * 4
+        self.d2h_bytes = self.pin_style.numel() * 2 + self.pin_fin.numel() * 4
+
+    def e2e_step(self):
+        self.cond.copy_(self.pin_cond, non_blocking=True)
+        self.step()
+        self.pin_style.copy_(self.style, non_blocking=True)
+        self.pin_fin.copy_(self.fin, non_blocking=True)
+
+
 def make_runner(name, torch, frt, rt, synth):
     base, _, m = name.partition(":")
     w = synth.WORKLOADS[base]
@@ -899,10 +959,17 @@ def make_runner(name, torch, frt, rt, synth):
         return FullRunner(w, torch, frt, rt, synth)
     if w.kind == "ditffn":
         return DitFfnRunner(w, torch, frt, rt, synth)
+    if w.kind == "style":
+        return StyleRunner(w, torch, frt, rt, synth)
     return ChainRunner(w, torch, frt, rt, synth)
 
 
 def workload_text(w):
+    if w.kind == "style":
+        return (f"{w.name}: {w.rows} conditioning row(s) of D={w.D} into the "
+                f"(scale, shift, gate) rows of {2 * w.layers + 1} norms "
+                f"(N={w.N}, bf16 weights {w.N * w.D * 2 / 2**20:.0f} MiB, fp32 bias); "
+                "tokens = conditioning rows")
     if w.kind == "ditffn":
         return (f"{w.name}: B={w.B} M={w.M} D={w.D} FFN {w.H}: table producer at the FFN "
                 "site (chunks 3/4) + up GEMM with GELU requant + down GEMM, both biased")
@@ -950,6 +1017,22 @@ def oracle_sampler(name, synth, rows_cap=None):
             hid, _ = oracle.geglu_quant(gu, 0.05)
             oracle.fp8_gemm(hid, dn_p["w8"], 0.05, dn_p["w_scale"])
         return fn, len(sel), f"{len(sel)} of {w.M} rows, full MLP per row"
+
+    if w.kind == "style":
+        # columns are independent: a leading block of output columns, for
+        # every conditioning row; tokens scale with the share of columns
+        n_norms = 2 * w.layers + 1
+        inp = synth.modulation_inputs(w.rows, w.D, n_norms, w.seed)
+        n = w.N if rows_cap is None else max(1, min(w.N, rows_cap))
+        if rows_cap is None:
+            n = min(w.N, max(3 * w.D, (1 << 27) // (w.D * w.rows)))
+        wsub, bsub = inp["w"][:n].copy(), inp["bias"][:n].copy()
+        cond = inp["cond"]
+        del inp
+
+        def fn():
+            oracle.style_project(cond, wsub, bsub, fin_col0=0)
+        return fn, w.rows * n / w.N, f"{n} of {w.N} output columns, all conditioning rows"
 
     if w.kind == "ditffn":
         n = rows_cap or 32
@@ -1090,6 +1173,8 @@ def run_reference(args):
         full = w.M if w.kind == "mlp" else w.rows
         if w.kind == "ditffn":
             full = 32
+        if w.kind == "style":
+            full = min(w.N, max(3 * w.D, (1 << 27) // (w.D * w.rows)))
         cap = max(1, int(full * 150.0 / (args.steps * t1) * 0.5))
         fn, tokens, text = oracle_sampler(args.config, synth, rows_cap=cap)
     for _ in range(args.warmup):
@@ -1104,7 +1189,8 @@ def run_reference(args):
     line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3/fp32",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": StyleRunner.dtype if w.kind == "style" else "e4m3/fp32",
             "data": "synthetic", "impl": "reference",
             "config": {"workload": workload_text(w),
                        "sample_per_step": text},
@@ -1341,7 +1427,7 @@ def run_gpu(args):
         "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "us_per_layer": 1e3 * ms_per_step / L,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3/fp32", "data": "synthetic",
+        "dtype": getattr(first, "dtype", "e4m3/fp32"), "data": "synthetic",
         "config": {"workload": workload_text(w),
                    "l2": (f"inputs larger than L2: {R} independent copies of "
                           f"the workload ({R * fp / 2**20:.0f} MiB) rotated "

@@ -114,6 +114,7 @@ _SIGS = {
     "frt_quantize_fp8_static": (_i, [_i, _i, _p, _l, _p, _p, _p, _p]),
     "frt_gelu_quant_fp8": (_i, [_i, _i, _p, _l, _p, _p, _p, _p]),
     "frt_ada_rms_tail": (_i, [_i, _i, _f, _p, _p, _p, _l, _p, _l, _p, _p]),
+    "frt_style_project": (_i, [_i, _i, _i, _p, _l, _p, _l, _p, _p, _l, _p, _l, _i, _p]),
     "frt_peak_fp8_mma": (_i, [_i, _i, _p]),
     "frt_peak_copy": (_i, [_p, _p, C.c_size_t, _p]),
 }
@@ -295,6 +296,16 @@ def frt_ada_rms_tail(rows, D, eps, res, delta, gate, gate_row_stride, fin, fin_r
                                  gate_row_stride, ptr(fin), fin_row_stride, ptr(out),
                                  _stream(stream)),
            "frt_ada_rms_tail")
+
+
+def frt_style_project(rows, K, N, cond, ld_cond, w, ldw, bias, style_out, ld_style,
+                      fin_out=None, ld_fin=0, fin_col0=0, stream=None) -> None:
+    """The stacked modulation projection: style = bf16(cond @ w.T + bias),
+    and the fp32 values of columns >= fin_col0 into fin_out."""
+    _check(_lib.frt_style_project(rows, K, N, ptr(cond), ld_cond, ptr(w), ldw, ptr(bias),
+                                  ptr(style_out), ld_style, ptr(fin_out), ld_fin, fin_col0,
+                                  _stream(stream)),
+           "frt_style_project")
 
 
 def frt_peak_fp8_mma(ctas: int, iters: int, stream=None) -> None:

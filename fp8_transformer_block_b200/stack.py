@@ -9,7 +9,11 @@ and the final tail).  Per layer l, on the current stream:
   frt_packed_fp8_gemm       the output projection -> dn_o
   frt_ffn_layer             producer at slot 2l + 1 (delta dn_o, gate g1)
                             -> gate/up GEMM with the GEGLU requant -> down
-then frt_ada_rms_tail on (res, dn, g2).  Attention itself is outside this
+then frt_ada_rms_tail on (res, dn, g2).  With on-device modulation, each
+step opens with frt_style_project: the conditioning row through the stacked
+dense projection of all 2L + 1 norms (`_style_stack`), whose bf16 rows the
+layers' producers read at norm slots 2l and 2l + 1 and whose final fp32
+rows the tail reads.  Attention itself is outside this
 library; the stand-in keeps every tensor's shape and the residual moving.
 Argument marshalling only: every step runs in the CUDA library.
 """
@@ -24,11 +28,15 @@ from . import runtime as rt
 
 
 class AdaRmsLayerStack:
-    def __init__(self, w, layers, fin, scales=None, x=None):
+    def __init__(self, w, layers, fin, scales=None, x=None, modulation=None):
         """w: a "full" Workload; layers: synth.full_layer_inputs per layer;
         fin: fp32 [3, D] rows of the final norm; scales: per layer dict
         (a_qkv, a_o, a_gu, a_dn), or None to calibrate on the GPU from the
-        quantizers' amax outputs over `x` (bf16 bits [rows, D])."""
+        quantizers' amax outputs over `x` (bf16 bits [rows, D]).
+        modulation: None (the layers' own style rows and `fin`), or a dict
+        of the stacked projection "w" (bf16 bits [(2L + 1) * 3D, D]), its
+        fp32 "bias" and one fp32 conditioning row "cond" [1, D]: every step
+        then computes all norms' rows on the device (`fin` is unused)."""
         assert w.hq * w.hd == w.D, "the attention stand-in needs hq * hd == D"
         self.w = w
         B, M, D, H = w.B, w.M, w.D, w.H
@@ -49,19 +57,35 @@ class AdaRmsLayerStack:
         self.hid8 = rt.empty_u8(rows, H)
         self.gu = rt.empty_bf16(rows, 2 * H)     # calibration only
         self.out = rt.empty_bf16(rows, D)
-        self.fin = rt.f32_dev(fin)
         self.rope = rt.empty_bf16(M, w.hd)
         frt.frt_build_rope_table(M, w.hd, w.P, w.theta, self.rope)
+        self.mod = None
+        if modulation is None:
+            self.fin = rt.f32_dev(fin)
+        else:
+            n_norms = 2 * self.L + 1
+            Nm = n_norms * 3 * D
+            assert modulation["w"].shape == (Nm, D), "one (scale, shift, gate) block per norm"
+            self.mod = {"w": rt.bf16_dev(modulation["w"]),
+                        "bias": rt.f32_dev(modulation["bias"]),
+                        "cond": rt.f32_dev(np.asarray(modulation["cond"], np.float32)
+                                           .reshape(1, D)),
+                        "N": Nm, "fin_col0": 3 * D * (n_norms - 1)}
+            self.styles = rt.empty_bf16(1, Nm)
+            self.fin = torch.empty(3, D, dtype=torch.float32, device=dev)
+            self._project()
         self.lay = []
-        for li in layers:
+        for l, li in enumerate(layers):
             self.lay.append({
                 "qkv": rt.pack(li["w"], layout=frt.FRT_PACK_QK_INTERLEAVE, hd=w.hd),
                 "o": rt.pack([li["o"]]),
                 "gu": rt.pack([li["mlp"]["gate"], li["mlp"]["up"]],
                               layout=frt.FRT_PACK_GATE_UP_BLOCKS),
                 "dn": rt.pack([li["mlp"]["down"]]),
-                "st_attn": rt.bf16_dev(li["styles"][0:1]),
-                "st_ffn": rt.bf16_dev(li["styles"][1:2]),
+                "st_attn": (rt.bf16_dev(li["styles"][0:1]) if self.mod is None
+                            else self.styles[:, 3 * D * (2 * l):3 * D * (2 * l + 1)]),
+                "st_ffn": (rt.bf16_dev(li["styles"][1:2]) if self.mod is None
+                           else self.styles[:, 3 * D * (2 * l + 1):3 * D * (2 * l + 2)]),
                 "pk": rt.bf16_dev(li["prefix_k"]) if w.P else None,
                 "pv": rt.bf16_dev(li["prefix_v"]) if w.P else None,
                 "kc": torch.zeros(B, w.T, w.hkv, w.hd, dtype=torch.bfloat16, device=dev),
@@ -114,8 +138,20 @@ class AdaRmsLayerStack:
         frt.frt_packed_fp8_gemm(rows, D, D, self.o8, ly["o"].w8, scale, ly["o"].w_scale, None,
                                 frt.FRT_EPI_BF16, self.dn_o, D, None, self.ws, self.ws_bytes)
 
+    def _project(self):
+        m, D = self.mod, self.w.D
+        frt.frt_style_project(1, D, m["N"], m["cond"], D, m["w"], D, m["bias"], self.styles,
+                              m["N"], self.fin, 3 * D, m["fin_col0"])
+
+    def set_cond(self, cond):
+        """Load a new conditioning row (fp32 [1, D]) for the next steps."""
+        self.mod["cond"].copy_(torch.from_numpy(np.asarray(cond, np.float32)
+                                                .reshape(1, self.w.D)))
+
     def step(self):
         """One pass of the whole stack on the current stream."""
+        if self.mod is not None:
+            self._project()
         for l in range(self.L):
             frt.frt_chain_layer(self.cdesc[l])
             self._out_project(l, self.sdev[l]["a_o"])

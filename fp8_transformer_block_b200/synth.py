@@ -36,12 +36,13 @@ CAL_OFFSET = 500
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
-    """fp32 -> bf16 bit pattern (uint16), nearest-even; finite input only."""
+    """fp32 -> bf16 bit pattern (uint16), nearest-even; finite input only:
+    adding 0x7FFF plus the kept part's lowest bit carries into the kept
+    half exactly when the dropped half is above one half, or equal to it
+    with an odd kept part."""
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    keep = (u >> 16).astype(np.uint32)
-    rest = u & np.uint32(0xFFFF)
-    up = (rest > 0x8000) | ((rest == 0x8000) & ((keep & 1) == 1))
-    return (keep + up.astype(np.uint32)).astype(np.uint16)
+    r = u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    return (r >> np.uint32(16)).astype(np.uint16)
 
 
 def bf16_value(h: np.ndarray) -> np.ndarray:
@@ -51,8 +52,21 @@ def bf16_value(h: np.ndarray) -> np.ndarray:
 
 
 def normal_bf16(rng: np.random.Generator, shape, std: float = 1.0):
-    return bf16_bits(rng.standard_normal(size=shape, dtype=np.float32)
-                     * np.float32(std))
+    """N(0, std) draws rounded to bf16 bit patterns.  Large arrays are drawn
+    in blocks of leading rows: the generator's stream, and so every value,
+    is the same as one draw of the whole shape."""
+    shape = tuple(np.atleast_1d(shape)) if not isinstance(shape, tuple) else shape
+    n = int(np.prod(shape))
+    if len(shape) < 2 or n <= (1 << 24):
+        return bf16_bits(rng.standard_normal(size=shape, dtype=np.float32)
+                         * np.float32(std))
+    out = np.empty(shape, np.uint16)
+    step = max(1, (1 << 24) // int(np.prod(shape[1:])))
+    for i in range(0, shape[0], step):
+        blk = (min(step, shape[0] - i),) + shape[1:]
+        out[i:i + blk[0]] = bf16_bits(rng.standard_normal(size=blk, dtype=np.float32)
+                                      * np.float32(std))
+    return out
 
 
 def outlier_rows(rng: np.random.Generator, rows: int, frac: float = 0.01):

@@ -419,6 +419,36 @@ int frt_ada_rms_tail(int rows, int D, float eps, const frt_bf16* res,
                      long gate_row_stride, const float* fin, long fin_row_stride,
                      frt_bf16* out, void* stream);
 
+/*
+ * frt_style_project (fp8_chain.py `_style_stack`: one stacked dense
+ * projection serves every norm's (scale, shift, gate); the binder there
+ * evaluates it with addmm in fp32 once per probed step and casts the rows
+ * to bf16, keeping the final norm's rows in fp32).  This computes it on the
+ * device for the live conditioning.  For each row r < rows and column n < N,
+ * fp32 throughout:
+ *   st[r, n]  = sum_k cond[r, k] * w[n, k] + bias[n]    (bias last)
+ *   style_out[r * ld_style + n] = bf16(st[r, n])        (round to nearest even)
+ *   fin_out[r * ld_fin + n - fin_col0] = st[r, n]       for n >= fin_col0
+ * cond: device fp32 [rows, K], rows ld_cond elements apart (16-byte aligned,
+ * ld_cond % 4 == 0).  w: device bf16 [N, K], rows ldw elements apart
+ * (16-byte aligned, ldw % 8 == 0): the norms' dense weights concatenated
+ * along their outputs, so norm i's scale, shift and gate are columns
+ * 3*D*i + {0, D, 2*D} (+ j) and the style rows of norm i start at column
+ * 3*D*i of style_out.  bias: device fp32 [N] or NULL.  fin_out: device fp32
+ * or NULL (skipped); with a stacked layout, fin_col0 = 3*D*(n_norms - 1)
+ * gives the final norm's (scale, shift, gate) rows D apart, the form
+ * frt_ada_rms_tail reads.  K % 8 == 0, 8 <= K <= 65536, N >= 1,
+ * 0 <= rows <= 65535 (0 is a no-op).  The sum's order differs from index
+ * order (lanes split K); each result is within (K + 2) * 2^-24 *
+ * (sum_k |cond * w| + |bias|) of the exact value.  w and bias are read
+ * before the launch waits on the kernel ahead of it in the stream (they are
+ * bind-time data): no kernel still running may write them.
+ */
+int frt_style_project(int rows, int K, int N, const float* cond, long ld_cond,
+                      const frt_bf16* w, long ldw, const float* bias,
+                      frt_bf16* style_out, long ld_style, float* fin_out,
+                      long ld_fin, int fin_col0, void* stream);
+
 /* ----------------------------------------------------------------------- */
 /* Self-test of the bounded device wait.                                    */
 /* ----------------------------------------------------------------------- */

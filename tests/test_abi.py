@@ -177,6 +177,18 @@ def test_output_side_validation(frt):
              frt.FRT_EPI_GELU_E4M3, A16, 256, None, None, 0, None) == frt.FRT_EINVAL
     assert q("frt_packed_fp8_gemm", 4, 256, 512, A16, A16, A16, A16, None, 9, A16, 256,
              A16, None, 0, None) == frt.FRT_EINVAL
+    # modulation projection: K % 8, a row stride below K, misalignment,
+    # fin_col0 past N, a missing operand; no rows is a no-op
+    sp = "frt_style_project"
+    assert q(sp, 1, 12, 64, A16, 12, A16, 16, None, A16, 64, None, 0, 0, None) == frt.FRT_ESHAPE
+    assert q(sp, 1, 64, 64, A16, 64, A16, 32, None, A16, 64, None, 0, 0, None) == frt.FRT_EALIGN
+    assert q(sp, 1, 64, 64, A16, 66, A16, 64, None, A16, 64, None, 0, 0, None) == frt.FRT_EALIGN
+    assert q(sp, 1, 64, 64, A16, 64, A16 + 8, 64, None, A16, 64, None, 0, 0, None) == \
+        frt.FRT_EALIGN
+    assert q(sp, 1, 64, 64, A16, 64, A16, 64, None, A16, 64, A16, 64, 65, None) == frt.FRT_ERANGE
+    assert q(sp, 1, 64, 64, None, 64, A16, 64, None, A16, 64, None, 0, 0, None) == frt.FRT_EINVAL
+    assert q(sp, 1, 64, 64, A16, 64, A16, 64, None, A16, 32, None, 0, 0, None) == frt.FRT_ESHAPE
+    assert q(sp, 0, 64, 64, A16, 64, A16, 64, None, A16, 64, A16, 192, 0, None) == frt.FRT_OK
     # FFN half: no descriptor; the peak probe: no CTAs
     assert q("frt_ffn_layer", None, None) == frt.FRT_EINVAL
     assert q("frt_peak_fp8_mma", 0, 10, None) == frt.FRT_EINVAL

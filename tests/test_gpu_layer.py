@@ -92,3 +92,49 @@ def test_layer_stack_gpu_calibration_runs(rt):
     assert frt.frt_device_status(True) == frt.FRT_OK
     out = bf16_value(runtime.bf16_host(st.out))
     assert np.all(np.isfinite(out)) and 0.5 < float(np.sqrt((out ** 2).mean())) < 50
+
+
+def test_layer_stack_modulation_on_device(rt):
+    """Every step computes all norms' (scale, shift, gate) rows from the
+    conditioning row on the device (`_style_stack`): the projection's rows
+    against the oracle's, then the whole stack against the oracle's
+    composition fed the oracle's rows, for two conditioning rows in turn."""
+    frt, runtime, stack, torch = rt
+    w = synth.WORKLOADS["adarms_layer18"].with_M(16)
+    L = 3
+    lays = [synth.full_layer_inputs(w, l) for l in range(L)]
+    mod = synth.modulation_inputs(2, w.D, 2 * L + 1, w.seed)
+    x = synth.adarms_inputs(w.rows, w.D, w.seed)["res"]
+    dims = {"B": w.B, "M": w.M, "D": w.D, "hq": w.hq, "hkv": w.hkv, "hd": w.hd,
+            "P": w.P, "T": w.T, "H": w.H, "theta": w.theta}
+    fin_col0 = 3 * w.D * 2 * L
+    st = None
+    for i in range(2):
+        cond = mod["cond"][i:i + 1]
+        style_ref, fin_ref = oracle.style_project(cond, mod["w"], mod["bias"], fin_col0=fin_col0)
+        lays_i = [dict(li, styles=style_ref[0, 3 * w.D * 2 * l:3 * w.D * (2 * l + 2)]
+                       .reshape(2, 3 * w.D)) for l, li in enumerate(lays)]
+        ol = _oracle_layers(lays_i, w)
+        fin = fin_ref.reshape(3, w.D)
+        if st is None:
+            _, _, scales = oracle.adarms_layer_stack(x, ol, fin, dims)
+            st = stack.AdaRmsLayerStack(w, lays, None, scales=scales,
+                                        modulation={"w": mod["w"], "bias": mod["bias"],
+                                                    "cond": cond})
+        else:
+            st.set_cond(cond)
+        ref, _, _ = oracle.adarms_layer_stack(x, ol, fin, dims, scales=scales)
+        st.load(x)
+        st.step()
+        torch.cuda.synchronize()
+        assert frt.frt_device_status(True) == frt.FRT_OK
+        gs = runtime.bf16_host(st.styles)
+        same = float((gs == style_ref).mean())
+        assert same >= 0.999, f"cond {i}: style rows {same:.5f} identical"
+        assert np.all(np.abs(bf16_value(gs) - bf16_value(style_ref))
+                      <= 2.0 ** -7 * np.abs(bf16_value(style_ref)) + 1e-6), f"cond {i}: style"
+        fg = st.fin.cpu().numpy().reshape(1, -1)
+        assert np.allclose(fg, fin_ref, rtol=0, atol=1e-5), f"cond {i}: final rows"
+        e = _rel_l2(runtime.bf16_host(st.out), ref)
+        print(f"modulated stack, cond {i}: final output rel-L2 {e:.3e}")
+        assert e <= 2e-2, f"cond {i}: final tail output"
