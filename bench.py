@@ -58,10 +58,11 @@ KERNEL_SOURCES = {
     "style": ("style.cu", "frt_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("vla_action_expert", "gemm_rope_kv"): (5_426_432, "6d41c1fed564231c"),
-    ("video_dit", "gemm_rope_kv"): (154_199_296, "6d41c1fed564231c"),
-    ("gateup_mlp", "gemm_gateup_geglu"): (72_549_376, "6d41c1fed564231c"),
+    ("vla_action_expert", "gemm_rope_kv"): (5_425_493, "354d15aca37e8da8"),
+    ("video_dit", "gemm_rope_kv"): (153_956_864, "354d15aca37e8da8"),
+    ("gateup_mlp", "gemm_gateup_geglu"): (72_654_848, "354d15aca37e8da8"),
     ("style_stack18", "style_project"): (58_503_936, "23ebdd084bfac401"),
+    ("style_vla18", "style_project"): (935_918_080, "23ebdd084bfac401"),
 }
 
 

@@ -65,7 +65,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 // The same wait with cluster-scope acquire, for phases completed by arrivals
-// from other CTAs of the cluster (mbar_arrive_release_cluster).
+// from other CTAs of the cluster (MMA commits multicast to them, remote
+// arrivals, bulk copies' transaction bytes).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -163,6 +164,15 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
       :: "r"(smem_u32(bar)) : "memory");
+}
+
+// Arrive once, when this thread's MMAs complete, on the barrier at `bar`'s
+// offset in every CTA of `cta_mask` (single-CTA MMAs).
+__device__ __forceinline__ void umma_commit_mc(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;"
+      :: "r"(smem_u32(bar)), "h"(cta_mask) : "memory");
 }
 
 // Instruction descriptor, kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B e4m3
@@ -321,9 +331,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar_clust
                :: "r"(bar_cluster), "r"(bytes) : "memory");
 }
 
-// Arrive, with cluster-scope release, on a barrier of another CTA.
-__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+// Arrive on a barrier of another CTA with no memory ordering: a bare signal,
+// for barriers that order nothing the arriving thread itself wrote or read.
+__device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];"
                :: "r"(bar_cluster) : "memory");
 }
 

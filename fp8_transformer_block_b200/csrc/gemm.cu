@@ -404,8 +404,9 @@ __host__ __device__ constexpr int smem_total() {
 
 // CLUSTER: the p.splits K-splits of a tile run as one thread-block cluster
 // (rank = split, one unit per CTA); each CTA stages its fp32 partial in its
-// shared memory.  Rank 0 (the leader) tells the others when its operand ring
-// is free (its last MMA is done); each other rank then bulk-copies its
+// shared memory.  The leader's (rank 0's) last MMA commit also arrives on
+// the other ranks' `go` barriers (commit multicast), so they learn its
+// operand ring is free the moment its MMAs complete; each then bulk-copies its
 // staged partial into slot rank-1 of the leader's ring, counted as
 // transaction bytes on the leader's barrier red_full, and leaves once the
 // leader confirms receipt.  The leader sums the partials in rank order from
@@ -548,6 +549,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     if (CLUSTER) cluster_wait();
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
+    // (cluster: the other ranks' barriers exist before the commit below
+    // arrives on them)
+    if (CLUSTER) cluster_wait();
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_e4m3_f32(BMT, BN);
       const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
@@ -576,6 +580,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         }
         if (!ok) break;
         umma_commit(&tfull[ab]);
+        // cluster leader: its ring is free once these MMAs complete; the
+        // same completion tells the other ranks to send their partials
+        if (CLUSTER && p.splits > 1 && cluster_ctarank() == 0)
+          umma_commit_mc(go, uint16_t(((1u << p.splits) - 1u) & ~1u));
       }
       if (!ok) {
         record_timeout(p.status);
@@ -585,7 +593,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       }
     }
     __syncwarp();  // converge before the block barrier and the TMEM release
-    if (CLUSTER) cluster_wait();
   } else {
     // ----------------------------------------------------------- epilogue --
     // The rope table is bind-time data: pull this CTA's first-unit rows into
@@ -647,13 +654,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       tc_fence_after();
       const uint32_t tbase = tmem_base + uint32_t(ab * BN) + (uint32_t(32 * q) << 16);
       if (CLUSTER) {
-        // one unit per CTA.  The leader's MMAs are done: its ring is free
-        // for the other ranks' partials.  Then stage this rank's partial.
+        // one unit per CTA: stage this rank's partial (the leader's MMA
+        // completion has already told the other ranks its ring is free)
         cluster_wait();
         cwaited = true;
-        if (crank == 0 && threadIdx.x == 64)
-          for (int j = 1; j < p.splits; ++j)
-            mbar_arrive_release_cluster(map_cluster(smem_u32(go), uint32_t(j)));
         stage_swap_tile<BMT, BN>(T, q, lane,
                                  [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); });
         staged = true;
@@ -764,7 +768,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         if (threadIdx.x == 64) {
           if (got) {
             for (int j = 1; j < p.splits; ++j)
-              mbar_arrive_release_cluster(map_cluster(smem_u32(done), uint32_t(j)));
+              mbar_arrive_relaxed_cluster(map_cluster(smem_u32(done), uint32_t(j)));
           } else {
             record_timeout(p.status);
           }
@@ -1227,10 +1231,12 @@ gemm_pair_split_kernel(const __grid_constant__ CUtensorMap tmA,
       __syncwarp();
     } else {
       // this CTA's MMAs are done: its ring may receive the other half's rows
-      if (threadIdx.x == 64) mbar_arrive_release_cluster(map_cluster(smem_u32(go), rank + 2u));
+      // (bare signals: what they order -- the MMAs' reads of the ring, the
+      // bulk copy's writes -- is ordered by the barriers those complete on)
+      if (threadIdx.x == 64) mbar_arrive_relaxed_cluster(map_cluster(smem_u32(go), rank + 2u));
       const bool in = mbar_wait_bounded_cluster(red_full, 0, kWaitNs);
       if (threadIdx.x == 64) {
-        if (in) mbar_arrive_release_cluster(map_cluster(smem_u32(done), rank + 2u));
+        if (in) mbar_arrive_relaxed_cluster(map_cluster(smem_u32(done), rank + 2u));
         else record_timeout(p.status);
       }
       if (in) {
