@@ -58,9 +58,9 @@ KERNEL_SOURCES = {
     "style": ("style.cu", "frt_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("vla_action_expert", "gemm_rope_kv"): (5_425_493, "354d15aca37e8da8"),
-    ("video_dit", "gemm_rope_kv"): (153_956_864, "354d15aca37e8da8"),
-    ("gateup_mlp", "gemm_gateup_geglu"): (72_654_848, "354d15aca37e8da8"),
+    ("vla_action_expert", "gemm_rope_kv"): (5_428_309, "ef7069072267bf17"),
+    ("video_dit", "gemm_rope_kv"): (156_936_192, "ef7069072267bf17"),
+    ("gateup_mlp", "gemm_gateup_geglu"): (72_675_328, "ef7069072267bf17"),
     ("style_stack18", "style_project"): (58_503_936, "23ebdd084bfac401"),
     ("style_vla18", "style_project"): (935_918_080, "23ebdd084bfac401"),
 }

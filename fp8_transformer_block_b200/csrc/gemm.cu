@@ -524,8 +524,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             if (SWAP) tma_load_2d(sA + stage * A_BYTES, wmap, &full[stage], kb * BK, ta * BMT);
             else tma_load_2d(sB + stage * B_BYTES, wmap, &full[stage], kb * BK, tb * BN);
           }
-          if (SWAP) tma_load_2d(sB + stage * B_BYTES, xmap, &full[stage], kb * BK, tb * BN);
-          else tma_load_2d(sA + stage * A_BYTES, xmap, &full[stage], kb * BK, ta * BMT);
+          if (!(SWAP && CLUSTER && pre)) {
+            if (SWAP) tma_load_2d(sB + stage * B_BYTES, xmap, &full[stage], kb * BK, tb * BN);
+            else tma_load_2d(sA + stage * A_BYTES, xmap, &full[stage], kb * BK, ta * BMT);
+          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -611,6 +613,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       }
     }
     pdl_wait();
+    if (SWAP && CLUSTER && lane == 0 && blockIdx.x < unsigned(p.units)) {
+      // the activation boxes of the stages prefetched with weights, spread
+      // over the four epilogue warps (idle until the accumulator is full):
+      // the stages fill in about the time of one box instead of one after
+      // another behind the producer thread's issue
+      const int u0 = blockIdx.x;
+      const int tile = u0 / p.splits, split = u0 % p.splits;
+      const int tb = tile / p.a_tiles;
+      const int kb0 = int(long(split) * p.k_blocks / p.splits);
+      const int kb1 = int(long(split + 1) * p.k_blocks / p.splits);
+      const int n_pre = kb1 - kb0 < STAGES ? kb1 - kb0 : STAGES;
+      for (int i = warp - 2; i < n_pre; i += 4)
+        tma_load_2d(sB + i * B_BYTES, &tmB, &full[i], (kb0 + i) * BK, tb * BN);
+    }
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
     const int row = acc_row<BMT>(q, lane);
