@@ -61,8 +61,8 @@ NCU_TRAFFIC = {
     ("vla_action_expert", "gemm_rope_kv"): (5_428_309, "ef7069072267bf17"),
     ("video_dit", "gemm_rope_kv"): (156_936_192, "ef7069072267bf17"),
     ("gateup_mlp", "gemm_gateup_geglu"): (72_675_328, "ef7069072267bf17"),
-    ("style_stack18", "style_project"): (58_503_936, "23ebdd084bfac401"),
-    ("style_vla18", "style_project"): (935_918_080, "23ebdd084bfac401"),
+    ("style_stack18", "style_project"): (58_491_392, "aefda1df19f33ba3"),
+    ("style_vla18", "style_project"): (935_920_640, "aefda1df19f33ba3"),
 }
 
 

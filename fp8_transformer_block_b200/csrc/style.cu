@@ -168,25 +168,35 @@ constexpr size_t kStyleSmem = size_t(kStyleWarps) * kStyleDepth * kStyleCols * 3
 
 }  // namespace
 
-// Resident CTAs per SM of the R-row kernel (its registers decide), asked of
-// the runtime once per instantiation.
+// Resident CTAs per SM of the R-row kernel (its registers and ring decide),
+// per device; the shared-memory limit is raised once per kernel and device.
 template <int R>
 int style_blocks_per_sm() {
-  static int cached = 0;
-  if (cached == 0) {
-    auto kern = style_project_kernel<R, kStyleDepth>;
-    int n = 0;
+  static int cache[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto kern = style_project_kernel<R, kStyleDepth>;
+  if (first_use(reinterpret_cast<const void*>(kern))) {
+    // (this claims the kernel's first use, so the carveout the launch helper
+    // sets on first use is set here too)
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(kStyleSmem)) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kStyleWarps * 32,
-                                                      kStyleSmem) != cudaSuccess ||
-        n < 1) {
+                             int(kStyleSmem)) != cudaSuccess) {
       cudaGetLastError();
-      n = 1;
+      return 0;
     }
-    cached = n;
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
   }
-  return cached;
+  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kStyleWarps * 32, kStyleSmem) !=
+          cudaSuccess ||
+      n < 1) {
+    cudaGetLastError();
+    n = 1;
+  }
+  if (dev < 64) cache[dev] = n;
+  return n;
 }
 
 }  // namespace frt
@@ -224,6 +234,8 @@ extern "C" int frt_style_project(int rows, int K, int N, const float* cond, long
   const dim3 block(frt::kStyleWarps * 32);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto go = [&](auto kern, int per_sm, unsigned groups) {
+    if (per_sm < 1)
+      return frt::fail(FRT_ECUDA, "style_project_kernel: cannot raise its shared-memory limit");
     // persistent: as many CTAs as fit on the SMs at once (row groups
     // share them), never more than there are tasks
     const long cap = long(per_sm) * frt::num_sms();
