@@ -440,12 +440,14 @@ class ChainRunner:
 
     # ---------------------------------------------------------------- e2e --
     def e2e_setup(self):
-        """Host-buffer form of the step: the step's inputs sit back to back
-        in one pinned host buffer and one device arena (the chain's input
-        tensors become views of it), so a step copies them in with one
+        """Host-buffer form of the step: the step's token inputs sit back to
+        back in one pinned host buffer and one device arena (the chain's
+        input tensors become views of it), so a step copies them in with one
         host->device copy; the residual, the last layer's q and gate outputs
         follow them in the arena and come back with one device->host copy,
-        the new K/V cache rows with one copy each."""
+        the new K/V cache rows with one copy each.  The prefix K/V stays in
+        device memory, like the weights: it is the host model's own cache,
+        which the chain gathers from on the device."""
         torch, w, L = self.torch, self.w, self.L
         lq = (L - 1) % 2
         # (name, device tensor, host array or None, setter)
@@ -462,12 +464,6 @@ class ChainRunner:
                         lambda t: setattr(self, "gate", t)))
             ins.append(("style", self.style1, self.host_in["style"],
                         lambda t: setattr(self, "style1", t)))
-        for l, lay in enumerate(self.layers):
-            if lay["pk_host"] is not None:
-                ins.append((f"pk{l}", lay["pkd"], lay["pk_host"],
-                            lambda t, lay=lay: lay.__setitem__("pkd", t)))
-                ins.append((f"pv{l}", lay["pvd"], lay["pv_host"],
-                            lambda t, lay=lay: lay.__setitem__("pvd", t)))
         outs = []
         if not self.dit:   # the residual is both an input and an output
             ins.append(("res", self.res, self.host_in["res"],
@@ -741,15 +737,13 @@ class FullRunner:
 
     # ---------------------------------------------------------------- e2e --
     def e2e_setup(self):
-        """The step's inputs (the rows entering the stack and every layer's
-        host prefix cache) back to back in one pinned buffer and one device
-        arena the stack reads directly (one host->device copy); the output
-        rows and each layer's new K/V rows come back with one copy each."""
+        """The step's input (the rows entering the stack) in a pinned buffer
+        and a device arena the stack reads directly (one host->device copy);
+        the output rows and each layer's new K/V rows come back with one copy
+        each.  Every layer's prefix K/V stays in device memory, like the
+        weights (the host model's own cache)."""
         torch, st, w = self.torch, self.st, self.w
         ins = [("x", st.res, self.x_host)]
-        for l, ly in enumerate(st.lay):
-            ins.append((f"pk{l}", ly["pk"], self.pk_host[l][0]))
-            ins.append((f"pv{l}", ly["pv"], self.pk_host[l][1]))
         offs, n = {}, 0
         for name, t, _ in ins:
             offs[name] = n
@@ -764,8 +758,6 @@ class FullRunner:
                 torch.from_numpy(np.ascontiguousarray(host).view(np.int16).reshape(-1)))
             views[name] = v
         st.res = views["x"]
-        for l, ly in enumerate(st.lay):
-            ly["pk"], ly["pv"] = views[f"pk{l}"], views[f"pv{l}"]
         st._build()
         self.arena, self.pin_arena, self.n_in = arena, pin, n
         self.outs = [(st.out, torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory())]
@@ -1439,7 +1431,11 @@ def run_gpu(args):
                    "timing": "K back-to-back steps replayed from CUDA graphs, "
                              "CUDA events around the K steps on the launching "
                              "stream; kernels timed the same way",
-                   "isolated_step_us_after_l2_flush": round(iso_us, 3)},
+                   "isolated_step_us_after_l2_flush": round(iso_us, 3),
+                   "e2e_scope": "each step copies the tokens' input rows in from pinned "
+                                "host memory and reads its output rows (and new K/V rows) "
+                                "back; weights, tables and the prefix K/V cache (the host "
+                                "model's device-resident cache) stay in device memory"},
         "roofline": {"bound": kd.bound, "kernel": kd.name,
                      "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic,
