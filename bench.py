@@ -644,7 +644,12 @@ class FullRunner:
         lays = [synth.full_layer_inputs(w, l) for l in range(L)]
         fin = synth.final_norm_rows(w)
         cal = synth.adarms_inputs(rows, D, w.seed + synth.CAL_OFFSET)["res"]
-        self.st = stack.AdaRmsLayerStack(w, lays, fin, x=cal)
+        mod = None
+        if w.live:
+            m = synth.modulation_inputs(1, D, 2 * L + 1, w.seed)
+            mod = {"w": m["w"], "bias": m["bias"], "cond": m["cond"]}
+            self.cond_host = m["cond"]
+        self.st = stack.AdaRmsLayerStack(w, lays, fin, x=cal, modulation=mod)
         self.x_host = synth.adarms_inputs(rows, D, w.seed)["res"]
         self.x0 = rt.bf16_dev(self.x_host)
         self.st.res.copy_(self.x0)
@@ -667,6 +672,11 @@ class FullRunner:
         ]
         self.tokens = rows
         self.launches = 7 * L + 1
+        if w.live:
+            Nm = (2 * L + 1) * 3 * D
+            self.kerns.insert(0, Kern("style_project", "hbm",
+                                      Nm * D * 2 + Nm * 4 + D * 4 + Nm * 2 + 12 * D))
+            self.launches += 1
 
     def footprint(self):
         st, seen, total = self.st, set(), 0
@@ -674,6 +684,8 @@ class FullRunner:
         for v in vars(st).values():
             if isinstance(v, list):
                 ts += [x for x in v if isinstance(x, self.torch.Tensor)]
+            elif isinstance(v, dict):
+                ts += [x for x in v.values() if isinstance(x, self.torch.Tensor)]
         for ly in st.lay:
             for v in ly.values():
                 if isinstance(v, self.torch.Tensor):
@@ -732,8 +744,10 @@ class FullRunner:
         def tail():
             frt.frt_ada_rms_tail(rows, D, w.eps, st.res, st.dn[0], st.g2[0], D, st.fin, D,
                                  st.out)
-        return list(zip(self.kerns, (prefix, producer, gemm_rope, quant, gemm_o, gemm_gu,
-                                     gemm_dn, tail)))
+        calls = [prefix, producer, gemm_rope, quant, gemm_o, gemm_gu, gemm_dn, tail]
+        if w.live:
+            calls.insert(0, st._project)
+        return list(zip(self.kerns, calls))
 
     # ---------------------------------------------------------------- e2e --
     def e2e_setup(self):
@@ -744,20 +758,25 @@ class FullRunner:
         weights (the host model's own cache)."""
         torch, st, w = self.torch, self.st, self.w
         ins = [("x", st.res, self.x_host)]
+        if w.live:   # the step's conditioning row (fp32) comes in with it
+            ins.append(("cond", st.mod["cond"], self.cond_host))
         offs, n = {}, 0
         for name, t, _ in ins:
             offs[name] = n
-            n += (t.numel() + 127) // 128 * 128
+            n += (t.numel() * t.element_size() // 2 + 127) // 128 * 128
         arena = torch.empty(n, dtype=torch.int16, device="cuda")
         pin = torch.empty(n, dtype=torch.int16).pin_memory()
         views = {}
         for name, t, host in ins:
-            v = arena[offs[name]:offs[name] + t.numel()].view(t.dtype).view(t.shape)
+            m = t.numel() * t.element_size() // 2
+            v = arena[offs[name]:offs[name] + m].view(t.dtype).view(t.shape)
             v.copy_(t)
-            pin[offs[name]:offs[name] + t.numel()].copy_(
+            pin[offs[name]:offs[name] + m].copy_(
                 torch.from_numpy(np.ascontiguousarray(host).view(np.int16).reshape(-1)))
             views[name] = v
         st.res = views["x"]
+        if w.live:
+            st.mod["cond"] = views["cond"]
         st._build()
         self.arena, self.pin_arena, self.n_in = arena, pin, n
         self.outs = [(st.out, torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory())]
@@ -970,7 +989,10 @@ def workload_text(w):
         return (f"{w.name}: B={w.B} M={w.M} D={w.D} Hq={w.hq}x{w.hd} Hkv={w.hkv}x{w.hd} "
                 f"P={w.P} T={w.T} FFN {w.H}, {w.layers} whole layers except attention "
                 "(q/k/v chain, output projection on the attention stand-in q_out, "
-                "FFN half) + final tail")
+                "FFN half) + final tail"
+                + (", every step opening with the modulation projection of one "
+                   f"conditioning row into all {2 * w.layers + 1} norms' rows"
+                   if w.live else ""))
     if w.kind == "mlp":
         return (f"{w.name}: M={w.M} D={w.D} gate/up {w.H} each (packed "
                 f"N={2 * w.H}) + GEGLU requant + down [{w.D},{w.H}]")
@@ -1058,11 +1080,19 @@ def oracle_sampler(name, synth, rows_cap=None):
         dims = {"B": 1, "M": n, "D": w.D, "hq": w.hq, "hkv": w.hkv, "hd": w.hd,
                 "P": w.P, "T": wl.T, "H": w.H, "theta": w.theta}
         fixed = [{"a_qkv": 0.01, "a_o": 0.01, "a_gu": 0.01, "a_dn": 0.05}] * w.layers
+        mod = synth.modulation_inputs(1, w.D, 2 * w.layers + 1, w.seed) if w.live else None
 
         def fn():
-            oracle.adarms_layer_stack(x, ol, fin, dims, scales=fixed, eps=w.eps)
+            f, layers = fin, ol
+            if mod is not None:
+                st, f = oracle.style_project(mod["cond"], mod["w"], mod["bias"],
+                                             fin_col0=3 * w.D * 2 * w.layers)
+                f = f.reshape(3, w.D)
+                layers = [dict(li, styles=st[0, 6 * w.D * l:6 * w.D * (l + 1)].reshape(2, 3 * w.D))
+                          for l, li in enumerate(ol)]
+            oracle.adarms_layer_stack(x, layers, f, dims, scales=fixed, eps=w.eps)
         return fn, n, (f"{n} of {w.rows} rows, {w.layers} whole layers except attention "
-                       "+ tail")
+                       "+ tail" + (", with the modulation projection" if w.live else ""))
 
     L = w.layers
     rows = w.rows

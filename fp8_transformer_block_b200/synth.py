@@ -104,6 +104,7 @@ class Workload:
     theta: float = 10000.0
     eps: float = 1e-6
     m_sweep: tuple = field(default_factory=tuple)
+    live: bool = False  # "full": every step projects the norms' rows from cond
 
     @property
     def seed(self) -> int:
@@ -147,6 +148,11 @@ WORKLOADS = {
     "adarms_layer18": Workload("adarms_layer18", 5, "full", B=1, M=50, D=512,
                                hq=8, hkv=1, hd=64, P=816, T=866, H=2048,
                                layers=18, cal_rows=64),
+    # the same loop with the modulation projection on device at the head of
+    # every step (one conditioning row into all 2 * 18 + 1 norms' rows)
+    "adarms_layer18_live": Workload("adarms_layer18_live", 9, "full", B=1, M=50, D=512,
+                                    hq=8, hkv=1, hd=64, P=816, T=866, H=2048,
+                                    layers=18, cal_rows=64, live=True),
     # not one of the five configurations: the video-DiT block's FFN half
     # (producer at the FFN site, chunks 3/4; up projection + GELU requant;
     # down projection; both with bias), FFN hidden 4 * D (a reading)
