@@ -257,7 +257,6 @@ class ChainRunner:
                 "vc": torch.zeros(B, w.T, w.hkv, w.hd, dtype=torch.bfloat16,
                                   device="cuda"),
                 "style": None if style is None else rt.bf16_dev(style),
-                "pk_host": pkh, "pv_host": pvh,
                 "pkd": None if pkh is None else rt.bf16_dev(pkh),
                 "pvd": None if pvh is None else rt.bf16_dev(pvh),
                 "T_src": 0 if pkh is None else int(pkh.shape[2])})
@@ -653,7 +652,6 @@ class FullRunner:
         self.x_host = synth.adarms_inputs(rows, D, w.seed)["res"]
         self.x0 = rt.bf16_dev(self.x_host)
         self.st.res.copy_(self.x0)
-        self.pk_host = [(li["prefix_k"], li["prefix_v"]) for li in lays]
         N = (w.hq + 2 * w.hkv) * w.hd
         gb = N * D + rows * D + w.M * w.hd * 2 + rows * N * 2
         gf = 2.0 * rows * N * D
