@@ -58,9 +58,9 @@ KERNEL_SOURCES = {
     "style": ("style.cu", "frt_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("vla_action_expert", "gemm_rope_kv"): (5_428_309, "ef7069072267bf17"),
-    ("video_dit", "gemm_rope_kv"): (156_936_192, "ef7069072267bf17"),
-    ("gateup_mlp", "gemm_gateup_geglu"): (72_675_328, "ef7069072267bf17"),
+    ("vla_action_expert", "gemm_rope_kv"): (5_428_309, "37cca62b76d214c9"),
+    ("video_dit", "gemm_rope_kv"): (156_936_192, "37cca62b76d214c9"),
+    ("gateup_mlp", "gemm_gateup_geglu"): (72_675_328, "37cca62b76d214c9"),
     ("style_stack18", "style_project"): (58_491_392, "aefda1df19f33ba3"),
     ("style_vla18", "style_project"): (935_920_640, "aefda1df19f33ba3"),
 }

@@ -1700,6 +1700,24 @@ extern "C" size_t frt_gemm_workspace_size(int M, int N, int K, int epilogue) {
       .ws_bytes;
 }
 
+extern "C" int frt_gemm_plan_info(int M, int N, int K, int epilogue, int* info, int n) {
+  frt::clear_error();
+  FRT_REQUIRE(info && n >= FRT_PLAN_INFO_LEN, FRT_EINVAL,
+              "info must hold FRT_PLAN_INFO_LEN (%d) ints", FRT_PLAN_INFO_LEN);
+  FRT_REQUIRE(M >= 0 && N > 0 && K > 0, FRT_ESHAPE, "M must be >= 0 and N, K positive");
+  FRT_REQUIRE(epilogue >= FRT_EPI_BF16 && epilogue <= FRT_EPI_GELU_E4M3, FRT_EINVAL,
+              "unknown epilogue %d", epilogue);
+  if (M == 0) {  // nothing is launched
+    for (int i = 0; i < FRT_PLAN_INFO_LEN; ++i) info[i] = 0;
+    return FRT_OK;
+  }
+  const frt::Plan pl = frt::make_plan(M, N, K, frt::epi_of(epilogue));
+  const int v[FRT_PLAN_INFO_LEN] = {pl.swap,  pl.pair,   pl.split2, pl.cluster, pl.bmt,
+                                    pl.bn,    pl.splits, pl.units,  pl.grid,    pl.k_blocks};
+  for (int i = 0; i < FRT_PLAN_INFO_LEN; ++i) info[i] = v[i];
+  return FRT_OK;
+}
+
 extern "C" int frt_packed_fp8_gemm(int M, int N, int K, const frt_e4m3* x8, const frt_e4m3* w8,
                                    const float* act_scale, const float* w_scale,
                                    const frt_bf16* bias, int epilogue, void* out, long ldo,

@@ -115,6 +115,7 @@ _SIGS = {
     "frt_gelu_quant_fp8": (_i, [_i, _i, _p, _l, _p, _p, _p, _p]),
     "frt_ada_rms_tail": (_i, [_i, _i, _f, _p, _p, _p, _l, _p, _l, _p, _p]),
     "frt_style_project": (_i, [_i, _i, _i, _p, _l, _p, _l, _p, _p, _l, _p, _l, _i, _p]),
+    "frt_gemm_plan_info": (_i, [_i, _i, _i, _i, _p, _i]),
     "frt_peak_fp8_mma": (_i, [_i, _i, _p]),
     "frt_peak_copy": (_i, [_p, _p, C.c_size_t, _p]),
 }
@@ -306,6 +307,19 @@ def frt_style_project(rows, K, N, cond, ld_cond, w, ldw, bias, style_out, ld_sty
                                   ptr(style_out), ld_style, ptr(fin_out), ld_fin, fin_col0,
                                   _stream(stream)),
            "frt_style_project")
+
+
+FRT_PLAN_INFO_LEN = 10
+_PLAN_KEYS = ("swap", "pair", "split2", "cluster", "tile_rows", "tile_cols", "splits",
+              "units", "grid", "k_blocks")
+
+
+def frt_gemm_plan_info(M, N, K, epilogue=0) -> dict:
+    """The GEMM schedule the library picks for this shape (host-side)."""
+    buf = (C.c_int * FRT_PLAN_INFO_LEN)()
+    _check(_lib.frt_gemm_plan_info(M, N, K, epilogue, buf, FRT_PLAN_INFO_LEN),
+           "frt_gemm_plan_info")
+    return dict(zip(_PLAN_KEYS, list(buf)))
 
 
 def frt_peak_fp8_mma(ctas: int, iters: int, stream=None) -> None:

@@ -153,6 +153,21 @@ enum { FRT_EPI_BF16 = 0, FRT_EPI_GEGLU_E4M3 = 1, FRT_EPI_GELU_E4M3 = 2 };
 size_t frt_gemm_workspace_size(int M, int N, int K, int epilogue);
 
 /*
+ * The schedule frt_packed_fp8_gemm (and the rope/KV form, which plans like
+ * FRT_EPI_BF16) picks for this shape on the current device (148 SMs when no
+ * device is visible), host-side only, for tests and tuning.  info[0 ..
+ * FRT_PLAN_INFO_LEN - 1] receives: swapped orientation (weights on the MMA M
+ * side), CTA pairs, K in halves over two pairs, K split in a cluster, the
+ * weight (swapped) or activation tile rows, the other tile side, K splits,
+ * work units, grid CTAs, 128-byte K-blocks.  A cluster launch may still use
+ * fewer splits when the device cannot hold every tile's cluster at once.
+ * M == 0 (nothing launched) gives all zeros.  FRT_EINVAL for a short or NULL info or an unknown epilogue, FRT_ESHAPE
+ * for M < 0, N <= 0 or K <= 0.
+ */
+enum { FRT_PLAN_INFO_LEN = 10 };
+int frt_gemm_plan_info(int M, int N, int K, int epilogue, int* info, int n);
+
+/*
  * frt_packed_fp8_gemm (qkv_pack/fp8_static.py `PackedLinear._run`;
  * fp8_chain.py `norm_project` / `down_project`):
  *   acc[m, n] = sum_k x8[m, k] * w8[n, k]            (fp32 accumulate)
