@@ -1691,6 +1691,34 @@ int validate_common(int M, int N, int K, const void* x8, const void* w8, const f
   return FRT_OK;
 }
 
+// Every host-side check of frt_packed_fp8_gemm's arguments (shared with the
+// no-allocation entry, which must reject a call before it touches the GPU).
+int validate_gemm(int M, int N, int K, const void* x8, const void* w8, const float* act_scale,
+                  const float* w_scale, const void* bias, int epilogue, const void* out, long ldo,
+                  const float* out_scale) {
+  int rc = validate_common(M, N, K, x8, w8, act_scale, w_scale);
+  if (rc) return rc;
+  FRT_REQUIRE(epilogue == FRT_EPI_BF16 || epilogue == FRT_EPI_GEGLU_E4M3 ||
+                  epilogue == FRT_EPI_GELU_E4M3,
+              FRT_EINVAL, "unknown epilogue %d", epilogue);
+  FRT_REQUIRE(out, FRT_EINVAL, "out is required");
+  FRT_REQUIRE(!bias || aligned(bias, 16), FRT_EALIGN, "bias must be 16-byte aligned");
+  FRT_REQUIRE(aligned(out, 16), FRT_EALIGN, "out must be 16-byte aligned");
+  if (epilogue == FRT_EPI_BF16) {
+    FRT_REQUIRE(ldo >= N && ldo % 8 == 0, FRT_EALIGN, "ldo must be >= N and a multiple of 8");
+  } else if (epilogue == FRT_EPI_GELU_E4M3) {
+    FRT_REQUIRE(out_scale, FRT_EINVAL, "the GELU epilogue needs out_scale");
+    FRT_REQUIRE(ldo >= N && ldo % 16 == 0, FRT_EALIGN,
+                "ldo must be >= N and a multiple of 16 bytes");
+  } else {
+    FRT_REQUIRE(N % 256 == 0, FRT_ESHAPE, "the GEGLU epilogue needs N %% 256 == 0, got %d", N);
+    FRT_REQUIRE(out_scale, FRT_EINVAL, "the GEGLU epilogue needs out_scale");
+    FRT_REQUIRE(ldo >= N / 2 && ldo % 16 == 0, FRT_EALIGN,
+                "ldo must be >= N/2 and a multiple of 16 bytes");
+  }
+  return FRT_OK;
+}
+
 }  // namespace
 }  // namespace frt
 
@@ -1723,28 +1751,10 @@ extern "C" int frt_packed_fp8_gemm(int M, int N, int K, const frt_e4m3* x8, cons
                                    const frt_bf16* bias, int epilogue, void* out, long ldo,
                                    const float* out_scale, void* workspace,
                                    size_t workspace_bytes, void* stream) {
-  using frt::aligned;
   frt::clear_error();
-  int rc = frt::validate_common(M, N, K, x8, w8, act_scale, w_scale);
+  int rc = frt::validate_gemm(M, N, K, x8, w8, act_scale, w_scale, bias, epilogue, out, ldo,
+                              out_scale);
   if (rc) return rc;
-  FRT_REQUIRE(epilogue == FRT_EPI_BF16 || epilogue == FRT_EPI_GEGLU_E4M3 ||
-                  epilogue == FRT_EPI_GELU_E4M3,
-              FRT_EINVAL, "unknown epilogue %d", epilogue);
-  FRT_REQUIRE(out, FRT_EINVAL, "out is required");
-  FRT_REQUIRE(!bias || aligned(bias, 16), FRT_EALIGN, "bias must be 16-byte aligned");
-  FRT_REQUIRE(aligned(out, 16), FRT_EALIGN, "out must be 16-byte aligned");
-  if (epilogue == FRT_EPI_BF16) {
-    FRT_REQUIRE(ldo >= N && ldo % 8 == 0, FRT_EALIGN, "ldo must be >= N and a multiple of 8");
-  } else if (epilogue == FRT_EPI_GELU_E4M3) {
-    FRT_REQUIRE(out_scale, FRT_EINVAL, "the GELU epilogue needs out_scale");
-    FRT_REQUIRE(ldo >= N && ldo % 16 == 0, FRT_EALIGN,
-                "ldo must be >= N and a multiple of 16 bytes");
-  } else {
-    FRT_REQUIRE(N % 256 == 0, FRT_ESHAPE, "the GEGLU epilogue needs N %% 256 == 0, got %d", N);
-    FRT_REQUIRE(out_scale, FRT_EINVAL, "the GEGLU epilogue needs out_scale");
-    FRT_REQUIRE(ldo >= N / 2 && ldo % 16 == 0, FRT_EALIGN,
-                "ldo must be >= N/2 and a multiple of 16 bytes");
-  }
   if (M == 0) return FRT_OK;
   const int epi = frt::epi_of(epilogue);
   frt::Plan pl = frt::make_plan(M, N, K, epi);
@@ -1839,27 +1849,28 @@ extern "C" int frt_packed_fp8_gemm_noalloc(int M, int N, int K, const frt_e4m3* 
                                            int epilogue, void* out, long ldo,
                                            const float* out_scale, void* stream) {
   frt::clear_error();
-  if (M > 0 && N > 0 && K > 0) {
-    const size_t need = frt_gemm_workspace_size(M, N, K, epilogue);
-    FRT_REQUIRE(need <= frt::kNoAllocScratchBytes, FRT_ERANGE,
-                "this shape needs %zu bytes of split-K workspace; the static scratch of "
-                "frt_packed_fp8_gemm_noalloc holds %zu (use frt_packed_fp8_gemm with a "
-                "caller workspace)",
-                need, frt::kNoAllocScratchBytes);
-    if (need > 0) {
-      void* ws = nullptr;
-      int rc = frt::noalloc_scratch(&ws);
-      if (rc) return rc;
-      // the split counters at the head of the workspace must start at zero;
-      // a completed call leaves them zero, an interrupted one might not
-      const size_t counters = size_t(frt::make_plan(M, N, K, frt::epi_of(epilogue)).counters_bytes);
-      if (counters > 0 &&
-          cudaMemsetAsync(ws, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return frt::fail(FRT_ECUDA, "clearing the static scratch counters");
-      return frt_packed_fp8_gemm(M, N, K, x8, w8, act_scale, w_scale, bias, epilogue, out, ldo,
-                                 out_scale, ws, need, stream);
-    }
-  }
+  // every argument check first: a rejected call must not touch the shared
+  // scratch (another call may be using it on the GPU)
+  int rc = frt::validate_gemm(M, N, K, x8, w8, act_scale, w_scale, bias, epilogue, out, ldo,
+                              out_scale);
+  if (rc) return rc;
+  if (M == 0) return FRT_OK;
+  const frt::Plan pl = frt::make_plan(M, N, K, frt::epi_of(epilogue));
+  FRT_REQUIRE(pl.ws_bytes <= frt::kNoAllocScratchBytes, FRT_ERANGE,
+              "this shape needs %zu bytes of split-K workspace; the static scratch of "
+              "frt_packed_fp8_gemm_noalloc holds %zu (use frt_packed_fp8_gemm with a "
+              "caller workspace)",
+              pl.ws_bytes, frt::kNoAllocScratchBytes);
+  if (pl.ws_bytes == 0)
+    return frt_packed_fp8_gemm(M, N, K, x8, w8, act_scale, w_scale, bias, epilogue, out, ldo,
+                               out_scale, nullptr, 0, stream);
+  void* ws = nullptr;
+  rc = frt::noalloc_scratch(&ws);
+  if (rc) return rc;
+  // the split counters at the head of the workspace must start at zero; a
+  // completed call leaves them zero, an interrupted one might not
+  if (cudaMemsetAsync(ws, 0, pl.counters_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return frt::fail(FRT_ECUDA, "clearing the static scratch counters");
   return frt_packed_fp8_gemm(M, N, K, x8, w8, act_scale, w_scale, bias, epilogue, out, ldo,
-                             out_scale, nullptr, 0, stream);
+                             out_scale, ws, pl.ws_bytes, stream);
 }

@@ -24,7 +24,11 @@ def e4m3_step_distance(a, b):
     same = a == b
     adjacent = (sa == sb) & (np.abs(ma - mb) == 1)
     zero_cross = ((ma == 0) & (mb <= 1)) | ((mb == 0) & (ma <= 1))
-    dist = np.where(same, 0, np.where(adjacent | zero_cross, 1, 2))
+    # 0x7F / 0xFF are e4m3fn's NaN: never one step from a finite code (the
+    # quantizer saturates at +-448, so a NaN is an error, not a rounding)
+    nan = (ma == 0x7F) | (mb == 0x7F)
+    near = (adjacent | zero_cross) & ~nan
+    dist = np.where(same, 0, np.where(near, 1, 2))
     return dist
 
 

@@ -98,6 +98,32 @@ def test_gemm_validation(frt):
     assert frt.frt_gemm_workspace_size(8192, 9216, 3072) == 0
 
 
+def _noalloc(frt, **kw):
+    args = dict(M=200, N=256, K=16384, x8=A16, w8=A16, act_scale=A16,
+                w_scale=A16, bias=None, epilogue=0, out=A16, ldo=256,
+                out_scale=None, stream=None)
+    args.update(kw)
+    return frt.raw_call("frt_packed_fp8_gemm_noalloc", *args.values())
+
+
+def test_noalloc_rejects_before_touching_the_device(frt):
+    """Bad arguments to the no-allocation entry come back with the
+    workspace entry's codes before any CUDA call: with no device here, a
+    call that reached the scratch set-up or its counter memset would report
+    FRT_ECUDA instead.  The shape (200 x 256 x 16384) splits K through the
+    scratch, so a valid call would clear its counters."""
+    assert frt.frt_gemm_workspace_size(200, 256, 16384) > 0
+    assert _noalloc(frt, epilogue=9) == frt.FRT_EINVAL
+    assert _noalloc(frt, out=A16 + 2) == frt.FRT_EALIGN
+    assert _noalloc(frt, ldo=200) == frt.FRT_EALIGN
+    assert _noalloc(frt, bias=A16 + 4) == frt.FRT_EALIGN
+    assert _noalloc(frt, x8=A16 + 8) == frt.FRT_EALIGN
+    assert _noalloc(frt, epilogue=2) == frt.FRT_EINVAL        # no out_scale
+    assert _noalloc(frt, epilogue=1, N=512, ldo=256) == frt.FRT_EINVAL
+    assert _noalloc(frt, K=520) == frt.FRT_ESHAPE
+    assert _noalloc(frt, M=0) == frt.FRT_OK                    # nothing to do
+
+
 def test_rope_and_cache_validation(frt):
     r = frt.raw_call("frt_packed_fp8_gemm_rope_kvcache", 1, 50, 2048, 8, 1,
                      256, 1000, 1024, A16, A16, A16, A16, None, A16, A16,
