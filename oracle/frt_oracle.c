@@ -260,23 +260,14 @@ void or_ada_layer_norm_quant_table(int rows, int D, float eps,
  *      an adjacent-pair rotation carries the host's rotate-half rotation;
  *      sibling 2 (v) keeps host order.  The map is the inverse of the
  *      chain's `kperm` (kperm[2i] = i, kperm[2i+1] = hd/2 + i).
- *   2  gate/up block interleave for two equal siblings of n rows: gate row
- *      j goes to (j / 128) * 256 + j % 128, up row j to that + 128, so one
- *      256-row block holds matching gate and up rows.  (A device layout,
- *      not the pages'; it only reorders the rows the pages concatenate.)
+ * Any other layout value is treated as 0.
  */
-static long pack_dest_row(int layout, int sib, long i, const int *n_i, long base,
-                          int hd)
+static long pack_dest_row(int layout, int sib, long i, long base, int hd)
 {
     if (layout == 1 && (sib == 0 || sib == 1)) {
         long head = i / hd, d = i % hd, half = hd / 2;
         long dst = d < half ? 2 * d : 2 * (d - half) + 1;
         return base + head * hd + dst;
-    }
-    if (layout == 2) {
-        long j = i;
-        (void)n_i;
-        return (j / 128) * 256 + (sib == 1 ? 128 : 0) + (j % 128);
     }
     return base + i;
 }
@@ -298,7 +289,7 @@ void or_pack_weights_fp8(int n_sib, const uint16_t *const *w, const int *n_i,
     long base = 0;
     for (int s = 0; s < n_sib; ++s) {
         for (long i = 0; i < n_i[s]; ++i) {
-            long dst = pack_dest_row(layout, s, i, n_i, base, hd);
+            long dst = pack_dest_row(layout, s, i, base, hd);
             for (int k = 0; k < K; ++k)
                 w8_out[dst * K + k] = q8(or_bf16_to_f32(w[s][i * K + k]), scale);
             if (bias_out)

@@ -181,7 +181,11 @@ def ada_layer_norm_quant_table(x, temb, table, shift_idx, scale_idx,
 
 def pack_weights_fp8(ws, biases=None, layout=0, hd=0):
     """Joint pack of sibling weights (list of [n_i, K] uint16).  Returns
-    dict(w8 [N, K], w_scale float, bias [N] uint16)."""
+    dict(w8 [N, K], w_scale float, bias [N] uint16).  layout 0 stacks the
+    siblings in order (the pages' torch.cat); layout 1 interleaves the q and
+    k rows per head (the chain's `_interleave_rows`)."""
+    if layout not in (0, 1):
+        raise ValueError(f"layout must be 0 (concatenation) or 1 (q/k interleave), got {layout}")
     ws = [_c(w, np.uint16) for w in ws]
     K = ws[0].shape[1]
     n_i = np.array([w.shape[0] for w in ws], dtype=np.int32)

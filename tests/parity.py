@@ -62,3 +62,16 @@ def bf16_ulps(got_bf16, ref_bf16):
     g = np.where(g & 0x8000, -(g & 0x7FFF), g)
     r = np.where(r & 0x8000, -(r & 0x7FFF), r)
     return np.abs(g - r)
+
+
+def gate_up_block_order(H, block=128):
+    """Row order of the library's gate/up block layout as indices into the
+    pages' concatenation [gate; up] (H rows each): packed row r of 256-row
+    block b holds gate row 128b + r for r < 128 and up row 128b + r - 128
+    after it.  Test-side only: the oracle packs in the pages' order and the
+    tests permute its rows to compare with the device layout."""
+    order = np.empty(2 * H, np.int64)
+    for b in range(H // block):
+        order[2 * block * b: 2 * block * b + block] = np.arange(block * b, block * (b + 1))
+        order[2 * block * b + block: 2 * block * (b + 1)] = H + np.arange(block * b, block * (b + 1))
+    return order

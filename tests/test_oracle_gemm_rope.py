@@ -70,18 +70,27 @@ def test_pack_qk_interleave_map(oracle_mod):
     assert np.array_equal(inter["w8"][:4][inv], plain["w8"][:4])
 
 
-def test_pack_gate_up_blocks_and_bias(oracle_mod):
+def test_pack_bias_concat_and_layouts(oracle_mod):
     rng = np.random.default_rng(22)
     g, u = _rand_bf(rng, (256, 16), 0.02), _rand_bf(rng, (256, 16), 0.02)
     bg = _rand_bf(rng, (256,), 0.01)
     plain = oracle_mod.pack_weights_fp8([g, u], [bg, None])
-    blk = oracle_mod.pack_weights_fp8([g, u], [bg, None], layout=2)
-    order = np.concatenate([np.arange(0, 128), np.arange(256, 384),
-                            np.arange(128, 256), np.arange(384, 512)])
-    assert np.array_equal(blk["w8"], plain["w8"][order])
-    assert np.array_equal(blk["bias"], plain["bias"][order])
     assert np.array_equal(plain["bias"][:256], bg)
     assert not plain["bias"][256:].any()
+    # the oracle packs only the pages' two orders (concatenation, q/k
+    # interleave); the library's gate/up block order is a test-side
+    # permutation of the concatenation
+    with pytest.raises(ValueError):
+        oracle_mod.pack_weights_fp8([g, u], layout=2)
+
+
+def test_gate_up_block_order_by_enumeration():
+    from parity import gate_up_block_order
+    o = gate_up_block_order(256)
+    want = list(range(0, 128)) + list(range(256, 384)) + \
+        list(range(128, 256)) + list(range(384, 512))
+    assert o.tolist() == want
+    assert sorted(gate_up_block_order(1024).tolist()) == list(range(2048))
 
 
 # ---------------------------------------------------------------- gemm ----
