@@ -1,24 +1,30 @@
 """Benchmark of the fused static-FP8 attention-input chain on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
-                    [--impl reference]
+                    [--impl reference] [--repeats R] [--no-subconfigs]
 
 One step = one pass of the chain over one batch of the workload, all inputs
-resident in HBM: for the default workload (the VLA action-expert layer: 50
-tokens behind an 816-token prefix, D=2048, 8 q heads + 1 kv head of 256,
-packed N=2560) that is the prefix copy into the layer's caches, the AdaRMS
-producer and the packed FP8 q/k/v GEMM with the split + RoPE + KV write in
-its epilogue: the three launches frt_chain_layer makes.  Other workloads
-(--config): tiny_adarms, video_dit, gateup_mlp, adarms_stack18[:M].
+resident in HBM.  The default workload is the video-DiT block form (B=2 x
+4096 tokens, D=3072, the per-token-table LayerNorm producer, the packed
+q/k/v FP8 GEMM (N=9216, bias) with the split + RoPE + KV write in its
+epilogue): the two launches frt_chain_layer makes.  The same JSON line
+carries one record per other configuration under "configs": the tiny
+AdaRMS layer, the action-expert layer (50 tokens behind an 816-token
+prefix), the gate/up MLP (producer, gate/up GEMM with the GEGLU requant,
+down GEMM) and the 18-layer AdaRMS stack at every row count of its sweep.
+Other workloads (--config): video_dit_ffn, adarms_layer18[_live],
+style_stack18, style_vla18, adarms_stack18:M.
 
-Timing: W untimed warm-up steps, then K timed steps.  Before every timed step
-the L2 is flushed (a 256 MB write) and the GPU is held by a short spin so the
-host has enqueued the whole step before its first event; each kernel is
-bracketed by CUDA events on the launching stream.  The JSON line reports the
-device time; `e2e` repeats the step through frt_chain_layer with pinned host
-inputs copied in and the outputs copied back inside the timed region.
-With N > 1 (torchrun) every rank runs an independent replica on its own
-batch (no data-path collective); value = all ranks' tokens / max rank time.
+Timing: W untimed warm-up steps, then R timed regions of exactly K steps,
+each bracketed by a barrier and a synchronize, K steps replayed back to
+back from CUDA graphs over independent copies of the workload (inputs
+larger than L2), CUDA events on the launching stream, max over ranks; the
+value comes from the median region, the spread is reported.  Each kernel is
+timed alone the same way.  `e2e` runs the step through the entry points
+with pinned host buffers copied in and the outputs copied back, timed on
+the host clock per step.  With N > 1 (torchrun) every rank runs an
+independent replica on its own batch (no data-path collective); value =
+all ranks' tokens / max rank time.
 
 --impl reference times the CPU oracle (the reference arm: plain C, OpenMP
 over rows) on the host cores on the same workload.
@@ -41,7 +47,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = ("chain tokens/s & µs/layer; GEMM % FP8 tensor peak, "
           "producer % HBM GB/s")
-DEFAULT_CONFIG = "vla_action_expert"
+DEFAULT_CONFIG = "video_dit"
 FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -436,6 +442,37 @@ class ChainRunner:
                    lambda: self._producer(0, self.act[0])))
         kc.append((by["gemm_rope_kv"], lambda: self._gemm(0, self.act[0])))
         return kc
+
+    def aux_calls(self):
+        """Kernels timed beside the step (not part of it), video-DiT form:
+        the standalone split + RoPE + KV write on a bf16 q/k/v buffer (the
+        unfused page form; HBM-bound, rows * (4N + 2hd) bytes per launch) and
+        the same GEMM with the plain bf16 epilogue (its time against the
+        fused one prices the split/RoPE/KV epilogue)."""
+        if not self.dit:
+            return []
+        frt, w, lay = self.frt, self.w, self.layers[0]
+        N = w.N
+        if not hasattr(self, "qkv_bf16"):
+            self.qkv_bf16 = self.rt.empty_bf16(self.rows, N)
+            frt.frt_packed_fp8_gemm(self.rows, N, w.D, self.x8, lay["pk"].w8, self.act[0],
+                                    lay["pk"].w_scale, lay["pk"].bias, frt.FRT_EPI_BF16,
+                                    self.qkv_bf16, N, None, self.ws, self.ws_bytes)
+
+        def split():
+            frt.frt_split_rope_kvcache(w.B, w.M, w.hq, w.hkv, w.hd, w.P, w.T, self.qkv_bf16,
+                                       self.rope, self.q[0], lay["kc"], lay["vc"])
+
+        def gemm_plain():
+            frt.frt_packed_fp8_gemm(self.rows, N, w.D, self.x8, lay["pk"].w8, self.act[0],
+                                    lay["pk"].w_scale, lay["pk"].bias, frt.FRT_EPI_BF16,
+                                    self.qkv_bf16, N, None, self.ws, self.ws_bytes)
+        rows = self.rows
+        return [
+            (Kern("split_rope_kv", "hbm", rows * (4.0 * N + 2 * w.hd)), split),
+            (Kern("gemm_bf16", "tensor", N * w.D + rows * w.D + rows * N * 2 + N * 2,
+                  2.0 * rows * N * w.D), gemm_plain),
+        ]
 
     # ---------------------------------------------------------------- e2e --
     def e2e_setup(self):
@@ -1014,7 +1051,7 @@ def oracle_sampler(name, synth, rows_cap=None):
         w = w.with_M(int(m))
     rng = np.random.default_rng(7)
     if w.kind == "mlp":
-        n = rows_cap or 32
+        n = rows_cap or 256
         sel = np.sort(rng.choice(w.M, size=min(n, w.M), replace=False))
         mw = synth.mlp_weights(w.D, w.H, w.seed)
         gu_p = oracle.pack_weights_fp8([mw["gate"], mw["up"]])
@@ -1262,52 +1299,53 @@ def _smallest_divisor_at_least(K, r):
     return K
 
 
-def run_gpu(args):
-    import torch
-    import torch.distributed as dist
+SUB_CONFIGS = ("tiny_adarms", "vla_action_expert", "gateup_mlp") + tuple(
+    f"adarms_stack18:{m}" for m in (1, 16, 50, 256, 1024, 4096))
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=dev)
-    from fp8_transformer_block_b200 import build
-    if rank == 0 or world == 1:
-        build.build()
-    if world > 1:
-        dist.barrier()
-    from fp8_transformer_block_b200 import frt, synth
-    from fp8_transformer_block_b200 import runtime as rt
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+class GpuEnv:
+    """What every measurement of one run shares: torch, the process group,
+    the binding, the L2 flush buffer and the peaks."""
 
-    # ---- R independent copies of the workload (weights, inputs, caches), so
-    # that consecutive steps read data no earlier step left in L2: the
-    # copies together exceed 1.5x the L2 (or one copy already does)
-    first = make_runner(args.config, torch, frt, rt, synth)
-    w = first.w
-    L = getattr(first, "L", 1)
-    fp = _footprint(first, torch)
-    K = args.steps
-    r_min = 1 if fp >= 1.5 * L2_BYTES else -(-int(1.5 * L2_BYTES) // fp)
-    R = _smallest_divisor_at_least(K, min(r_min, K))
-    runners = [first] + [make_runner(args.config, torch, frt, rt, synth)
-                         for _ in range(R - 1)]
-    torch.cuda.synchronize()
-    for _ in range(args.warmup):
-        for r in runners:
-            r.step()
-    torch.cuda.synchronize()
-    assert frt.frt_device_status(True) == frt.FRT_OK
+    def __init__(self, args):
+        import torch
+        import torch.distributed as dist
+        self.torch, self.dist, self.args = torch, dist, args
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        self.dev = torch.device("cuda", local)
+        if self.world > 1:
+            from datetime import timedelta
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                    device_id=self.dev)
+        from fp8_transformer_block_b200 import build
+        if self.rank == 0 or self.world == 1:
+            build.build()
+        self.barrier()
+        from fp8_transformer_block_b200 import frt, synth
+        from fp8_transformer_block_b200 import runtime as rt
+        self.frt, self.synth, self.rt = frt, synth, rt
+        self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=self.dev)
+        self.gpu_id = None
+        try:
+            self.gpu_id = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
+        except Exception:  # noqa: BLE001
+            pass
+        self.peaks = _peaks()
+        self.own = None
 
-    def capture(calls):
-        cap = torch.cuda.Stream(device=dev)
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max_ms(self, ms):
+        return max_over_ranks(ms, self.torch, self.dist, self.world, self.dev)
+
+    def capture(self, calls):
+        torch = self.torch
+        cap = torch.cuda.Stream(device=self.dev)
         cap.wait_stream(torch.cuda.current_stream())
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap):
@@ -1316,65 +1354,112 @@ def run_gpu(args):
         torch.cuda.current_stream().wait_stream(cap)
         return g
 
-    g_steps = capture([r.step for r in runners])
+
+def _kern_entry(ms, k, hbm, fp8_peak, own):
+    e = {"kernel": k.name, "us": round(ms * 1e3, 3),
+         "launches_per_step": k.per_step, "bound": k.bound,
+         "algo_bytes": int(k.algo_bytes),
+         "GB_s": round(k.algo_bytes / (ms * 1e-3) / 1e9, 1),
+         "hbm_frac": round(k.algo_bytes / (ms * 1e-3) / 1e9 / hbm, 4)}
+    if k.flops:
+        e["TFLOP_s"] = round(k.flops / (ms * 1e-3) / 1e12, 2)
+        e["fp8_frac"] = round(e["TFLOP_s"] / fp8_peak, 4)
+        e["fp8_frac_own"] = round(e["TFLOP_s"] / own["fp8_dense_tflops"], 4)
+    e["hbm_frac_own"] = round(e["GB_s"] / own["hbm_copy_gbs"], 4)
+    return e
+
+
+def measure(env, name, n_rep, cpu_seconds):
+    """One workload: R independent copies stepped in rotation (inputs larger
+    than L2), n_rep timed regions of exactly K steps each (CUDA events on
+    the launching stream around K steps replayed from CUDA graphs, a barrier
+    and a synchronize on both sides, max over ranks), each kernel alone the
+    same way, an isolated step after an L2 flush, the end-to-end step with
+    host buffers on the host clock, and the oracle on the host cores."""
+    torch, frt, args = env.torch, env.frt, env.args
+    first = make_runner(name, torch, frt, env.rt, env.synth)
+    w = first.w
+    L = getattr(first, "L", 1)
+    fp = _footprint(first, torch)
+    K = args.steps
+    r_min = 1 if fp >= 1.5 * L2_BYTES else -(-int(1.5 * L2_BYTES) // fp)
+    R = _smallest_divisor_at_least(K, min(r_min, K))
+    runners = [first] + [make_runner(name, torch, frt, env.rt, env.synth)
+                         for _ in range(R - 1)]
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        for r in runners:
+            r.step()
+    torch.cuda.synchronize()
+    assert frt.frt_device_status(True) == frt.FRT_OK
+    g_steps = env.capture([r.step for r in runners])
     for _ in range(2):
         g_steps.replay()
     torch.cuda.synchronize()
     assert frt.frt_device_status(True) == frt.FRT_OK
 
     mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    gpu_id = None
-    try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:  # noqa: BLE001
-        pass
-    clocks = ClockSampler(gpu_id)
     reps = K // R
-    e0, e1 = mk(), mk()
-    barrier()
+    clocks = ClockSampler(env.gpu_id)
+    region_ms = []
+    env.barrier()
     torch.cuda.synchronize()
     clocks.start()
     t_wall = time.perf_counter()
-    torch.cuda._sleep(2_000_000)   # hold the GPU while the replays queue
-    torch.cuda.nvtx.range_push("timed_steps")
-    e0.record()
-    for _ in range(reps):
-        g_steps.replay()
-    e1.record()
-    torch.cuda.nvtx.range_pop()
-    torch.cuda.synchronize()
-    barrier()
+    for _ in range(n_rep):
+        e0, e1 = mk(), mk()
+        env.barrier()
+        torch.cuda.synchronize()
+        torch.cuda._sleep(2_000_000)   # hold the GPU while the replays queue
+        torch.cuda.nvtx.range_push("timed_steps")
+        e0.record()
+        for _ in range(reps):
+            g_steps.replay()
+        e1.record()
+        torch.cuda.nvtx.range_pop()
+        torch.cuda.synchronize()
+        env.barrier()
+        region_ms.append(env.max_ms(e0.elapsed_time(e1)))
     wall = time.perf_counter() - t_wall
     clk = clocks.stop()
     assert frt.frt_device_status(True) == frt.FRT_OK
-    max_total_ms = max_over_ranks(e0.elapsed_time(e1), torch, dist, world, dev)
-    ms_per_step = max_total_ms / K
-    value = job_throughput(first.tokens, K, max_total_ms, world)
+    med_ms = statistics.median(region_ms)
+    ms_per_step = med_ms / K
+    value = job_throughput(first.tokens, K, med_ms, env.world)
 
-    # ---- each kernel alone, back to back over the same R copies
-    kinds, kern_ms = [], []
-    for kk in range(len(first.kernel_calls())):
-        calls = [r.kernel_calls()[kk][1] for r in runners]
-        kinds.append(first.kernel_calls()[kk][0])
-        gk = capture(calls)
+    # ---- each kernel alone (and the aux kernels), back to back over the R copies
+    def time_alone(calls, label):
+        gk = env.capture(calls)
         gk.replay()
         torch.cuda.synchronize()
         a, b = mk(), mk()
         torch.cuda._sleep(2_000_000)
-        torch.cuda.nvtx.range_push(f"kernel_{kinds[-1].name}")
+        torch.cuda.nvtx.range_push(f"kernel_{label}")
         a.record()
         for _ in range(reps):
             gk.replay()
         b.record()
         torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
-        kern_ms.append(a.elapsed_time(b) / (reps * R))
-        del gk
+        return env.max_ms(a.elapsed_time(b)) / (reps * R)
+
+    kinds, kern_ms = [], []
+    for kk in range(len(first.kernel_calls())):
+        kinds.append(first.kernel_calls()[kk][0])
+        kern_ms.append(time_alone([r.kernel_calls()[kk][1] for r in runners],
+                                  kinds[-1].name))
+    aux = []
+    if hasattr(first, "aux_calls"):
+        n_aux = len(first.aux_calls())
+        for kk in range(n_aux):
+            k = first.aux_calls()[kk][0]
+            aux.append((k, time_alone([r.aux_calls()[kk][1] for r in runners], k.name)))
+    assert frt.frt_device_status(True) == frt.FRT_OK
 
     # ---- one step per event pair after an L2 flush: the latency of an
     # isolated step as a stream sees it (event and launch costs included)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    g_one = capture([first.step])
+    flush = env.flush
+    g_one = env.capture([first.step])
     n_iso = min(K, 100)
     iso = [(mk(), mk()) for _ in range(n_iso)]
     for i in range(n_iso):
@@ -1387,14 +1472,30 @@ def run_gpu(args):
     iso_us = 1e3 * sum(a.elapsed_time(b) for a, b in iso) / n_iso
     del g_one, g_steps
 
-    # ---- e2e through the public entry points with host buffers
+    # ---- e2e through the public entry points with host buffers: every
+    # step copies its inputs in from pinned host memory, runs, and reads its
+    # outputs back; timed on the host clock from the first call to the
+    # synchronize after the read-back (host-side launch and marshalling
+    # included), after an L2 flush that has completed
     first.e2e_setup()
     for _ in range(3):
         first.e2e_step()
     torch.cuda.synchronize()
-    KE = min(K, 200)
+    KE = min(K, 100)
+    host_s = 0.0
+    env.barrier()
+    for i in range(KE):
+        flush.fill_(i & 0xFF)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        first.e2e_step()
+        torch.cuda.synchronize()
+        host_s += time.perf_counter() - t0
+    e_ms = env.max_ms(1e3 * host_s)
+    e2e_value = job_throughput(first.tokens, KE, e_ms, env.world)
+    # the same steps' device time alone (the GPU held by a spin while the
+    # host enqueues, so host-side costs are not in it)
     e_ev = [(mk(), mk()) for _ in range(KE)]
-    barrier()
     for i in range(KE):
         flush.fill_(i & 0xFF)
         torch.cuda._sleep(1_000_000)
@@ -1402,89 +1503,133 @@ def run_gpu(args):
         first.e2e_step()
         e_ev[i][1].record()
     torch.cuda.synchronize()
-    e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), torch, dist, world, dev)
-    e2e_value = job_throughput(first.tokens, KE, e_ms, world)
+    ed_ms = env.max_ms(sum(a.elapsed_time(b) for a, b in e_ev))
+    assert frt.frt_device_status(True) == frt.FRT_OK
 
     # ---- roofline of the dominant kernel (largest share of a step)
-    hbm, bf16_burst, bf16_sust, src = _peaks()
+    hbm, bf16_burst, _, src = env.peaks
+    fp8_peak = bf16_burst * FP8_PER_BF16
+    own = env.own
     shares = [ms * k.per_step for ms, k in zip(kern_ms, kinds)]
     dom = int(np.argmax(shares))
     kd = kinds[dom]
     if kd.bound == "tensor":
         achieved = kd.flops / (kern_ms[dom] * 1e-3) / 1e12
-        peak = bf16_burst * FP8_PER_BF16
-        unit = "TFLOP/s"
+        peak, unit, peak_own = fp8_peak, "TFLOP/s", own["fp8_dense_tflops"]
     else:
         achieved = kd.algo_bytes / (kern_ms[dom] * 1e-3) / 1e9
-        peak = hbm
-        unit = "GB/s"
-    tr = NCU_TRAFFIC.get((args.config, kd.name))
+        peak, unit, peak_own = hbm, "GB/s", own["hbm_copy_gbs"]
+    base = name.partition(":")[0]
+    tr = NCU_TRAFFIC.get((name, kd.name)) or NCU_TRAFFIC.get((base, kd.name))
     traffic = tr[0] if tr and tr[1] == _src_hash(kd.name) else None
-    own = own_peaks(torch, frt)
-    kern_list = []
-    for ms, k in zip(kern_ms, kinds):
-        e = {"kernel": k.name, "us": round(ms * 1e3, 3),
-             "launches_per_step": k.per_step, "bound": k.bound,
-             "algo_bytes": int(k.algo_bytes),
-             "GB_s": round(k.algo_bytes / (ms * 1e-3) / 1e9, 1),
-             "hbm_frac": round(k.algo_bytes / (ms * 1e-3) / 1e9 / hbm, 4)}
-        if k.flops:
-            e["TFLOP_s"] = round(k.flops / (ms * 1e-3) / 1e12, 2)
-            e["fp8_frac"] = round(k.flops / (ms * 1e-3) / 1e12 /
-                                  (bf16_burst * FP8_PER_BF16), 4)
-            e["fp8_frac_own"] = round(e["TFLOP_s"] / own["fp8_dense_tflops"], 4)
-        e["hbm_frac_own"] = round(e["GB_s"] / own["hbm_copy_gbs"], 4)
-        kern_list.append(e)
+    roof = {"bound": kd.bound, "kernel": kd.name, "achieved": achieved,
+            "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": traffic,
+            "peak_source": f"{src} " + ("(bf16 burst x 2, nominal fp8/bf16 ratio)"
+                                        if unit == "TFLOP/s" else "(HBM copy)"),
+            "algo_per_launch": kd.flops if unit == "TFLOP/s" else kd.algo_bytes,
+            "peak_own": peak_own, "frac_own": achieved / peak_own,
+            "peak_own_source": ("the library's own tcgen05 e4m3 MMA loop" if unit == "TFLOP/s"
+                                else "the library's own device copy")}
+    if unit == "TFLOP/s":
+        roof["fp8_frac_own"] = roof["frac_own"]
+    kern_list = [_kern_entry(ms, k, hbm, fp8_peak, own) for ms, k in zip(kern_ms, kinds)]
+    aux_list = [_kern_entry(ms, k, hbm, fp8_peak, own) for k, ms in aux]
+    if aux:
+        by = {e["kernel"]: e for e in aux_list}
+        if "gemm_bf16" in by and kd.name == "gemm_rope_kv":
+            by["gemm_bf16"]["fused_epilogue_cost_us"] = round(
+                kern_ms[dom] * 1e3 - by["gemm_bf16"]["us"], 3)
 
-    if rank != 0:
-        if world > 1:
-            dist.destroy_process_group()
-        return 0
     cpu = None
-    if world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(args.config, synth, seconds=args.cpu_seconds)
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "us_per_layer": 1e3 * ms_per_step / L,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": getattr(first, "dtype", "e4m3/fp32"), "data": "synthetic",
-        "config": {"workload": workload_text(w),
-                   "l2": (f"inputs larger than L2: {R} independent copies of "
-                          f"the workload ({R * fp / 2**20:.0f} MiB) rotated "
-                          "step by step" if R > 1 else
-                          f"inputs larger than L2 ({fp / 2**20:.0f} MiB per "
-                          "step)"),
-                   "parallelism": "replicas" if world > 1 else "single",
-                   "timing": "K back-to-back steps replayed from CUDA graphs, "
-                             "CUDA events around the K steps on the launching "
-                             "stream; kernels timed the same way",
-                   "isolated_step_us_after_l2_flush": round(iso_us, 3),
-                   "e2e_scope": "each step copies the tokens' input rows in from pinned "
-                                "host memory and reads its output rows (and new K/V rows) "
-                                "back; weights, tables and the prefix K/V cache (the host "
-                                "model's device-resident cache) stay in device memory"},
-        "roofline": {"bound": kd.bound, "kernel": kd.name,
-                     "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"{src} "
-                     + ("(bf16 burst x 2, nominal fp8/bf16 ratio)"
-                        if unit == "TFLOP/s" else "(HBM copy)"),
-                     "algo_per_launch": kd.flops if unit == "TFLOP/s"
-                     else kd.algo_bytes},
-        "kernels": kern_list,
-        "peaks_own": own,
+    if env.rank == 0 and env.world == 1 and not args.no_cpu and cpu_seconds > 0:
+        cpu = cpu_baseline(name, env.synth, seconds=cpu_seconds)
+    rec = {
+        "workload": workload_text(w), "value": value, "unit": "tokens/s",
+        "steps": K, "ms_per_step": ms_per_step, "us_per_layer": 1e3 * ms_per_step / L,
+        "timed_regions": {"n": n_rep, "steps_each": K,
+                          "ms_per_step": [round(m / K, 6) for m in region_ms],
+                          "median": round(ms_per_step, 6),
+                          "min": round(min(region_ms) / K, 6),
+                          "max": round(max(region_ms) / K, 6),
+                          "spread": round((max(region_ms) - min(region_ms)) / med_ms, 4)},
+        "dtype": getattr(first, "dtype", "e4m3/fp32"),
+        "l2": (f"inputs larger than L2: {R} independent copies of the workload "
+               f"({R * fp / 2**20:.0f} MiB) rotated step by step" if R > 1 else
+               f"inputs larger than L2 ({fp / 2**20:.0f} MiB per step)"),
+        "isolated_step_us_after_l2_flush": round(iso_us, 3),
+        "roofline": roof, "kernels": kern_list,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": int(first.h2d_bytes),
-                "d2h_bytes_per_step": int(first.d2h_bytes)},
-        "gpu_launches": first.launches * K,
-        "clocks": clk,
-        "wall_s_timed_loop": round(wall, 3),
+                "d2h_bytes_per_step": int(first.d2h_bytes),
+                "clock": "host (perf_counter), call to synchronize, per step",
+                "us_per_step": round(1e3 * e_ms / KE, 3), "steps": KE},
+        "e2e_device": {"value": job_throughput(first.tokens, KE, ed_ms, env.world),
+                       "unit": "tokens/s", "us_per_step": round(1e3 * ed_ms / KE, 3),
+                       "clock": "CUDA events around each step, GPU held while it queued"},
+        "gpu_launches": first.launches * K * n_rep,
+        "gpu_launches_per_region": first.launches * K,
+        "clocks": clk, "wall_s_timed_loop": round(wall, 3),
     }
+    if aux_list:
+        rec["aux_kernels"] = aux_list
+    for r in runners:
+        for attr in list(vars(r)):
+            setattr(r, attr, None)
+    del runners, first
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_gpu(args):
+    env = GpuEnv(args)
+    torch = env.torch
+    env.own = own_peaks(torch, env.frt)
+    main_rec = measure(env, args.config, args.repeats, args.cpu_seconds)
+    subs = {}
+    if args.config == DEFAULT_CONFIG and not args.no_subconfigs:
+        for name in SUB_CONFIGS:
+            subs[name] = measure(env, name, 3, args.cpu_seconds_sub)
+    if env.rank != 0:
+        if env.world > 1:
+            env.dist.destroy_process_group()
+        return 0
+    line = {
+        "metric": METRIC, "value": main_rec["value"], "unit": "tokens/s",
+        "n_gpus": env.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": main_rec["ms_per_step"], "us_per_layer": main_rec["us_per_layer"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": main_rec["dtype"], "data": "synthetic",
+        "config": {"workload": main_rec["workload"], "l2": main_rec["l2"],
+                   "parallelism": "replicas" if env.world > 1 else "single",
+                   "timing": (f"{args.repeats} timed regions of exactly K steps each "
+                              "(K back-to-back steps replayed from CUDA graphs, CUDA "
+                              "events on the launching stream, barrier + synchronize "
+                              "on both sides, max over ranks); value from the median "
+                              "region; kernels timed the same way"),
+                   "isolated_step_us_after_l2_flush":
+                       main_rec["isolated_step_us_after_l2_flush"],
+                   "e2e_scope": "each step copies the tokens' input rows in from pinned "
+                                "host memory and reads its output rows (and new K/V rows) "
+                                "back; weights, tables and the prefix K/V cache (the host "
+                                "model's device-resident cache) stay in device memory; "
+                                "timed on the host clock"},
+        "timed_regions": main_rec["timed_regions"],
+        "roofline": main_rec["roofline"], "kernels": main_rec["kernels"],
+        "peaks_own": env.own, "cpu_baseline": main_rec["cpu_baseline"],
+        "e2e": main_rec["e2e"], "e2e_device": main_rec["e2e_device"],
+        "gpu_launches": main_rec["gpu_launches"],
+        "gpu_launches_per_region": main_rec["gpu_launches_per_region"],
+        "clocks": main_rec["clocks"], "wall_s_timed_loop": main_rec["wall_s_timed_loop"],
+    }
+    if "aux_kernels" in main_rec:
+        line["aux_kernels"] = main_rec["aux_kernels"]
+    if subs:
+        line["configs"] = subs
     print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    if env.world > 1:
+        env.dist.destroy_process_group()
     return 0
 
 
@@ -1497,6 +1642,12 @@ def main():
     ap.add_argument("--impl", default="frt", choices=["frt", "reference"])
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds-sub", type=float, default=3.0,
+                    help="oracle seconds per sub-configuration record")
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="timed regions of K steps for the main line (median reported)")
+    ap.add_argument("--no-subconfigs", action="store_true",
+                    help="only the selected workload (no per-configuration records)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -288,6 +288,8 @@ void or_pack_weights_fp8(int n_sib, const uint16_t *const *w, const int *n_i,
     *w_scale_out = scale;
     long base = 0;
     for (int s = 0; s < n_sib; ++s) {
+        /* rows are quantized independently (one shared scale) */
+        #pragma omp parallel for schedule(static)
         for (long i = 0; i < n_i[s]; ++i) {
             long dst = pack_dest_row(layout, s, i, base, hd);
             for (int k = 0; k < K; ++k)
