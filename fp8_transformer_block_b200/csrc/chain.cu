@@ -11,8 +11,8 @@
 // programmatic dependent launch (each starts while its predecessor drains):
 //   FRT_CHAIN_FUSED_ROPE: producer (its extra blocks copy the prefix) ->
 //     packed GEMM with the split + RoPE + KV write in its epilogue;
-//   FRT_CHAIN_UNFUSED: producer -> packed GEMM -> qkv -> split kernel that
-//     also copies the prefix.
+//   FRT_CHAIN_UNFUSED: producer -> packed GEMM -> qkv -> prefix copy (when
+//     there is a prefix) -> split kernel.
 #include "frt_internal.cuh"
 
 extern "C" size_t frt_chain_workspace_size(const frt_chain_desc* d) {

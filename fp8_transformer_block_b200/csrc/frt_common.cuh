@@ -168,6 +168,24 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&f)[8]) {
                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
 }
 
+// Adjacent-pair rotation of 8 bf16 values x (4 pairs) with 4 (cos, sin)
+// pairs r (the rope table's interleaved layout): (x0, x1) -> (x0*c - x1*s,
+// x0*s + x1*c) in fp32, each product and sum rounded once, then bf16.  The
+// fused GEMM epilogue and the standalone split kernel both use this, so
+// their results agree bit for bit.
+__device__ __forceinline__ uint4 rope_rotate8(const uint4& xv, const uint4& rv) {
+  float x[8], r[8], o[8];
+  unpack8(xv, x);
+  unpack8(rv, r);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const float x0 = x[2 * p], x1 = x[2 * p + 1], c = r[2 * p], s = r[2 * p + 1];
+    o[2 * p] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, s));
+    o[2 * p + 1] = __fadd_rn(__fmul_rn(x0, s), __fmul_rn(x1, c));
+  }
+  return pack8_bf16(o);
+}
+
 // 8 floats already divided by the scale -> 8 e4m3 codes in a uint2.
 __device__ __forceinline__ uint2 pack8_e4m3(const float (&q)[8]) {
   uint32_t lo = pack_e4m3x2(q[0], q[1]) | (uint32_t(pack_e4m3x2(q[2], q[3])) << 16);

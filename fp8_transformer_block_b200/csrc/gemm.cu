@@ -39,6 +39,8 @@ namespace {
 constexpr int BM = 128;             // MMA M of the normal orientation
 constexpr int BK = 128;             // K bytes per stage: one swizzle row
 constexpr int kThreads = 192;
+constexpr int kPairEpiWarps = 8;    // CTA-pair kernel: two epilogue warps per TMEM lane quarter
+constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
 constexpr int kMaxCluster = 8;      // portable thread-block cluster size
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per wait
 constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s to drain after an abort
@@ -81,29 +83,8 @@ __device__ __forceinline__ void record_timeout(int* status) {
 
 // ---------------------------------------------------------------- epilogue --
 
-// y = bf16(acc * alpha [+ bias]) as a float (the value the unfused path
-// stores and the split kernel reads back).
-__device__ __forceinline__ float scale_bias_bf16(float acc, float alpha, const uint16_t* bias,
-                                                 int n) {
-  float y = __fmul_rn(acc, alpha);
-  if (bias) y = __fadd_rn(y, bf2f(__ldg(bias + n)));
-  return bf2f(f2bf(y));
-}
-
-// 32 consecutive bf16 starting at a 64-byte aligned address -> floats.
-__device__ __forceinline__ void load32_bf16(const uint16_t* src, float (&f)[32]) {
-  const uint4* s4 = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    float t[8];
-    unpack8(__ldg(s4 + k), t);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) f[8 * k + j] = t[j];
-  }
-}
-
 // One token row m, output columns n0 .. n0 + W - 1 (W = 8 or 16, n0 % W == 0,
-// inside one head): the same arithmetic as epi_rows_chunk at 16-byte
+// inside one head): the same arithmetic as warp_rows_epilogue at 16-byte
 // granularity, in two steps.  item_plan works out, ahead of the
 // accumulators, where each 8-column piece goes and loads the rope and bias
 // pieces it needs; item_apply then only scales, adds, rotates and stores
@@ -176,98 +157,230 @@ __device__ __forceinline__ void item_apply(const GemmParams& p, const float (&v)
   }
 }
 
-// This thread owns token row m, output columns n0 .. n0 + 31 (the normal
-// orientation, and the swapped one after the shared-memory transpose).
-__device__ __forceinline__ void epi_rows_chunk(const GemmParams& p, const float (&v)[32], int m,
-                                               int n0, float alpha) {
-  if (m >= p.M) return;
-  float y[32];
-  if (p.bias) {
-    float b[32];
-    load32_bf16(p.bias + n0, b);
+// ------------------------------------------------- staged row epilogue --
+//
+// The normal orientation leaves accumulator row m_base + lane of a warp's 32
+// rows in each thread.  Written straight from registers, every store
+// instruction of the warp would touch 32 rows (32 cache lines for 16 bytes
+// each), which made the output path slower than the main loop.  Instead each
+// warp stages 32 rows x 128 bytes of finished output in its own 4 KB of
+// shared memory (16-byte units swizzled by row, so both the row-wise writes
+// and the column-wise reads are conflict-free) and writes them back as whole
+// 128-byte row segments: eight threads per row, four rows per store.  The
+// RoPE rotation runs in that write-back, on the staged bf16 values (the
+// unfused form rotates the same bf16-rounded values), so the rope-table
+// loads are row segments too.
+constexpr int kEpiStageBytes = 32 * 128;   // one warp's staging buffer
+
+__device__ __forceinline__ void stage_put(uint8_t* buf, int row, int unit, const uint4& v) {
+  *reinterpret_cast<uint4*>(buf + row * 128 + ((unit ^ (row & 7)) << 4)) = v;
+}
+__device__ __forceinline__ uint4 stage_get(const uint8_t* buf, int row, int unit) {
+  return *reinterpret_cast<const uint4*>(buf + row * 128 + ((unit ^ (row & 7)) << 4));
+}
+
+// Write-back of the staged bf16 rows of one 64-column group.  Thread (row
+// r = lane/8 + 4i, unit u = lane % 8) writes output columns n0 + 8u .. +7 of
+// token row m_base + r; with the RoPE epilogue q and k heads are rotated
+// with the table row of their position and q / k / v go to their buffers
+// (the 8 columns of a unit lie inside one head: hd % 8 == 0).  The rope
+// rows are requested (rope_rows) before the group's accumulators are read,
+// so those loads overlap the TMEM loads and the arithmetic.
+__device__ __forceinline__ void rope_rows(const GemmParams& p, int lane, int m_base, int n0,
+                                          uint4 (&rv)[8]) {
+  const int n = n0 + 8 * (lane & 7);
+  const int h = n / p.hd, d0 = n - h * p.hd;
+  if (p.epi != EPI_ROPE || n >= p.N || h >= p.hq + p.hkv) return;
+  const int m0 = m_base + (lane >> 3);
+  int b = m0 / p.Mseq, s = m0 - b * p.Mseq;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) y[j] = bf2f(f2bf(__fadd_rn(__fmul_rn(v[j], alpha), b[j])));
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) y[j] = bf2f(f2bf(__fmul_rn(v[j], alpha)));
+  for (int i = 0; i < 8; ++i) {
+    if (m0 + 4 * i < p.M)
+      rv[i] = __ldg(reinterpret_cast<const uint4*>(p.rope + long(s) * p.hd + d0));
+    s += 4;
+    while (s >= p.Mseq) { s -= p.Mseq; ++b; }
   }
-  uint16_t* dst;
-  if (p.epi == EPI_BF16) {
-    dst = static_cast<uint16_t*>(p.out) + long(m) * p.ldo + n0;
-  } else {  // EPI_ROPE: the 32 columns lie inside one head (hd % 32 == 0)
-    const int b = m / p.Mseq, s = m % p.Mseq;
-    const int h = n0 / p.hd, d0 = n0 % p.hd;
-    if (h < p.hq + p.hkv) {
-      float r[32];
-      load32_bf16(p.rope + long(s) * p.hd + d0, r);
+}
+
+__device__ __forceinline__ void flush_rows_bf16(const GemmParams& p, const uint8_t* buf, int lane,
+                                                int m_base, int n0, int units,
+                                                const uint4 (&rv)[8]) {
+  __syncwarp();
+  const int u = lane & 7, r0 = lane >> 3;
+  const int n = n0 + 8 * u;
+  if (u < units && n < p.N) {
+    const int m0 = m_base + r0;
+    if (p.epi == EPI_BF16) {
+      uint16_t* base = static_cast<uint16_t*>(p.out) + n;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float c = r[2 * i], sn = r[2 * i + 1];
-        const float x0 = y[2 * i], x1 = y[2 * i + 1];
-        y[2 * i] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, sn));
-        y[2 * i + 1] = __fadd_rn(__fmul_rn(x0, sn), __fmul_rn(x1, c));
+      for (int i = 0; i < 8; ++i)
+        if (m0 + 4 * i < p.M)
+          *reinterpret_cast<uint4*>(base + long(m0 + 4 * i) * p.ldo) =
+              stage_get(buf, r0 + 4 * i, u);
+    } else {  // EPI_ROPE
+      const int h = n / p.hd, d0 = n - h * p.hd;
+      const bool rot = h < p.hq + p.hkv;
+      int b = m0 / p.Mseq, s = m0 - b * p.Mseq;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (m0 + 4 * i < p.M) {
+          uint4 x = stage_get(buf, r0 + 4 * i, u);
+          uint16_t* dst;
+          if (h < p.hq) {
+            dst = p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d0;
+          } else if (rot) {
+            dst = p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d0;
+          } else {
+            dst = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq - p.hkv)) * p.hd + d0;
+          }
+          if (rot) x = rope_rotate8(x, rv[i]);
+          *reinterpret_cast<uint4*>(dst) = x;
+        }
+        s += 4;
+        while (s >= p.Mseq) { s -= p.Mseq; ++b; }
       }
-      dst = h < p.hq ? p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d0
-                     : p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d0;
-    } else {
-      const int hv = h - p.hq - p.hkv;
-      dst = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + hv) * p.hd + d0;
     }
   }
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  __syncwarp();
+}
+
+// Write back `units` 16-byte units of each staged e4m3 row: row r holds
+// output bytes col0 .. col0 + 16 * units - 1 of token row m_base + r.
+__device__ __forceinline__ void flush_rows_u8(const GemmParams& p, const uint8_t* buf, int lane,
+                                              int m_base, int col0, int units) {
+  __syncwarp();
+  const int u = lane & 7;
+  if (u < units) {
+    uint8_t* base = static_cast<uint8_t*>(p.out) + col0 + 16 * u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = (lane >> 3) + 4 * i;
+      if (m_base + r < p.M)
+        *reinterpret_cast<uint4*>(base + long(m_base + r) * p.ldo) = stage_get(buf, r, u);
+    }
+  }
+  __syncwarp();
+}
+
+// 32 bias values of columns n .. n + 31 (bf16 -> fp32); zeros without bias.
+__device__ __forceinline__ void load_bias32(const GemmParams& p, int n, uint4 (&b4)[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    b4[k] = p.bias ? __ldg(reinterpret_cast<const uint4*>(p.bias + n) + k) : make_uint4(0, 0, 0, 0);
+}
+
+// v = bf16(acc * alpha [+ bias]) as a float, in place: the value the plain
+// epilogue stores and the gated epilogues and the rotation start from.
+__device__ __forceinline__ void scale_bias32(const GemmParams& p, float (&v)[32],
+                                             const uint4 (&b4)[4], float alpha) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    float f[8];
+    float b[8];
+    unpack8(b4[k], b);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) f[j] = y[8 * k + j];
-    d4[k] = pack8_bf16(f);
+    for (int j = 0; j < 8; ++j) {
+      const float a = __fmul_rn(v[8 * k + j], alpha);
+      v[8 * k + j] = bf2f(f2bf(p.bias ? __fadd_rn(a, b[j]) : a));
+    }
   }
 }
 
-// GEGLU (normal orientation, BN = 256): gate columns 32c.., up columns
-// 128 + 32c.. of the same tile; output column tb * 128 + 32c ...
-__device__ __forceinline__ void epi_geglu_chunk(const GemmParams& p, const float (&g)[32],
-                                                const float (&u)[32], int m, int n_gate0,
-                                                int n_up0, int out_col0, float alpha) {
-  if (m >= p.M) return;
-  const float inv_os = __frcp_rn(__ldg(p.out_scale));
-  float q[32];
+// 8 accumulators of columns n .. n + 7 -> their 8 bf16 outputs bf16(acc *
+// alpha [+ bias]), rounded once, computed as paired fp32 operations (each
+// lane rounded exactly as the scalar operation: the same bits, half the
+// instructions).
+__device__ __forceinline__ uint4 scale_bias_pack8(const float* v, const uint4& b4, uint64_t alpha2,
+                                                  bool has_bias) {
+  const uint32_t w[4] = {b4.x, b4.y, b4.z, b4.w};
+  uint32_t o[4];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const float gv = scale_bias_bf16(g[j], alpha, p.bias, n_gate0 + j);
-    const float uv = scale_bias_bf16(u[j], alpha, p.bias, n_up0 + j);
-    q[j] = __fmul_rn(gelu_tanh_mul(gv, uv), inv_os);
+  for (int i = 0; i < 4; ++i) {
+    uint64_t a = mul2(f2_pack(v[2 * i], v[2 * i + 1]), alpha2);
+    if (has_bias) a = add2(a, bf16x2_to_f2(w[i]));
+    o[i] = pack_bf16x2(f2_lo(a), f2_hi(a));
   }
-  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + long(m) * p.ldo + out_col0);
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    float a[8], b[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) { a[j] = q[16 * k + j]; b[j] = q[16 * k + 8 + j]; }
-    const uint2 lo = pack8_e4m3(a), hi = pack8_e4m3(b);
-    dst[k] = make_uint4(lo.x, lo.y, hi.x, hi.y);
-  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// GELU + static requant of one row's 32 columns (the DiT FFN's fp8_gelu_mlp
-// middle step): h = gelu_tanh(bf16(acc * alpha + bias)), out = e4m3(h / s)
-// computed as h * fp32(1 / s), as the GEGLU epilogue does.
-__device__ __forceinline__ void epi_gelu_chunk(const GemmParams& p, const float (&v)[32], int m,
-                                               int n0, float alpha) {
-  if (m >= p.M) return;
-  const float inv_os = __frcp_rn(__ldg(p.out_scale));
-  float q[32];
+// The epilogue of one warp's 32 accumulator rows m_base .. m_base + 31 over
+// the accumulator chunks cb .. ce - 1 (32 columns each); load(c, v) fills
+// chunk c of this thread's row (warp-uniform), done() runs once this warp's
+// last chunk is loaded (it releases the TMEM accumulator).
+//   bf16 / RoPE: chunk c -> output columns col0 + 32c (RoPE: rotated);
+//   GELU:        the same columns as e4m3(gelu_tanh(y) / out_scale);
+//   GEGLU:       chunks c in [cb, ce) (within 0..3) are gate columns
+//                col0 + 32c, chunks c + 4 the matching up columns
+//                col0 + 128 + 32c; output e4m3 columns out0 + 32c =
+//                e4m3(gelu_tanh(gate) * up / out_scale).
+// y = bf16(acc * alpha [+ bias]) everywhere; division by out_scale is a
+// multiplication by its correctly rounded reciprocal, as in the standalone
+// kernels.  Each group of chunks (two for bf16, up to four for e4m3: one
+// 128-byte row segment) requests its bias pieces and rope rows first.
+template <class Load, class Done>
+__device__ __forceinline__ void warp_rows_epilogue(const GemmParams& p, uint8_t* buf, int lane,
+                                                   int m_base, int col0, int cb, int ce, int out0,
+                                                   float alpha, Load load, Done done) {
+  if (p.epi == EPI_GEGLU || p.epi == EPI_GELU) {
+    const float inv_os = __frcp_rn(__ldg(p.out_scale));
+    const bool geglu = p.epi == EPI_GEGLU;
+#pragma unroll 1
+    for (int c0 = cb; c0 < ce; c0 += 4) {
+      const int cn = ce - c0 < 4 ? ce - c0 : 4;
+#pragma unroll 1
+      for (int c = c0; c < c0 + cn; ++c) {
+        uint4 bg[4], bu[4];
+        load_bias32(p, col0 + 32 * c, bg);
+        if (geglu) load_bias32(p, col0 + 128 + 32 * c, bu);
+        float q[32];
+        load(c, q);
+        if (!geglu && c == ce - 1) done();
+        scale_bias32(p, q, bg, alpha);
+        if (geglu) {
+          float z[32];
+          load(c + 4, z);
+          if (c == ce - 1) done();
+          scale_bias32(p, z, bu, alpha);
 #pragma unroll
-  for (int j = 0; j < 32; ++j)
-    q[j] = __fmul_rn(gelu_tanh_mul(scale_bias_bf16(v[j], alpha, p.bias, n0 + j), 1.0f), inv_os);
-  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + long(m) * p.ldo + n0);
+          for (int j = 0; j < 32; ++j) q[j] = __fmul_rn(gelu_tanh_mul(q[j], z[j]), inv_os);
+        } else {
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    float a[8], b[8];
+          for (int j = 0; j < 32; ++j) q[j] = __fmul_rn(gelu_tanh_mul(q[j], 1.0f), inv_os);
+        }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { a[j] = q[16 * k + j]; b[j] = q[16 * k + 8 + j]; }
-    const uint2 lo = pack8_e4m3(a), hi = pack8_e4m3(b);
-    dst[k] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        for (int k = 0; k < 2; ++k) {
+          float a8[8], b8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) { a8[j] = q[16 * k + j]; b8[j] = q[16 * k + 8 + j]; }
+          const uint2 lo = pack8_e4m3(a8), hi = pack8_e4m3(b8);
+          stage_put(buf, lane, 2 * (c - c0) + k, make_uint4(lo.x, lo.y, hi.x, hi.y));
+        }
+      }
+      flush_rows_u8(p, buf, lane, m_base, (geglu ? out0 : col0) + 32 * c0, 2 * cn);
+    }
+    return;
+  }
+#pragma unroll 1
+  for (int c0 = cb; c0 < ce; c0 += 2) {
+    const int cn = ce - c0 < 2 ? ce - c0 : 2;
+    uint4 rv[8];
+    rope_rows(p, lane, m_base, col0 + 32 * c0, rv);
+    uint4 b4[2][4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      if (j < cn) load_bias32(p, col0 + 32 * (c0 + j), b4[j]);
+    const uint64_t alpha2 = f2_pack(alpha, alpha);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      if (j < cn) {
+        float v[32];
+        load(c0 + j, v);
+        if (c0 + j == ce - 1) done();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          stage_put(buf, lane, 4 * j + k, scale_bias_pack8(v + 8 * k, b4[j][k], alpha2, p.bias));
+      }
+    }
+    flush_rows_bf16(p, buf, lane, m_base, col0 + 32 * c0, 4 * cn, rv);
   }
 }
 
@@ -313,38 +426,20 @@ __device__ __forceinline__ void emit_swap_items(const GemmParams& p, int ta, int
 // (32 columns of this thread's TMEM lane); it is called warp-uniformly.
 // done() runs once every chunk has been loaded (it releases the TMEM
 // accumulator when the chunks come from TMEM).
-// Swapped orientation: the chunks are staged in the shared-memory tile T
-// (fp32 [BMT output columns][BN tokens], row stride BN + 4) and read back
-// transposed, so each thread then owns one token row with 32 contiguous
-// output columns and the row epilogue applies unchanged.
+// Normal orientation: the warp's rows go through warp_rows_epilogue, staged
+// in the warp's buffer ebuf.  Swapped orientation: the chunks are staged in
+// the shared-memory tile T (fp32 [BMT output columns][BN tokens], row
+// stride BN + 4) and read back transposed, token-major, so neighbouring
+// threads write neighbouring 16-byte pieces of one token row.
 template <bool SWAP, int BMT, int BN, class Load, class Done>
 __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int tb, int q, int lane,
-                                              float alpha, float* T, Load load, Done done) {
-  if (!SWAP && p.epi == EPI_GEGLU) {
-    const int m = ta * BMT + 32 * q + lane;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      float g[32], u[32];
-      load(c, g);
-      load(c + 4, u);
-      if (c == 3) done();
-      epi_geglu_chunk(p, g, u, m, tb * BN + 32 * c, tb * BN + 128 + 32 * c, tb * 128 + 32 * c,
-                      alpha);
-    }
-    return;
-  }
+                                              float alpha, float* T, uint8_t* ebuf, Load load,
+                                              Done done) {
   if (!SWAP) {
-    const int m = ta * BMT + 32 * q + lane;
     int c_last = BN / 32 - 1;
     while (c_last > 0 && tb * BN + 32 * c_last >= p.N) --c_last;
-#pragma unroll 1
-    for (int c = 0; c <= c_last; ++c) {
-      float v[32];
-      load(c, v);
-      if (c == c_last) done();
-      if (p.epi == EPI_GELU) epi_gelu_chunk(p, v, m, tb * BN + 32 * c, alpha);
-      else epi_rows_chunk(p, v, m, tb * BN + 32 * c, alpha);
-    }
+    warp_rows_epilogue(p, ebuf, lane, ta * BMT + 32 * q, tb * BN, 0,
+                       p.epi == EPI_GEGLU ? 4 : c_last + 1, tb * 128, alpha, load, done);
     return;
   }
   constexpr int TS = BMT + 4;
@@ -397,9 +492,16 @@ __host__ __device__ constexpr int t_tile_bytes() {
   return SWAP ? BN * (BMT + 4) * 4 : 0;
 }
 
+// normal orientation: the four epilogue warps' row staging buffers
+template <bool SWAP>
+__host__ __device__ constexpr int epi_stage_total() {
+  return SWAP ? 0 : 4 * kEpiStageBytes;
+}
+
 template <bool SWAP, int BMT, int BN, int STAGES>
 __host__ __device__ constexpr int smem_total() {
-  return STAGES * (BMT * BK + BN * BK) + t_tile_bytes<SWAP, BMT, BN>() + 1024 + 512;
+  return STAGES * (BMT * BK + BN * BK) + t_tile_bytes<SWAP, BMT, BN>() + epi_stage_total<SWAP>() +
+         1024 + 512;
 }
 
 // CLUSTER: the p.splits K-splits of a tile run as one thread-block cluster
@@ -428,8 +530,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
   float* T = reinterpret_cast<float*>(sB + STAGES * B_BYTES);
-  uint64_t* full =
-      reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES + t_tile_bytes<SWAP, BMT, BN>());
+  uint8_t* ebuf_base = sB + STAGES * B_BYTES + t_tile_bytes<SWAP, BMT, BN>();
+  uint64_t* full = reinterpret_cast<uint64_t*>(ebuf_base + epi_stage_total<SWAP>());
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -628,6 +730,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         tma_load_2d(sB + i * B_BYTES, &tmB, &full[i], (kb0 + i) * BK, tb * BN);
     }
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint8_t* ebuf = ebuf_base + (warp - 2) * kEpiStageBytes;  // normal orientation only
     const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
     const int row = acc_row<BMT>(q, lane);
     const bool valid = acc_row_valid<BMT>(lane);
@@ -686,7 +789,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       };
       if (p.splits == 1) {
         tile_epilogue<SWAP, BMT, BN>(
-            p, ta, tb, q, lane, alpha, T,
+            p, ta, tb, q, lane, alpha, T, ebuf,
             [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); }, release_tmem);
       } else {
         // spill this split's fp32 partial, accumulator-row major
@@ -714,7 +817,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           __threadfence();
           const float* base = p.partials + long(tile) * p.splits * (BMT * BN) + long(row) * BN;
           tile_epilogue<SWAP, BMT, BN>(
-              p, ta, tb, q, lane, alpha, T,
+              p, ta, tb, q, lane, alpha, T, ebuf,
               [&](int c, float (&v)[32]) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = 0.0f;
@@ -842,11 +945,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 //             both CTAs' TMA loads complete on it
 //   empty[s]  (each CTA) released by the even CTA's multicast commit
 //   tfull[b]  (each CTA) accumulator b ready, multicast commit
-//   tempty[b] (even CTA) 8 arrivals: the four epilogue warps of each CTA
+//   tempty[b] (even CTA) 16 arrivals: the eight epilogue warps of each CTA
+//             (two per TMEM lane quarter, each draining half the columns)
 // All waits are bounded; a final cluster barrier keeps both CTAs (their
 // shared memory and TMEM) alive until the pair is done.
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const GemmParams p) {
   constexpr int A_BYTES = 128 * BK;
@@ -857,14 +961,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint8_t* ebuf_base = sB + STAGES * B_BYTES;  // the epilogue warps' row staging
+  uint64_t* full = reinterpret_cast<uint64_t*>(ebuf_base + kPairEpiWarps * kEpiStageBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* epi_ok = abort_flag + 2;  // [4]
+  volatile int* epi_ok = abort_flag + 2;  // [kPairEpiWarps]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -879,7 +984,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 8);
+      mbar_init(&tempty[b], 2 * kPairEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -990,7 +1095,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   } else {
     // ----------------------------------------------------------- epilogue --
     pdl_wait();
-    const int q = warp & 3;
+    const int ew = warp - 2;               // 0 .. kPairEpiWarps - 1
+    const int q = warp & 3;                // TMEM lane quarter this warp may access
+    const int half = ew >> 2;              // which half of the tile's chunks it drains
+    uint8_t* ebuf = ebuf_base + ew * kEpiStageBytes;
+    // chunks [cb, ce) of this warp: the two warps of a lane quarter split
+    // the tile's columns (GEGLU: its four gate chunks, each with its up chunk)
+    constexpr int NCH = BN / 32;
+    const int nch = p.epi == EPI_GEGLU ? 4 : NCH;
+    const int cb = half ? (nch + 1) / 2 : 0, ce = half ? nch : (nch + 1) / 2;
     const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
     int local = 0;
     for (int u = pair; u < p.units; u += npairs, ++local) {
@@ -999,10 +1112,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const uint32_t aph = (local >> 1) & 1;
       const bool got = __all_sync(0xffffffffu,
                                   mbar_wait_bounded(&tfull[ab], aph, kWaitNs, abort_flag));
-      if (lane == 0) epi_ok[q] = got ? 1 : 0;
-      named_bar_sync(1, 128);
-      const bool all_ok = epi_ok[0] && epi_ok[1] && epi_ok[2] && epi_ok[3];
-      named_bar_sync(1, 128);
+      if (lane == 0) epi_ok[ew] = got ? 1 : 0;
+      named_bar_sync(1, 32 * kPairEpiWarps);
+      bool all_ok = true;
+#pragma unroll
+      for (int i = 0; i < kPairEpiWarps; ++i) all_ok = all_ok && epi_ok[i];
+      named_bar_sync(1, 32 * kPairEpiWarps);
       if (!all_ok) {
         if (lane == 0) record_timeout(p.status);
         *abort_flag = 1;
@@ -1016,27 +1131,234 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty_lead + 8u * ab);
       };
-      const int m = tm * 256 + int(rank) * 128 + 32 * q + lane;
-      if (p.epi == EPI_GEGLU) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float g[32], uu[32];
-          load(c, g);
-          load(c + 4, uu);
-          if (c == 3) release();
-          epi_geglu_chunk(p, g, uu, m, tn * BN + 32 * c, tn * BN + 128 + 32 * c,
-                          tn * 128 + 32 * c, alpha);
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          load(c, v);
-          if (c == BN / 32 - 1) release();
-          if (p.epi == EPI_GELU) epi_gelu_chunk(p, v, m, tn * BN + 32 * c, alpha);
-          else epi_rows_chunk(p, v, m, tn * BN + 32 * c, alpha);
+      warp_rows_epilogue(p, ebuf, lane, tm * 256 + int(rank) * 128 + 32 * q, tn * BN, cb, ce,
+                         tn * 128, alpha, load, release);
+    }
+  }
+
+  cluster_sync_all();  // the pair is done with both CTAs' memory
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------- wide CTA-pair kernel --
+//
+// Normal orientation, tiles of 256 rows x 512 columns per CTA pair: per
+// K-step the even CTA issues two tcgen05.mma.cta_group::2 (M = 256, N =
+// 256), one per 256-column half of the tile, into the two halves of the
+// whole TMEM (512 columns x 128 lanes per CTA).  Per K-block an SM loads 16
+// KB of x8 and 2 x 16 KB of weights (48 KB) for 8.4 M MACs, against 32 KB
+// for 4.2 M MACs in gemm_pair_kernel: a quarter fewer operand bytes per MAC,
+// which is what bounds the pair kernel's main loop (the shared-memory fill).
+// The accumulator takes the whole TMEM, so it is single-buffered: the
+// epilogue (eight warps, two per TMEM lane quarter, one 256-column half
+// each) drains it while the producer keeps filling the 4-stage ring with the
+// next tile's operands, and the MMAs of the next tile start once every
+// epilogue warp of both CTAs has read its columns.
+//   full[s]   (even CTA) 2 arrivals: each CTA's producer arms its bytes
+//   empty[s]  (each CTA) released by the even CTA's multicast commit
+//   tfull     (each CTA) the accumulator is complete, multicast commit
+//   tempty    (even CTA) 16 arrivals: eight epilogue warps per CTA
+// Half h of the tile holds weight rows tn*512 + h*256 .. +255 (each CTA the
+// 128 rows rank*128 .. of that half), so the column mapping is that of two
+// adjacent 256-column tiles.  All waits are bounded; a final cluster barrier
+// keeps both CTAs (their shared memory and TMEM) alive until the pair is done.
+constexpr int kWideEpiWarps = 8;
+constexpr int kWideThreads = 64 + 32 * kWideEpiWarps;
+
+template <int STAGES>
+__global__ void __launch_bounds__(kWideThreads, 1)
+gemm_pair_wide_kernel(const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+  constexpr int BN = 256;                      // one MMA's N; the tile is 2 x BN
+  constexpr int A_BYTES = 128 * BK;
+  constexpr int B_HALF = (BN / 2) * BK;        // this CTA's rows of one half
+  constexpr int B_BYTES = 2 * B_HALF;
+  constexpr uint32_t TMEM_COLS = 512;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint8_t* ebuf_base = sB + STAGES * B_BYTES;  // the epilogue warps' row staging
+  uint64_t* full = reinterpret_cast<uint64_t*>(ebuf_base + kWideEpiWarps * kEpiStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 1;
+  uint64_t* drain = tempty + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* epi_ok = abort_flag + 2;  // [kWideEpiWarps]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool lead = rank == 0;
+  const int pair = int(blockIdx.x >> 1), npairs = int(gridDim.x >> 1);
+  pdl_trigger();
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 2);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 2 * kWideEpiWarps);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint32_t full_lead = map_cluster(smem_u32(full), 0);
+  const uint32_t tempty_lead = map_cluster(smem_u32(tempty), 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      const int u0 = pair;
+      const int brow = int(rank) * (BN / 2);
+      int n_pre = 0;
+      if (u0 < p.units) {  // weights first, before the dependency wait
+        const int tn = u0 / p.a_tiles;
+        n_pre = p.k_blocks < STAGES ? p.k_blocks : STAGES;
+        for (int i = 0; i < n_pre; ++i) {
+          mbar_arrive_expect_tx_cluster(full_lead + 8u * i, A_BYTES + B_BYTES);
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d_pair(sB + i * B_BYTES + h * B_HALF, &tmB, full_lead + 8u * i, i * BK,
+                             tn * 2 * BN + h * BN + brow);
         }
       }
+      pdl_wait();
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = u0; u < p.units && ok; u += npairs) {
+        const int tm = u % p.a_tiles, tn = u / p.a_tiles;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          const bool pre = (u == u0) && (kb < n_pre);
+          if (!pre) {
+            if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitNs, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx_cluster(full_lead + 8u * stage, A_BYTES + B_BYTES);
+            for (int h = 0; h < 2; ++h)
+              tma_load_2d_pair(sB + stage * B_BYTES + h * B_HALF, &tmB, full_lead + 8u * stage,
+                               kb * BK, tn * 2 * BN + h * BN + brow);
+          }
+          tma_load_2d_pair(sA + stage * A_BYTES, &tmA, full_lead + 8u * stage, kb * BK,
+                           tm * 256 + int(rank) * 128);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        record_timeout(p.status);
+        *abort_flag = 1;
+        if (lead) {  // the even CTA's barriers count both CTAs' copies
+          int st = stage;
+          uint32_t ph = phase;
+          for (int i = 0; i < issued && i < STAGES; ++i) {
+            if (--st < 0) { st = STAGES - 1; ph ^= 1u; }
+            mbar_wait_bounded(&full[st], ph, kDrainNs, nullptr);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------ MMA issuer (even CTA) --
+    if (lane == 0 && lead) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(256, BN);
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      int stage = 0, local = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = pair; u < p.units && ok; u += npairs, ++local) {
+        if (!mbar_wait_bounded(tempty, (local & 1) ^ 1u, kWaitNs, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, kWaitNs, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = sdesc_k_sw128(a_base + stage * A_BYTES);
+          const uint64_t bd0 = sdesc_k_sw128(b_base + stage * B_BYTES);
+          const uint64_t bd1 = sdesc_k_sw128(b_base + stage * B_BYTES + B_HALF);
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k) {
+            const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+            umma_pair_e4m3(tmem_base, ad + 2 * k, bd0 + 2 * k, idesc, acc);
+            umma_pair_e4m3(tmem_base + BN, ad + 2 * k, bd1 + 2 * k, idesc, acc);
+          }
+          umma_pair_commit(&empty[stage], 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_pair_commit(tfull, 0x3);
+      }
+      if (!ok) {
+        record_timeout(p.status);
+        *abort_flag = 1;
+        umma_pair_commit(drain, 0x1);
+        mbar_wait_bounded(drain, 0, kDrainNs, nullptr);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ----------------------------------------------------------- epilogue --
+    pdl_wait();
+    const int ew = warp - 2;               // 0 .. 7
+    const int q = warp & 3;                // TMEM lane quarter this warp may access
+    const int h = ew >> 2;                 // the 256-column half it drains
+    uint8_t* ebuf = ebuf_base + ew * kEpiStageBytes;
+    const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
+    int local = 0;
+    for (int u = pair; u < p.units; u += npairs, ++local) {
+      const int tm = u % p.a_tiles, tn = u / p.a_tiles;
+      const bool got = __all_sync(0xffffffffu,
+                                  mbar_wait_bounded(tfull, local & 1, kWaitNs, abort_flag));
+      if (lane == 0) epi_ok[ew] = got ? 1 : 0;
+      named_bar_sync(1, 32 * kWideEpiWarps);
+      bool all_ok = true;
+#pragma unroll
+      for (int i = 0; i < kWideEpiWarps; ++i) all_ok = all_ok && epi_ok[i];
+      named_bar_sync(1, 32 * kWideEpiWarps);
+      if (!all_ok) {
+        if (lane == 0) record_timeout(p.status);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + uint32_t(h * BN) + (uint32_t(32 * q) << 16);
+      auto load = [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); };
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_lead);
+      };
+      // the half's first output column; with the GEGLU epilogue it holds
+      // gate block (tn*2 + h) in columns 0..127 and the matching up block in
+      // 128..255 (the gate/up block layout)
+      const int n0 = tn * 2 * BN + h * BN;
+      warp_rows_epilogue(p, ebuf, lane, tm * 256 + int(rank) * 128 + 32 * q, n0, 0,
+                         p.epi == EPI_GEGLU ? 4 : BN / 32, (tn * 2 + h) * 128, alpha, load,
+                         release);
     }
   }
 
@@ -1083,7 +1405,8 @@ gemm_pair_split_kernel(const __grid_constant__ CUtensorMap tmA,
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint8_t* ebuf_base = sB + STAGES * B_BYTES;  // the epilogue warps' row staging
+  uint64_t* full = reinterpret_cast<uint64_t*>(ebuf_base + 4 * kEpiStageBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* drain = tfull + 1;
@@ -1212,6 +1535,7 @@ gemm_pair_split_kernel(const __grid_constant__ CUtensorMap tmA,
     pdl_wait();
     const int q = warp & 3;
     const int row = 32 * q + lane;
+    uint8_t* ebuf = ebuf_base + (warp - 2) * kEpiStageBytes;
     const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
     const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(tfull, 0, kWaitNs, abort_flag));
     if (lane == 0) epi_ok[q] = got ? 1 : 0;
@@ -1256,7 +1580,6 @@ gemm_pair_split_kernel(const __grid_constant__ CUtensorMap tmA,
         else record_timeout(p.status);
       }
       if (in) {
-        const int m = tm * 256 + int(rank & 1u) * 128 + row;
         const float* pr = part + row * RS;
         auto load = [&](int c, float (&v)[32]) {
           tmem_ld32(tmem_base + 32 * c + (uint32_t(32 * q) << 16), v);
@@ -1270,24 +1593,8 @@ gemm_pair_split_kernel(const __grid_constant__ CUtensorMap tmA,
             v[4 * k + 3] = __fadd_rn(v[4 * k + 3], f.w);
           }
         };
-        if (p.epi == EPI_GEGLU) {
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            float g[32], uu[32];
-            load(c, g);
-            load(c + 4, uu);
-            epi_geglu_chunk(p, g, uu, m, tn * BN + 32 * c, tn * BN + 128 + 32 * c,
-                            tn * 128 + 32 * c, alpha);
-          }
-        } else {
-#pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
-            float v[32];
-            load(c, v);
-            if (p.epi == EPI_GELU) epi_gelu_chunk(p, v, m, tn * BN + 32 * c, alpha);
-            else epi_rows_chunk(p, v, m, tn * BN + 32 * c, alpha);
-          }
-        }
+        warp_rows_epilogue(p, ebuf, lane, tm * 256 + int(rank & 1u) * 128 + 32 * q, tn * BN, 0,
+                           p.epi == EPI_GEGLU ? 4 : BN / 32, tn * 128, alpha, load, [] {});
       }
     }
   }
@@ -1379,15 +1686,20 @@ Plan make_plan(int M, int N, int K, int epi) {
     const long cost1 = ((tiles1 + sms - 1) / sms) * (16384L + pl.bn * 128L) * kb;
     const long mt2 = (M + 255L) / 256;
     if (M >= 256) {
-      static const int kPairBn[] = {256, 192, 160, 128};
+      // 512: the wide pair tile (two 256-column MMAs into the whole TMEM)
+      static const int kPairBn[] = {512, 256, 192, 160, 128};
       int best = 0;
       bool best_split = false;
       long best_cost = cost1;
       for (int bn2 : kPairBn) {
-        if (N % bn2 != 0 || (epi == EPI_GEGLU && bn2 != 256)) continue;
+        if (N % bn2 != 0 || (epi == EPI_GEGLU && bn2 != 256 && bn2 != 512)) continue;
         const long units2 = mt2 * (N / bn2);
         if (units2 < 16) continue;
-        const long cost2 = ((units2 + npairs - 1) / npairs) * (16384L + bn2 * 64L) * kb;
+        // the wide tile's accumulator fills the TMEM, so its epilogue does
+        // not overlap the next tile's main loop: measured at about 20
+        // K-blocks of main-loop time per tile
+        const long kb_eff = bn2 == 512 ? kb + 20 : kb;
+        const long cost2 = ((units2 + npairs - 1) / npairs) * (16384L + bn2 * 64L) * kb_eff;
         if (cost2 < best_cost || (epi == EPI_GEGLU && !best)) {
           best = bn2;
           best_cost = cost2;
@@ -1564,7 +1876,8 @@ int launch_swap(Plan pl, const CUtensorMap& ta, const CUtensorMap& tb, GemmParam
 template <int BN, int STAGES>
 int launch_pair(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                 cudaStream_t s) {
-  constexpr int smem = STAGES * (128 * BK + (BN / 2) * BK) + 1024 + 256;
+  constexpr int smem =
+      STAGES * (128 * BK + (BN / 2) * BK) + kPairEpiWarps * kEpiStageBytes + 1024 + 256;
   static_assert(smem <= 232448, "shared memory budget");
   auto kern = gemm_pair_kernel<BN, STAGES>;
   if (first_use(reinterpret_cast<const void*>(kern))) {
@@ -1576,7 +1889,7 @@ int launch_pair(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, co
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kPairThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
@@ -1596,10 +1909,45 @@ int launch_pair(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, co
   return FRT_OK;
 }
 
+template <int STAGES>
+int launch_pair_wide(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb,
+                     const GemmParams& p, cudaStream_t s) {
+  constexpr int smem = STAGES * (128 * BK + 256 * BK) + kWideEpiWarps * kEpiStageBytes + 1024 + 256;
+  static_assert(smem <= 232448, "shared memory budget");
+  auto kern = gemm_pair_wide_kernel<STAGES>;
+  if (first_use(reinterpret_cast<const void*>(kern))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return fail(FRT_ECUDA, "cudaFuncSetAttribute(max dynamic smem %d)", smem);
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.grid);
+  cfg.blockDim = dim3(kWideThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FRT_ECUDA, "gemm_pair_wide_kernel: %s", cudaGetErrorString(e));
+  }
+  return FRT_OK;
+}
+
 template <int BN, int STAGES>
 int launch_pair_split(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb,
                       const GemmParams& p, cudaStream_t s) {
-  constexpr int smem = STAGES * (128 * BK + (BN / 2) * BK) + 1024 + 256;
+  constexpr int smem = STAGES * (128 * BK + (BN / 2) * BK) + 4 * kEpiStageBytes + 1024 + 256;
   static_assert(smem <= 232448, "shared memory budget");
   auto kern = gemm_pair_split_kernel<BN, STAGES>;
   if (first_use(reinterpret_cast<const void*>(kern))) {
@@ -1650,14 +1998,16 @@ int run_gemm(const Plan& pl, GemmParams& p, const void* x8, const void* w8, void
   int rc;
   if (pl.pair) {  // each CTA loads 128 rows of x8 and BN/2 rows of w8
     if ((rc = make_map(&ta, x8, p.M, p.K, 128))) return rc;
-    if ((rc = make_map(&tb, w8, p.N, p.K, pl.bn / 2))) return rc;
+    // weight box: this CTA's half of one MMA's 256 (or bn) columns
+    if ((rc = make_map(&tb, w8, p.N, p.K, (pl.bn > 256 ? 256 : pl.bn) / 2))) return rc;
     if (pl.split2) {
       if (pl.bn == 256) return launch_pair_split<256, 6>(pl, ta, tb, p, s);
       return launch_pair_split<128, 8>(pl, ta, tb, p, s);
     }
+    if (pl.bn == 512) return launch_pair_wide<4>(pl, ta, tb, p, s);
     if (pl.bn == 256) return launch_pair<256, 6>(pl, ta, tb, p, s);
-    if (pl.bn == 192) return launch_pair<192, 7>(pl, ta, tb, p, s);
-    if (pl.bn == 160) return launch_pair<160, 8>(pl, ta, tb, p, s);
+    if (pl.bn == 192) return launch_pair<192, 6>(pl, ta, tb, p, s);
+    if (pl.bn == 160) return launch_pair<160, 7>(pl, ta, tb, p, s);
     return launch_pair<128, 8>(pl, ta, tb, p, s);
   }
   if (!pl.swap) {

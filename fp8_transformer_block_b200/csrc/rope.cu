@@ -8,8 +8,10 @@
 // `ad:prefix` range gathers the host's prefix keys through `kperm` and copies
 // the values) and `_alloc` (q [1,S,nh,hd], caches [1,T,kv,hd]).
 //
-// All three are HBM-bound streams: 16-byte loads and stores, one 8-element
-// chunk per thread step, grid-stride loops sized to the SM count.
+// All three are HBM-bound streams of 16-byte loads and stores: the split
+// kernel one block per token and column slice with every load of a thread
+// issued before its first store, the prefix copy a grid-stride loop sized to
+// the SM count.
 #include "frt_internal.cuh"
 
 namespace frt {
@@ -37,62 +39,83 @@ struct SplitArgs {
   uint16_t* q_out;
   uint16_t* k_cache;
   uint16_t* v_cache;
-  long suffix_units;
-  PrefixArgs pre;  // pre.units == 0: no prefix copy
 };
 
-// Rotate 4 adjacent pairs of x (8 bf16) with 4 (cos, sin) pairs of r.
-__device__ __forceinline__ uint4 rotate8(const uint4& xv, const uint4& rv) {
-  float x[8], r[8], o[8];
-  unpack8(xv, x);
-  unpack8(rv, r);
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const float x0 = x[2 * p], x1 = x[2 * p + 1], c = r[2 * p], s = r[2 * p + 1];
-    o[2 * p] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, s));
-    o[2 * p + 1] = __fadd_rn(__fmul_rn(x0, s), __fmul_rn(x1, c));
-  }
-  return pack8_bf16(o);
-}
+// Units (16 bytes: 8 columns of one row's q, k or v) per thread per step of
+// the split kernel: their loads are all issued before the first store.
+constexpr int kSplitUnroll = 4;
+constexpr int kSplitThreads = 128;
 
-__global__ void split_rope_kernel(SplitArgs a) {
+// Split + RoPE + KV write.  Block (x, s, b) takes token s of batch b (no
+// index division for the row) and units x*T*U + t + T*k (k < U) of its
+// N/8: the row's q/k/v pieces and their rope-table pieces are requested
+// first, then rotated and stored.
+__global__ void __launch_bounds__(kSplitThreads)
+split_rope_kernel(SplitArgs a) {
+  const int s = int(blockIdx.y), b = int(blockIdx.z);
   const int hd8 = a.hd / 8;
-  const int heads = a.hq + 2 * a.hkv;
-  const long N8 = long(heads) * hd8;
-  const long total = a.suffix_units + a.pre.units;
+  const int N8 = (a.hq + 2 * a.hkv) * hd8;
+  const long r = long(b) * a.M + s;
+  const uint16_t* src = a.qkv + r * N8 * 8;
+  const uint16_t* rrow = a.rope + long(s) * a.hd;
+  const long krow = (long(b) * a.T + a.P + s) * a.hkv;   // cache row (in heads)
+  const long qrow = r * a.hq;                            // q_out row (in heads)
   pdl_trigger();
   pdl_wait();
-  for (long g = blockIdx.x * long(blockDim.x) + threadIdx.x; g < total;
-       g += long(gridDim.x) * blockDim.x) {
-    if (g < a.suffix_units) {
-      const long r = g / N8;
-      const int c8 = int(g % N8);
-      const int b = int(r / a.M), s = int(r % a.M);
-      const int h = c8 / hd8, d0 = (c8 % hd8) * 8;
-      const uint4 xv = __ldg(reinterpret_cast<const uint4*>(a.qkv + r * N8 * 8 + long(c8) * 8));
-      if (h < a.hq + a.hkv) {
-        const uint4 rv = __ldg(reinterpret_cast<const uint4*>(a.rope + long(s) * a.hd + d0));
-        const uint4 o = rotate8(xv, rv);
-        uint16_t* dst = h < a.hq
-            ? a.q_out + ((long(b) * a.M + s) * a.hq + h) * a.hd + d0
-            : a.k_cache + ((long(b) * a.T + a.P + s) * a.hkv + (h - a.hq)) * a.hd + d0;
-        *reinterpret_cast<uint4*>(dst) = o;
+  const int c_base = int(blockIdx.x) * kSplitThreads * kSplitUnroll + int(threadIdx.x);
+  uint4 xv[kSplitUnroll], rv[kSplitUnroll];
+#pragma unroll
+  for (int k = 0; k < kSplitUnroll; ++k) {
+    const int c8 = c_base + k * kSplitThreads;
+    if (c8 < N8) {
+      const int h = c8 / hd8, d0 = (c8 - h * hd8) * 8;
+      xv[k] = __ldg(reinterpret_cast<const uint4*>(src + c8 * 8));
+      if (h < a.hq + a.hkv) rv[k] = __ldg(reinterpret_cast<const uint4*>(rrow + d0));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kSplitUnroll; ++k) {
+    const int c8 = c_base + k * kSplitThreads;
+    if (c8 < N8) {
+      const int h = c8 / hd8, d0 = (c8 - h * hd8) * 8;
+      uint16_t* dst;
+      uint4 o = xv[k];
+      if (h < a.hq) {
+        dst = a.q_out + (qrow + h) * a.hd + d0;
+        o = rope_rotate8(o, rv[k]);
+      } else if (h < a.hq + a.hkv) {
+        dst = a.k_cache + (krow + (h - a.hq)) * a.hd + d0;
+        o = rope_rotate8(o, rv[k]);
       } else {
-        const int hv = h - a.hq - a.hkv;
-        *reinterpret_cast<uint4*>(a.v_cache + ((long(b) * a.T + a.P + s) * a.hkv + hv) * a.hd + d0) = xv;
+        dst = a.v_cache + (krow + (h - a.hq - a.hkv)) * a.hd + d0;
       }
-    } else {
-      prefix_unit(a.pre, g - a.suffix_units);
+      *reinterpret_cast<uint4*>(dst) = o;
     }
   }
 }
 
 int launch_split(const SplitArgs& a, cudaStream_t s) {
-  const long total = a.suffix_units + a.pre.units;
-  if (total == 0) return FRT_OK;
-  const long blocks_needed = (total + 255) / 256;
-  const int grid = int(blocks_needed < num_sms() * 16L ? blocks_needed : num_sms() * 16L);
-  return launch_pdl("split_rope_kernel", split_rope_kernel, dim3(grid), dim3(256), 0, s, a);
+  if (long(a.B) * a.M == 0) return FRT_OK;
+  const int N8 = (a.hq + 2 * a.hkv) * (a.hd / 8);
+  const int gx = (N8 + kSplitThreads * kSplitUnroll - 1) / (kSplitThreads * kSplitUnroll);
+  return launch_pdl("split_rope_kernel", split_rope_kernel, dim3(gx, a.M, a.B),
+                    dim3(kSplitThreads), 0, s, a);
+}
+
+// The prefix copy alone: 16-byte units over a grid sized to the SM count.
+__global__ void prefix_copy_kernel(PrefixArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  for (long g = blockIdx.x * long(blockDim.x) + threadIdx.x; g < a.units;
+       g += long(gridDim.x) * blockDim.x)
+    prefix_unit(a, g);
+}
+
+int launch_prefix(const PrefixArgs& a, cudaStream_t s) {
+  if (a.units == 0) return FRT_OK;
+  const long blocks_needed = (a.units + 255) / 256;
+  const int grid = int(blocks_needed < num_sms() * 8L ? blocks_needed : num_sms() * 8L);
+  return launch_pdl("prefix_copy_kernel", prefix_copy_kernel, dim3(grid), dim3(256), 0, s, a);
 }
 
 }  // namespace
@@ -153,26 +176,30 @@ extern "C" int frt_split_rope_kvcache(int B, int M, int hq, int hkv, int hd, int
     FRT_REQUIRE(aligned(qkv, 16) && aligned(rope, 16) && (!q_out || aligned(q_out, 16)),
                 FRT_EALIGN, "qkv, rope and q_out must be 16-byte aligned");
   }
+  FRT_REQUIRE(M <= 65535 && B <= 65535, FRT_ESHAPE,
+              "the split kernel takes at most 65535 tokens and batches, got M=%d B=%d", M, B);
   frt::SplitArgs a{};
   a.B = B; a.M = M; a.hq = hq; a.hkv = hkv; a.hd = hd; a.P = P; a.T = T;
   a.qkv = qkv; a.rope = rope; a.q_out = q_out; a.k_cache = k_cache; a.v_cache = v_cache;
-  a.suffix_units = long(B) * M * (hq + 2 * hkv) * (hd / 8);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (prefix_k) {
+    frt::PrefixArgs pre{};
     int rc = frt::prefix_args(B, hkv, hd, P, T, prefix_T_src, prefix_k, prefix_v,
-                              prefix_interleave, k_cache, v_cache, &a.pre);
+                              prefix_interleave, k_cache, v_cache, &pre);
+    if (rc) return rc;
+    rc = frt::launch_prefix(pre, st);
     if (rc) return rc;
   }
-  return frt::launch_split(a, static_cast<cudaStream_t>(stream));
+  return frt::launch_split(a, st);
 }
 
 extern "C" int frt_prefix_copy_kv(int B, int hkv, int hd, int P, int T, int T_src,
                                   const frt_bf16* prefix_k, const frt_bf16* prefix_v, int interleave,
                                   frt_bf16* k_cache, frt_bf16* v_cache, void* stream) {
   frt::clear_error();
-  frt::SplitArgs a{};
+  frt::PrefixArgs pre{};
   int rc = frt::prefix_args(B, hkv, hd, P, T, T_src, prefix_k, prefix_v, interleave, k_cache,
-                            v_cache, &a.pre);
+                            v_cache, &pre);
   if (rc) return rc;
-  a.hkv = hkv; a.hd = hd;
-  return frt::launch_split(a, static_cast<cudaStream_t>(stream));
+  return frt::launch_prefix(pre, static_cast<cudaStream_t>(stream));
 }

@@ -260,8 +260,9 @@ int frt_build_rope_table(int M, int hd, int P, double theta,
  * For q and k heads every adjacent pair (x0, x1) with c = rope[s, 2i],
  * sn = rope[s, 2i+1] becomes (x0*c - x1*sn, x0*sn + x1*c) (fp32, rounded to
  * bf16).  q_out: [B, M, hq, hd]; k_cache, v_cache: [B, T, hkv, hd], written
- * at rows P + s (v copied).  If prefix_k is non-NULL the same launch also
- * copies the prefix (see frt_prefix_copy_kv).  Requires P + M <= T,
+ * at rows P + s (v copied).  If prefix_k is non-NULL the call also copies
+ * the prefix (frt_prefix_copy_kv, launched first).  Requires P + M <= T,
+ * M <= 65535 and B <= 65535,
  * hd % 8 == 0, 16-byte aligned pointers.
  */
 int frt_split_rope_kvcache(int B, int M, int hq, int hkv, int hd, int P,

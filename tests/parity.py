@@ -49,9 +49,27 @@ def rel_rms_err(got_bf16, ref_bf16):
 
 
 def assert_rms(got_bf16, ref_bf16, tol=RMS_TOL, what="values"):
-    e = rel_rms_err(got_bf16, ref_bf16)
-    assert e <= tol, f"{what}: max|err| = {e:.3e} * rms(ref) > {tol}"
-    return e
+    """max|err| <= tol * rms(ref), where an element that differs from the
+    reference by exactly one bf16 step is always within the bar.  Both
+    sides round an fp32 value to bf16, and the two fp32 values (sums taken
+    in different orders) can straddle a rounding boundary; one bf16 step is
+    2^-8 .. 2^-7 of the value, which exceeds 2e-2 * rms for outputs beyond
+    about 5 * rms (present at these sizes).  Every element off by more than
+    one step must meet the bar."""
+    g = bf16_value(got_bf16).astype(np.float64)
+    r = bf16_value(ref_bf16).astype(np.float64)
+    if not r.size:
+        return 0.0
+    rms = np.sqrt((r ** 2).mean())
+    err = np.abs(g - r)
+    over = err > tol * rms
+    if over.any():
+        steps = bf16_ulps(np.asarray(got_bf16)[over], np.asarray(ref_bf16)[over])
+        bad = int((steps > 1).sum())
+        worst = float(err[over][steps > 1].max() / rms) if bad else 0.0
+        assert bad == 0, (f"{what}: {bad} values beyond {tol} * rms(ref) and more than "
+                          f"one bf16 step off (worst {worst:.3e} * rms)")
+    return float(err.max() / rms)
 
 
 def bf16_ulps(got_bf16, ref_bf16):

@@ -209,12 +209,75 @@ GEMM_CASES = [
     (1024, 2048, 4096, False),     # K in halves over two 256-wide pairs
     (1100, 1024, 4096, True),      # K in halves, ragged 256-row tile
     (1100, 2304, 1024, True),      # BN = 256 pairs (N not a multiple of 512)
-    # wide CTA pairs (256 x 512 tiles, two 256-column MMAs per K-step)
     (2560, 8192, 256, True),       # several tiles per pair, K < ring depth
     (1300, 5120, 1152, False),     # ragged last 256-row tile, K tail of 1 block
     (3000, 2048, 2048, True),      # ragged rows, K beyond the ring
-    (4096, 4096, 1024, False),     # two tiles on most pairs
 ]
+
+
+# wide CTA pairs (256 x 512 tiles, two 256-column MMAs per K-step): long K
+# only, so the oracle checks seeded sampled rows (rows are independent)
+WIDE_CASES = [
+    # M, N, K, bias, epilogue
+    (2048, 4096, 8192, True, "bf16"),      # one tile per pair
+    (4000, 4096, 8192, False, "bf16"),     # two tiles on most pairs, ragged rows
+    (2048, 8192, 8192, False, "geglu"),    # gate/up blocks, two per wide tile
+    (2048, 4096, 8192, True, "gelu"),
+]
+
+
+@pytest.mark.parametrize("M,N,K,bias,epi", WIDE_CASES)
+def test_gemm_wide_parity_sampled(rt, M, N, K, bias, epi):
+    frt, runtime, torch = rt
+    code = {"bf16": frt.FRT_EPI_BF16, "geglu": frt.FRT_EPI_GEGLU_E4M3,
+            "gelu": frt.FRT_EPI_GELU_E4M3}[epi]
+    plan = frt.frt_gemm_plan_info(M, N, K, code)
+    assert plan["pair"] == 1 and plan["tile_cols"] == 512, plan
+    rng = np.random.default_rng(M + N + K)
+    x8 = _x8_codes(M, K, 300 + M)
+    w = normal_bf16(rng, (N, K), 0.02)
+    b = normal_bf16(rng, (N,), 0.5) if bias else None
+    a = 0.0173
+    sel = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 62, replace=False)]))
+    if epi == "geglu":
+        H = N // 2
+        ws = [w[:H], w[H:]]
+        cat = oracle.pack_weights_fp8(ws)
+        pk = runtime.pack(ws, layout=frt.FRT_PACK_GATE_UP_BLOCKS)
+        gu = oracle.fp8_gemm(x8, cat["w8"], a, cat["w_scale"], rows=sel)
+        s_out = max(oracle.geglu_quant(gu, 1.0)[1] / 448.0, 1e-8)
+        ref, _ = oracle.geglu_quant(gu, s_out)
+        out = torch.full((M, H), 0x7F, dtype=torch.uint8, device="cuda")
+        ldo = H
+    else:
+        pk_ref = oracle.pack_weights_fp8([w], [b])
+        pk = runtime.pack([w], [b] if bias else None)
+        y = oracle.fp8_gemm(x8, pk_ref["w8"], a, pk_ref["w_scale"],
+                            pk_ref["bias"] if bias else None, rows=sel)
+        if epi == "gelu":
+            s_out = max(oracle.gelu_quant(y, 1.0)[1] / 448.0, 1e-8)
+            ref, _ = oracle.gelu_quant(y, s_out)
+            out = torch.full((M, N), 0x7F, dtype=torch.uint8, device="cuda")
+        else:
+            s_out, ref = None, y
+            out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ldo = N
+    wsb = frt.frt_gemm_workspace_size(M, N, K, code)
+    frt.frt_packed_fp8_gemm(M, N, K, runtime.u8_dev(x8), pk.w8, runtime.scale_dev(a),
+                            pk.w_scale, pk.bias if bias else None, code, out, ldo,
+                            None if s_out is None else runtime.scale_dev(s_out),
+                            runtime.workspace(wsb), wsb)
+    _sync(torch)
+    assert frt.frt_device_status(True) == frt.FRT_OK
+    if epi == "bf16":
+        got = runtime.bf16_host(out)[sel]
+        assert_rms(got, ref, what=f"wide GEMM {M}x{N}x{K}")
+        assert np.percentile(bf16_ulps(got, ref), 99.9) <= 1
+        # rows past the sample are written too (no NaN left anywhere)
+        assert not torch.isnan(out).any().item()
+    else:
+        assert_codes(runtime.u8_host(out)[sel], ref, what=f"wide {epi} {M}x{N}x{K}")
+        assert not (out == 0x7F).all(dim=1).any().item()
 
 
 @pytest.mark.parametrize("M,N,K,bias", GEMM_CASES)

@@ -29,3 +29,23 @@ def test_step_distance_nan_is_never_one_step():
     assert e4m3_step_distance([0xFF], [0xFE])[0] == 2
     assert e4m3_step_distance([0xFE], [0xFF])[0] == 2
     assert e4m3_step_distance([0x7F], [0x7F])[0] == 0
+
+
+def test_rms_bar_accepts_one_bf16_step_only():
+    import pytest
+    from parity import assert_rms
+    from fp8_transformer_block_b200.synth import bf16_bits
+    rng = np.random.default_rng(0)
+    ref = bf16_bits(rng.standard_normal(4096).astype(np.float32))
+    big = int(np.argmax(np.abs(ref.view(np.int16).astype(np.int32) & 0x7FFF)))
+    got = ref.copy()
+    got[big] += 1                     # one step at the largest value: accepted
+    assert_rms(got, ref)
+    got[big] += 1                     # two steps (> 2e-2 * rms there): rejected
+    with pytest.raises(AssertionError):
+        assert_rms(got, ref)
+    got = ref.copy()
+    small = int(np.argmin(np.abs(ref.view(np.int16).astype(np.int32) & 0x7FFF)))
+    got[small] = bf16_bits(np.array([0.5], np.float32))[0]   # far off at a small value: rejected
+    with pytest.raises(AssertionError):
+        assert_rms(got, ref)

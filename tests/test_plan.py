@@ -31,11 +31,19 @@ def frt():
                                  grid=148)),
     # gate/up with the GEGLU epilogue: pairs, 256-wide (gate and up together)
     ((1024, 32768, 2048, 1), dict(swap=0, pair=1, tile_cols=256, units=512)),
+    # long K: the wide (256 x 512) pair tiles, whose single-buffered
+    # accumulator exposes the epilogue, pay off
+    ((2048, 4096, 8192, 0), dict(pair=1, split2=0, tile_cols=512, units=64)),
+    ((2048, 8192, 8192, 1), dict(pair=1, tile_cols=512, units=128)),
+    # less than a wave of wide tiles: 256-wide pairs keep more SMs busy
+    ((1100, 2048, 512, 1), dict(pair=1, tile_cols=256, units=40)),
+    ((256, 9216, 3072, 0), dict(pair=1, tile_cols=128, units=72)),
     # MLP down projection (K 16384, 32 tiles): K in halves over two pairs
     ((1024, 2048, 16384, 0), dict(pair=1, split2=1, tile_cols=256, units=32, grid=128,
                                   k_blocks=128)),
-    # DiT FFN with the GELU epilogue
+    # DiT FFN with the GELU epilogue, and its down projection (K 12288: wide)
     ((8192, 12288, 3072, 2), dict(pair=1, tile_cols=256, units=1536)),
+    ((8192, 3072, 12288, 0), dict(pair=1, split2=0, tile_cols=512, units=192)),
     # 4096-row stack layer (N 640): 160-wide pair tiles, 16 x 4 tiles
     ((4096, 640, 512, 0), dict(pair=1, tile_cols=160, units=64)),
     # the gated epilogues never swap, even at 50 tokens
