@@ -74,8 +74,25 @@ __global__ void gelu_kernel(int M, int H, const uint16_t* u, long ld, const floa
   }
 }
 
+__global__ void gelu_selftest_kernel(const float* x, float* y, long n) {
+  for (long i = blockIdx.x * long(blockDim.x) + threadIdx.x; i < n; i += long(gridDim.x) * blockDim.x)
+    y[i] = gelu_tanh_mul(x[i], 1.0f);
+}
+
 }  // namespace
 }  // namespace frt
+
+extern "C" int frt_selftest_gelu(const float* x, float* y, long n, void* stream) {
+  frt::clear_error();
+  FRT_REQUIRE(n >= 0, FRT_ESHAPE, "n must be >= 0");
+  FRT_REQUIRE(n == 0 || (x && y), FRT_EINVAL, "x and y are required");
+  FRT_REQUIRE(frt::aligned(x, 4) && frt::aligned(y, 4), FRT_EALIGN, "x and y must be 4-byte aligned");
+  if (n == 0) return FRT_OK;
+  const long need = (n + 255) / 256;
+  const int grid = int(need < frt::num_sms() * 8L ? need : frt::num_sms() * 8L);
+  frt::gelu_selftest_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return frt::check_launch("frt_selftest_gelu");
+}
 
 extern "C" int frt_geglu_quant_fp8(int M, int H, const frt_bf16* gu, long ld_gu,
                                    const float* out_scale, frt_e4m3* hid8, float* amax_out,

@@ -192,16 +192,19 @@ __device__ __forceinline__ void rope_rows(const GemmParams& p, int lane, int m_b
   const int h = n / p.hd, d0 = n - h * p.hd;
   if (p.epi != EPI_ROPE || n >= p.N || h >= p.hq + p.hkv) return;
   const int m0 = m_base + (lane >> 3);
-  int b = m0 / p.Mseq, s = m0 - b * p.Mseq;
+  int s = m0 % p.Mseq;
+  const uint16_t* rr = p.rope + long(s) * p.hd + d0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    if (m0 + 4 * i < p.M)
-      rv[i] = __ldg(reinterpret_cast<const uint4*>(p.rope + long(s) * p.hd + d0));
+    if (m0 + 4 * i < p.M) rv[i] = __ldg(reinterpret_cast<const uint4*>(rr));
+    rr += 4 * p.hd;
     s += 4;
-    while (s >= p.Mseq) { s -= p.Mseq; ++b; }
+    while (s >= p.Mseq) { s -= p.Mseq; rr -= long(p.Mseq) * p.hd; }
   }
 }
 
+// The destinations of one unit's rows step by a constant: q rows are token
+// rows (b * M + s), cache rows b * T + P + s jump by T - M where s wraps.
 __device__ __forceinline__ void flush_rows_bf16(const GemmParams& p, const uint8_t* buf, int lane,
                                                 int m_base, int n0, int units,
                                                 const uint4 (&rv)[8]) {
@@ -220,24 +223,30 @@ __device__ __forceinline__ void flush_rows_bf16(const GemmParams& p, const uint8
     } else {  // EPI_ROPE
       const int h = n / p.hd, d0 = n - h * p.hd;
       const bool rot = h < p.hq + p.hkv;
-      int b = m0 / p.Mseq, s = m0 - b * p.Mseq;
+      const int b = m0 / p.Mseq;
+      int s = m0 - b * p.Mseq;
+      uint16_t* dst;
+      long step, wrap;
+      if (h < p.hq) {
+        dst = p.q_out + (long(m0) * p.hq + h) * p.hd + d0;
+        step = 4L * p.hq * p.hd;
+        wrap = 0;
+      } else {
+        const int hh = rot ? h - p.hq : h - p.hq - p.hkv;
+        dst = (rot ? p.k_cache : p.v_cache) + ((long(b) * p.T + p.P + s) * p.hkv + hh) * p.hd + d0;
+        step = 4L * p.hkv * p.hd;
+        wrap = long(p.T - p.Mseq) * p.hkv * p.hd;
+      }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         if (m0 + 4 * i < p.M) {
           uint4 x = stage_get(buf, r0 + 4 * i, u);
-          uint16_t* dst;
-          if (h < p.hq) {
-            dst = p.q_out + ((long(b) * p.Mseq + s) * p.hq + h) * p.hd + d0;
-          } else if (rot) {
-            dst = p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d0;
-          } else {
-            dst = p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq - p.hkv)) * p.hd + d0;
-          }
           if (rot) x = rope_rotate8(x, rv[i]);
           *reinterpret_cast<uint4*>(dst) = x;
         }
+        dst += step;
         s += 4;
-        while (s >= p.Mseq) { s -= p.Mseq; ++b; }
+        while (s >= p.Mseq) { s -= p.Mseq; dst += wrap; }
       }
     }
   }

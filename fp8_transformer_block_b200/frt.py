@@ -111,6 +111,7 @@ _SIGS = {
     "frt_ffn_workspace_size": (_z, [C.POINTER(frt_ffn_desc)]),
     "frt_ffn_layer": (_i, [C.POINTER(frt_ffn_desc), _p]),
     "frt_selftest_bounded_wait": (_i, [_i, _p]),
+    "frt_selftest_gelu": (_i, [_p, _p, _l, _p]),
     "frt_quantize_fp8_static": (_i, [_i, _i, _p, _l, _p, _p, _p, _p]),
     "frt_gelu_quant_fp8": (_i, [_i, _i, _p, _l, _p, _p, _p, _p]),
     "frt_ada_rms_tail": (_i, [_i, _i, _f, _p, _p, _p, _l, _p, _l, _p, _p]),
@@ -336,6 +337,11 @@ def frt_peak_copy(src, dst, nbytes: int, stream=None) -> None:
 def frt_selftest_bounded_wait(timeout_us: int, stream=None) -> int:
     """Returns the status (FRT_ETIMEOUT expected); does not raise."""
     return _lib.frt_selftest_bounded_wait(timeout_us, _stream(stream))
+
+
+def frt_selftest_gelu(x, y, n: int, stream=None) -> None:
+    """y = the device GELU of x (n fp32 values each)."""
+    _check(_lib.frt_selftest_gelu(ptr(x), ptr(y), n, _stream(stream)), "frt_selftest_gelu")
 
 
 def raw_call(name: str, *args) -> int:

@@ -482,6 +482,15 @@ int frt_style_project(int rows, int K, int N, const float* cond, long ld_cond,
  */
 int frt_selftest_bounded_wait(int timeout_us, void* stream);
 
+/*
+ * Evaluates the device GELU the GEGLU and GELU epilogues use:
+ * y[i] = gelu_tanh(x[i]) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
+ * in fp32, for n device floats (x, y 4-byte aligned, n >= 0), so a test can
+ * hold it to an error bound against a higher-precision evaluation.
+ * Asynchronous on `stream`.
+ */
+int frt_selftest_gelu(const float* x, float* y, long n, void* stream);
+
 /* ----------------------------------------------------------------------- */
 /* The library's own peak probes (no counterpart on the pages).             */
 /* ----------------------------------------------------------------------- */

@@ -492,6 +492,30 @@ def test_geglu_fused_epilogue(rt, M, H):
     assert_codes(runtime.u8_host(h1), ref_a, what="standalone GEGLU vs oracle")
 
 
+def test_device_gelu_error_bound(rt):
+    """The device GELU (tanh from the exponential) against an fp64
+    evaluation of the tanh-form GELU: within 5e-7 * max(1, |x|) plus four
+    fp32 ulps of the value over [-12, 12] and at small magnitudes; exactly x
+    once tanh saturates (x >= 10) and signed zero at zero."""
+    frt, runtime, torch = rt
+    x = np.concatenate([np.linspace(-12.0, 12.0, 240001),
+                        [0.0, -0.0, 1e-30, -1e-30, 1e-5, -1e-5, 3e-3, -3e-3]]).astype(np.float32)
+    xd = torch.from_numpy(x).cuda()
+    yd = torch.empty_like(xd)
+    frt.frt_selftest_gelu(xd, yd, x.size)
+    _sync(torch)
+    y = yd.cpu().numpy().astype(np.float64)
+    xx = x.astype(np.float64)
+    ref = 0.5 * xx * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (xx + 0.044715 * xx ** 3)))
+    ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
+    err = np.abs(y - ref)
+    bound = 5e-7 * np.maximum(1.0, np.abs(xx)) + 4 * ulp
+    assert (err <= bound).all(), f"worst {(err / bound).max():.2f} of the bound at x={xx[np.argmax(err / bound)]}"
+    big = xx >= 10
+    assert np.array_equal(y[big], xx[big])
+    assert y[x.size - 8] == 0.0 and np.signbit(yd.cpu().numpy()[x.size - 7])
+
+
 # ------------------------------------------------------------ peak probes --
 def test_peak_probes_run_and_are_plausible(rt):
     frt, runtime, torch = rt
