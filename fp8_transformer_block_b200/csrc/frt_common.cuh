@@ -226,29 +226,34 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// tanh(y) from the exponential, tanh(|y|) = 1 - 2 / (exp(2|y|) + 1) with
-// the sign of y restored, using the hardware exponential and reciprocal
-// (__expf, __fdividef): a few instructions instead of a library tanh.
-// Where |tanh| nears 1 the subtracted term is small and carries only its
-// own relative error, so the result is within about half an ulp there --
-// which is where GELU's 1 + tanh(y) cancels (y < 0) and every bit of tanh
-// counts.  Near 0 the error is a few ulps of 1 in absolute terms, which
-// 1 + tanh absorbs.  |y| > 44 gives exactly +-1 (exp overflows to inf).
-__device__ __forceinline__ float tanh_from_exp(float y) {
-  const float e = __expf(__fmul_rn(2.0f, fabsf(y)));
-  return copysignf(__fsub_rn(1.0f, __fdividef(2.0f, __fadd_rn(e, 1.0f))), y);
-}
-
-// gelu_tanh(g) * u with gelu_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x +
-// 0.044715 x^3))) (the tanh form of Hendrycks & Gimpel's GELU), every step
-// an explicitly rounded fp32 operation; tanh as tanh_from_exp.
-__device__ __forceinline__ float gelu_tanh_mul(float g, float u) {
-  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
-  const float k1 = 0.044715f;
-  const float g3 = __fmul_rn(__fmul_rn(g, g), g);
-  const float inner = __fmul_rn(k0, __fadd_rn(g, __fmul_rn(k1, g3)));
-  const float gl = __fmul_rn(__fmul_rn(0.5f, g), __fadd_rn(1.0f, tanh_from_exp(inner)));
-  return __fmul_rn(gl, u);
+// gelu_tanh(g) * u on two lanes at once, with gelu_tanh(x) = 0.5 x (1 +
+// tanh(sqrt(2/pi) (x + 0.044715 x^3))) (the tanh form of Hendrycks &
+// Gimpel's GELU).  Every multiply and add is an explicitly rounded fp32
+// operation, issued as a paired instruction (each lane rounded exactly as
+// the scalar operation would be).  tanh comes from the exponential:
+// tanh(|y|) = 1 - 2 / (exp(2|y|) + 1), the sign of y restored, with the
+// hardware exponential and reciprocal (__expf, __fdividef) per lane -- a
+// few instructions instead of a library tanh.  Where |tanh| nears 1 the
+// subtracted term is small and carries only its own relative error, so
+// tanh is within about half an ulp there, which is where 1 + tanh(y)
+// cancels (y < 0) and every bit counts; near 0 the error is a few ulps of
+// 1 in absolute terms, which 1 + tanh absorbs; |y| > 44 gives exactly +-1
+// (the exponential overflows to inf).
+__device__ __forceinline__ uint64_t gelu_tanh_mul2(uint64_t g, uint64_t u) {
+  const uint64_t k0 = f2_pack(0.7978845608028654f, 0.7978845608028654f);
+  const uint64_t k1 = f2_pack(0.044715f, 0.044715f);
+  const uint64_t one = f2_pack(1.0f, 1.0f), two = f2_pack(2.0f, 2.0f);
+  const uint64_t half = f2_pack(0.5f, 0.5f);
+  const uint64_t g3 = mul2(mul2(g, g), g);
+  const uint64_t inner = mul2(k0, add2(g, mul2(k1, g3)));
+  // tanh_from_exp per lane: |y|, 2|y|, exp, + 1, 2 / ., 1 - ., sign of y
+  const uint64_t ay = inner & 0x7FFFFFFF7FFFFFFFull;
+  const uint64_t x2 = mul2(two, ay);
+  const uint64_t e1 = add2(f2_pack(__expf(f2_lo(x2)), __expf(f2_hi(x2))), one);
+  const uint64_t r = f2_pack(__fdividef(2.0f, f2_lo(e1)), __fdividef(2.0f, f2_hi(e1)));
+  const uint64_t t = sub2(one, r) | (inner & 0x8000000080000000ull);  // t >= +0 before the sign
+  const uint64_t gl = mul2(mul2(half, g), add2(one, t));
+  return mul2(gl, u);
 }
 
 }  // namespace frt

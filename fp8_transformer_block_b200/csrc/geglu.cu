@@ -6,7 +6,7 @@
 // quantized with the down projection's static input scale) and the bind
 // check that the FFN activation is the tanh-approximate GELU.
 // gelu_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), the tanh
-// form of Hendrycks & Gimpel's GELU (frt::gelu_tanh_mul, shared with the
+// form of Hendrycks & Gimpel's GELU (frt::gelu_tanh_mul2, shared with the
 // fused GEMM epilogue so both forms give the same codes).
 #include "frt_common.cuh"
 
@@ -30,10 +30,11 @@ __global__ void geglu_kernel(int M, int H, const uint16_t* gu, long ld, const fl
     unpack8(__ldg(reinterpret_cast<const uint4*>(gu + m * ld + 8 * c)), gv);
     unpack8(__ldg(reinterpret_cast<const uint4*>(gu + m * ld + H + 8 * c)), uv);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float h = gelu_tanh_mul(gv[j], uv[j]);
-      mx = fmaxf(mx, fabsf(h));
-      q[j] = __fmul_rn(h, inv_os);
+    for (int j = 0; j < 8; j += 2) {
+      const uint64_t h = gelu_tanh_mul2(f2_pack(gv[j], gv[j + 1]), f2_pack(uv[j], uv[j + 1]));
+      mx = absmax2(mx, h);
+      q[j] = __fmul_rn(f2_lo(h), inv_os);
+      q[j + 1] = __fmul_rn(f2_hi(h), inv_os);
     }
     *reinterpret_cast<uint2*>(hid8 + m * H + 8 * c) = pack8_e4m3(q);
   }
@@ -61,10 +62,11 @@ __global__ void gelu_kernel(int M, int H, const uint16_t* u, long ld, const floa
     float uv[8], q[8];
     unpack8(__ldg(reinterpret_cast<const uint4*>(u + m * ld + 8 * c)), uv);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float h = gelu_tanh_mul(uv[j], 1.0f);
-      mx = fmaxf(mx, fabsf(h));
-      q[j] = __fmul_rn(h, inv_os);
+    for (int j = 0; j < 8; j += 2) {
+      const uint64_t h = gelu_tanh_mul2(f2_pack(uv[j], uv[j + 1]), f2_pack(1.0f, 1.0f));
+      mx = absmax2(mx, h);
+      q[j] = __fmul_rn(f2_lo(h), inv_os);
+      q[j + 1] = __fmul_rn(f2_hi(h), inv_os);
     }
     *reinterpret_cast<uint2*>(hid8 + m * H + 8 * c) = pack8_e4m3(q);
   }
@@ -74,9 +76,17 @@ __global__ void gelu_kernel(int M, int H, const uint16_t* u, long ld, const floa
   }
 }
 
+// The device GELU on pairs of elements (an odd tail paired with 0).
 __global__ void gelu_selftest_kernel(const float* x, float* y, long n) {
-  for (long i = blockIdx.x * long(blockDim.x) + threadIdx.x; i < n; i += long(gridDim.x) * blockDim.x)
-    y[i] = gelu_tanh_mul(x[i], 1.0f);
+  const long pairs = (n + 1) / 2;
+  for (long i = blockIdx.x * long(blockDim.x) + threadIdx.x; i < pairs;
+       i += long(gridDim.x) * blockDim.x) {
+    const bool two = 2 * i + 1 < n;
+    const uint64_t h =
+        gelu_tanh_mul2(f2_pack(x[2 * i], two ? x[2 * i + 1] : 0.0f), f2_pack(1.0f, 1.0f));
+    y[2 * i] = f2_lo(h);
+    if (two) y[2 * i + 1] = f2_hi(h);
+  }
 }
 
 }  // namespace
@@ -88,7 +98,7 @@ extern "C" int frt_selftest_gelu(const float* x, float* y, long n, void* stream)
   FRT_REQUIRE(n == 0 || (x && y), FRT_EINVAL, "x and y are required");
   FRT_REQUIRE(frt::aligned(x, 4) && frt::aligned(y, 4), FRT_EALIGN, "x and y must be 4-byte aligned");
   if (n == 0) return FRT_OK;
-  const long need = (n + 255) / 256;
+  const long need = ((n + 1) / 2 + 255) / 256;
   const int grid = int(need < frt::num_sms() * 8L ? need : frt::num_sms() * 8L);
   frt::gelu_selftest_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return frt::check_launch("frt_selftest_gelu");

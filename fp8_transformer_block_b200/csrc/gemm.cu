@@ -344,16 +344,27 @@ __device__ __forceinline__ void warp_rows_epilogue(const GemmParams& p, uint8_t*
         load(c, q);
         if (!geglu && c == ce - 1) done();
         scale_bias32(p, q, bg, alpha);
+        const uint64_t inv2 = f2_pack(inv_os, inv_os);
         if (geglu) {
           float z[32];
           load(c + 4, z);
           if (c == ce - 1) done();
           scale_bias32(p, z, bu, alpha);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) q[j] = __fmul_rn(gelu_tanh_mul(q[j], z[j]), inv_os);
+          for (int j = 0; j < 32; j += 2) {
+            const uint64_t h = mul2(gelu_tanh_mul2(f2_pack(q[j], q[j + 1]), f2_pack(z[j], z[j + 1])),
+                                    inv2);
+            q[j] = f2_lo(h);
+            q[j + 1] = f2_hi(h);
+          }
         } else {
+          const uint64_t one = f2_pack(1.0f, 1.0f);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) q[j] = __fmul_rn(gelu_tanh_mul(q[j], 1.0f), inv_os);
+          for (int j = 0; j < 32; j += 2) {
+            const uint64_t h = mul2(gelu_tanh_mul2(f2_pack(q[j], q[j + 1]), one), inv2);
+            q[j] = f2_lo(h);
+            q[j + 1] = f2_hi(h);
+          }
         }
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
