@@ -124,6 +124,12 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+// a * b + c per lane with one rounding (fused multiply-add)
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
 // Two bf16 in one 32-bit word (lo in the low half) -> an fp32 pair.
 __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
   return (uint64_t(w & 0xFFFF0000u) << 32) | uint64_t(w << 16);
@@ -228,30 +234,38 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // gelu_tanh(g) * u on two lanes at once, with gelu_tanh(x) = 0.5 x (1 +
 // tanh(sqrt(2/pi) (x + 0.044715 x^3))) (the tanh form of Hendrycks &
-// Gimpel's GELU).  Every multiply and add is an explicitly rounded fp32
-// operation, issued as a paired instruction (each lane rounded exactly as
-// the scalar operation would be).  tanh comes from the exponential:
-// tanh(|y|) = 1 - 2 / (exp(2|y|) + 1), the sign of y restored, with the
-// hardware exponential and reciprocal (__expf, __fdividef) per lane -- a
-// few instructions instead of a library tanh.  Where |tanh| nears 1 the
-// subtracted term is small and carries only its own relative error, so
-// tanh is within about half an ulp there, which is where 1 + tanh(y)
-// cancels (y < 0) and every bit counts; near 0 the error is a few ulps of
-// 1 in absolute terms, which 1 + tanh absorbs; |y| > 44 gives exactly +-1
-// (the exponential overflows to inf).
+// Gimpel's GELU).  Every multiply and add of that formula is an explicitly
+// rounded fp32 operation, issued as a paired instruction (each lane rounded
+// exactly as the scalar operation would be).
+// tanh comes from one exponential per lane: with E = exp(-2|y|) (the
+// hardware exponential, __expf), tanh(|y|) = 1 - w, w = 2E / (1 + E), and
+// the sign of y restored.  1 / (1 + E), an argument in [1, 2], is three
+// Newton steps r <- r + r (1 - d r) from the linear seed 24/17 - 8/17 d
+// (relative error at most 1/17, squared by each step: within about one ulp
+// after three), so the special-function unit does one operation per lane
+// instead of two.  Where |tanh| nears 1, w is small and carries only its
+// own relative error, so tanh is within about one ulp there -- which is
+// where 1 + tanh(y) cancels (y < 0) and every bit counts; near 0 the error
+// is a few ulps of 1 in absolute terms, which 1 + tanh absorbs; large |y|
+// gives exactly +-1 (E underflows to 0).
 __device__ __forceinline__ uint64_t gelu_tanh_mul2(uint64_t g, uint64_t u) {
   const uint64_t k0 = f2_pack(0.7978845608028654f, 0.7978845608028654f);
   const uint64_t k1 = f2_pack(0.044715f, 0.044715f);
   const uint64_t one = f2_pack(1.0f, 1.0f), two = f2_pack(2.0f, 2.0f);
   const uint64_t half = f2_pack(0.5f, 0.5f);
+  constexpr uint64_t kSign = 0x8000000080000000ull;
   const uint64_t g3 = mul2(mul2(g, g), g);
   const uint64_t inner = mul2(k0, add2(g, mul2(k1, g3)));
-  // tanh_from_exp per lane: |y|, 2|y|, exp, + 1, 2 / ., 1 - ., sign of y
-  const uint64_t ay = inner & 0x7FFFFFFF7FFFFFFFull;
-  const uint64_t x2 = mul2(two, ay);
-  const uint64_t e1 = add2(f2_pack(__expf(f2_lo(x2)), __expf(f2_hi(x2))), one);
-  const uint64_t r = f2_pack(__fdividef(2.0f, f2_lo(e1)), __fdividef(2.0f, f2_hi(e1)));
-  const uint64_t t = sub2(one, r) | (inner & 0x8000000080000000ull);  // t >= +0 before the sign
+  // tanh(|inner|) = 1 - 2E / (1 + E), E = exp(-2|inner|)
+  const uint64_t x2 = mul2(two, inner | kSign);  // -2|y|
+  const uint64_t E = f2_pack(__expf(f2_lo(x2)), __expf(f2_hi(x2)));
+  const uint64_t d = add2(E, one);
+  uint64_t r = fma2(f2_pack(-8.0f / 17.0f, -8.0f / 17.0f), d,
+                    f2_pack(24.0f / 17.0f, 24.0f / 17.0f));
+#pragma unroll
+  for (int i = 0; i < 3; ++i) r = fma2(r, fma2(d ^ kSign, r, one), r);
+  const uint64_t w = mul2(mul2(two, E), r);
+  const uint64_t t = sub2(one, w) | (inner & kSign);  // 1 - w >= +0 before the sign
   const uint64_t gl = mul2(mul2(half, g), add2(one, t));
   return mul2(gl, u);
 }
