@@ -761,7 +761,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     constexpr int LNI = CLUSTER ? BN * (BMT / LW) / 128 : 1;  // items per thread
     ItemPlan<LW> lplan[LNI];
     const uint32_t crank = CLUSTER ? cluster_ctarank() : 0u;
-    if (CLUSTER && crank == 0 && blockIdx.x < unsigned(p.units)) {
+    if constexpr (CLUSTER) if (crank == 0 && blockIdx.x < unsigned(p.units)) {
       const int tile = int(blockIdx.x) / p.splits;
       const int ta = tile % p.a_tiles, tb = tile / p.a_tiles;
 #pragma unroll
@@ -792,7 +792,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + uint32_t(ab * BN) + (uint32_t(32 * q) << 16);
-      if (CLUSTER) {
+      if constexpr (CLUSTER) {
         // one unit per CTA: stage this rank's partial (the leader's MMA
         // completion has already told the other ranks its ring is free)
         cluster_wait();
@@ -842,34 +842,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = 0.0f;
                 if (!valid) return;
-                // two splits per step keep 16 loads in flight per thread
-                int s = 0;
-                for (; s + 1 < p.splits; s += 2) {
+                // the splits in order, eight 16-byte loads in flight per step
+#pragma unroll 1
+                for (int s = 0; s < p.splits; ++s) {
                   const float4* s0 =
                       reinterpret_cast<const float4*>(base + long(s) * (BMT * BN) + 32 * c);
-                  const float4* s1 =
-                      reinterpret_cast<const float4*>(base + long(s + 1) * (BMT * BN) + 32 * c);
-                  float4 f0[8], f1[8];
+                  float4 f[8];
 #pragma unroll
-                  for (int k = 0; k < 8; ++k) { f0[k] = __ldcg(s0 + k); f1[k] = __ldcg(s1 + k); }
+                  for (int k = 0; k < 8; ++k) f[k] = __ldcg(s0 + k);
 #pragma unroll
                   for (int k = 0; k < 8; ++k) {
-                    v[4 * k] = __fadd_rn(__fadd_rn(v[4 * k], f0[k].x), f1[k].x);
-                    v[4 * k + 1] = __fadd_rn(__fadd_rn(v[4 * k + 1], f0[k].y), f1[k].y);
-                    v[4 * k + 2] = __fadd_rn(__fadd_rn(v[4 * k + 2], f0[k].z), f1[k].z);
-                    v[4 * k + 3] = __fadd_rn(__fadd_rn(v[4 * k + 3], f0[k].w), f1[k].w);
-                  }
-                }
-                if (s < p.splits) {
-                  const float4* s0 =
-                      reinterpret_cast<const float4*>(base + long(s) * (BMT * BN) + 32 * c);
-#pragma unroll
-                  for (int k = 0; k < 8; ++k) {
-                    const float4 f = __ldcg(s0 + k);
-                    v[4 * k] = __fadd_rn(v[4 * k], f.x);
-                    v[4 * k + 1] = __fadd_rn(v[4 * k + 1], f.y);
-                    v[4 * k + 2] = __fadd_rn(v[4 * k + 2], f.z);
-                    v[4 * k + 3] = __fadd_rn(v[4 * k + 3], f.w);
+                    v[4 * k] = __fadd_rn(v[4 * k], f[k].x);
+                    v[4 * k + 1] = __fadd_rn(v[4 * k + 1], f[k].y);
+                    v[4 * k + 2] = __fadd_rn(v[4 * k + 2], f[k].z);
+                    v[4 * k + 3] = __fadd_rn(v[4 * k + 3], f[k].w);
                   }
                 }
               },
@@ -879,7 +865,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         named_bar_sync(1, 128);
       }
     }
-    if (CLUSTER) {
+    if constexpr (CLUSTER) {
       if (!cwaited) cluster_wait();
       constexpr uint32_t TB = uint32_t(t_tile_bytes<SWAP, BMT, BN>());
       const bool fits = uint32_t(p.splits - 1) * TB <= uint32_t(STAGES * (A_BYTES + B_BYTES));
