@@ -21,8 +21,16 @@ struct PrefixArgs {
   long units;  // 2 * B * P * hkv * hd / 8 sixteen-byte units
 };
 
-// Copy unit u (one 8-element chunk of one key or value row).
-__device__ __forceinline__ void prefix_unit(const PrefixArgs& a, long u) {
+// Unit u (one 8-element chunk of one key or value row): where it lands in
+// the chain's cache, and the source data it needs (a key chunk gathers two
+// half chunks of the host row).
+struct PrefixUnit {
+  uint16_t* dst;
+  uint2 lo, hi;   // key gather halves, or the value chunk's two halves
+  bool gather;
+};
+
+__device__ __forceinline__ PrefixUnit prefix_load(const PrefixArgs& a, long u) {
   const int hd8 = a.hd / 8;
   const int which = int(u & 1);
   u >>= 1;
@@ -34,23 +42,55 @@ __device__ __forceinline__ void prefix_unit(const PrefixArgs& a, long u) {
   const int b = int(u / a.P);
   const long src_row = ((long(b) * a.hkv + h) * a.T_src + p) * a.hd;
   const long dst = ((long(b) * a.T + p) * a.hkv + h) * a.hd + 8 * c;
-  if (which == 1 || !a.interleave) {
-    const uint16_t* src = (which ? a.pv : a.pk) + src_row + 8 * c;
-    uint16_t* d = (which ? a.v_cache : a.k_cache) + dst;
-    *reinterpret_cast<uint4*>(d) = __ldg(reinterpret_cast<const uint4*>(src));
+  PrefixUnit r;
+  r.gather = which == 0 && a.interleave;
+  r.dst = (which ? a.v_cache : a.k_cache) + dst;
+  if (!r.gather) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>((which ? a.pv : a.pk) + src_row + 8 * c));
+    r.lo = make_uint2(v.x, v.y);
+    r.hi = make_uint2(v.z, v.w);
   } else {
     // destination slots 8c..8c+7 take sources 4c..4c+3 (even slots) and
     // hd/2 + 4c .. +3 (odd slots)
-    const uint2 lo = __ldg(reinterpret_cast<const uint2*>(a.pk + src_row + 4 * c));
-    const uint2 hi = __ldg(reinterpret_cast<const uint2*>(a.pk + src_row + a.hd / 2 + 4 * c));
-    const uint32_t l[2] = {lo.x, lo.y}, m[2] = {hi.x, hi.y};
-    uint32_t o[4];
+    r.lo = __ldg(reinterpret_cast<const uint2*>(a.pk + src_row + 4 * c));
+    r.hi = __ldg(reinterpret_cast<const uint2*>(a.pk + src_row + a.hd / 2 + 4 * c));
+  }
+  return r;
+}
+
+__device__ __forceinline__ void prefix_store(const PrefixUnit& r) {
+  if (!r.gather) {
+    *reinterpret_cast<uint4*>(r.dst) = make_uint4(r.lo.x, r.lo.y, r.hi.x, r.hi.y);
+    return;
+  }
+  const uint32_t l[2] = {r.lo.x, r.lo.y}, m[2] = {r.hi.x, r.hi.y};
+  uint32_t o[4];
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      o[2 * k] = (l[k] & 0xFFFFu) | (m[k] << 16);
-      o[2 * k + 1] = (l[k] >> 16) | (m[k] & 0xFFFF0000u);
-    }
-    *reinterpret_cast<uint4*>(a.k_cache + dst) = make_uint4(o[0], o[1], o[2], o[3]);
+  for (int k = 0; k < 2; ++k) {
+    o[2 * k] = (l[k] & 0xFFFFu) | (m[k] << 16);
+    o[2 * k + 1] = (l[k] >> 16) | (m[k] & 0xFFFF0000u);
+  }
+  *reinterpret_cast<uint4*>(r.dst) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Copy unit u.
+__device__ __forceinline__ void prefix_unit(const PrefixArgs& a, long u) {
+  prefix_store(prefix_load(a, u));
+}
+
+// Copy units first, first + stride, ... (< a.units): every load of up to
+// kPrefixBatch units is issued before the first store, so a thread with
+// several units pays one memory round trip per batch, not one per unit.
+constexpr int kPrefixBatch = 8;
+__device__ __forceinline__ void prefix_units_strided(const PrefixArgs& a, long first, long stride) {
+  for (long u0 = first; u0 < a.units; u0 += stride * kPrefixBatch) {
+    PrefixUnit r[kPrefixBatch];
+#pragma unroll
+    for (int i = 0; i < kPrefixBatch; ++i)
+      if (u0 + i * stride < a.units) r[i] = prefix_load(a, u0 + i * stride);
+#pragma unroll
+    for (int i = 0; i < kPrefixBatch; ++i)
+      if (u0 + i * stride < a.units) prefix_store(r[i]);
   }
 }
 

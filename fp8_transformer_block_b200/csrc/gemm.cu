@@ -404,6 +404,106 @@ __device__ __forceinline__ void warp_rows_epilogue(const GemmParams& p, uint8_t*
   }
 }
 
+// The single-CTA kernel's epilogue (normal orientation): each thread writes
+// its own accumulator row m straight from registers, columns col0 + 32c for
+// chunks c < nch (GEGLU: gate chunks c < 4 with up chunks c + 4, output
+// columns out0 + 32c).  That kernel runs at most one tile per CTA (larger
+// tile counts go to CTA pairs), so a staged write-back would only add a
+// round trip to a latency-bound tile.  The same arithmetic as
+// warp_rows_epilogue; each chunk's bias and rope pieces are requested
+// before its accumulators are read.
+template <class Load, class Done>
+__device__ __forceinline__ void rows_direct_epilogue(const GemmParams& p, int m, int col0, int nch,
+                                                     int out0, float alpha, Load load,
+                                                     Done done) {
+  const bool ok = m < p.M;
+  if (p.epi == EPI_GEGLU || p.epi == EPI_GELU) {
+    const bool geglu = p.epi == EPI_GEGLU;
+    const float inv_os = __frcp_rn(__ldg(p.out_scale));
+    const uint64_t inv2 = f2_pack(inv_os, inv_os);
+    const int nout = geglu ? 4 : nch;
+#pragma unroll 1
+    for (int c = 0; c < nout; ++c) {
+      uint4 bg[4], bu[4];
+      load_bias32(p, col0 + 32 * c, bg);
+      if (geglu) load_bias32(p, col0 + 128 + 32 * c, bu);
+      float q[32];
+      load(c, q);
+      if (!geglu && c == nout - 1) done();
+      scale_bias32(p, q, bg, alpha);
+      if (geglu) {
+        float z[32];
+        load(c + 4, z);
+        if (c == nout - 1) done();
+        scale_bias32(p, z, bu, alpha);
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const uint64_t h =
+              mul2(gelu_tanh_mul2(f2_pack(q[j], q[j + 1]), f2_pack(z[j], z[j + 1])), inv2);
+          q[j] = f2_lo(h);
+          q[j + 1] = f2_hi(h);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const uint64_t h = mul2(gelu_tanh_mul2(f2_pack(q[j], q[j + 1]), f2_pack(1.0f, 1.0f)),
+                                  inv2);
+          q[j] = f2_lo(h);
+          q[j + 1] = f2_hi(h);
+        }
+      }
+      if (ok) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + long(m) * p.ldo +
+                                              (geglu ? out0 : col0) + 32 * c);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          float a8[8], b8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) { a8[j] = q[16 * k + j]; b8[j] = q[16 * k + 8 + j]; }
+          const uint2 lo = pack8_e4m3(a8), hi = pack8_e4m3(b8);
+          dst[k] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
+      }
+    }
+    return;
+  }
+  const uint64_t alpha2 = f2_pack(alpha, alpha);
+#pragma unroll 1
+  for (int c = 0; c < nch; ++c) {
+    const int n = col0 + 32 * c;
+    uint4 b4[4], rv[4];
+    load_bias32(p, n, b4);
+    const int h = p.epi == EPI_ROPE ? n / p.hd : 0, d0 = p.epi == EPI_ROPE ? n - h * p.hd : 0;
+    const bool rot = p.epi == EPI_ROPE && h < p.hq + p.hkv;
+    const int s = ok && p.epi == EPI_ROPE ? m % p.Mseq : 0;
+    if (rot && ok) {
+      const uint4* rr = reinterpret_cast<const uint4*>(p.rope + long(s) * p.hd + d0);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) rv[k] = __ldg(rr + k);
+    }
+    float v[32];
+    load(c, v);
+    if (c == nch - 1) done();
+    if (!ok) continue;
+    uint16_t* dst;
+    if (p.epi == EPI_BF16) {
+      dst = static_cast<uint16_t*>(p.out) + long(m) * p.ldo + n;
+    } else {  // the 32 columns lie inside one head (hd % 32 == 0)
+      const int b = m / p.Mseq;
+      dst = h < p.hq ? p.q_out + (long(m) * p.hq + h) * p.hd + d0
+          : h < p.hq + p.hkv
+              ? p.k_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq)) * p.hd + d0
+              : p.v_cache + ((long(b) * p.T + p.P + s) * p.hkv + (h - p.hq - p.hkv)) * p.hd + d0;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint4 x = scale_bias_pack8(v + 8 * k, b4[k], alpha2, p.bias);
+      if (rot) x = rope_rotate8(x, rv[k]);
+      reinterpret_cast<uint4*>(dst)[k] = x;
+    }
+  }
+}
+
 // TMEM lane holding accumulator row r of an MMA with M = BMT rows: all 128
 // lanes for M = 128; for M = 64 the rows fill the first 16 lanes of each
 // 32-lane quarter (rows 16q .. 16q+15 in lanes 32q .. 32q+15).  The epilogue
@@ -446,20 +546,19 @@ __device__ __forceinline__ void emit_swap_items(const GemmParams& p, int ta, int
 // (32 columns of this thread's TMEM lane); it is called warp-uniformly.
 // done() runs once every chunk has been loaded (it releases the TMEM
 // accumulator when the chunks come from TMEM).
-// Normal orientation: the warp's rows go through warp_rows_epilogue, staged
-// in the warp's buffer ebuf.  Swapped orientation: the chunks are staged in
+// Normal orientation: each thread's row through rows_direct_epilogue.
+// Swapped orientation: the chunks are staged in
 // the shared-memory tile T (fp32 [BMT output columns][BN tokens], row
 // stride BN + 4) and read back transposed, token-major, so neighbouring
 // threads write neighbouring 16-byte pieces of one token row.
 template <bool SWAP, int BMT, int BN, class Load, class Done>
 __device__ __forceinline__ void tile_epilogue(const GemmParams& p, int ta, int tb, int q, int lane,
-                                              float alpha, float* T, uint8_t* ebuf, Load load,
-                                              Done done) {
+                                              float alpha, float* T, Load load, Done done) {
   if (!SWAP) {
     int c_last = BN / 32 - 1;
     while (c_last > 0 && tb * BN + 32 * c_last >= p.N) --c_last;
-    warp_rows_epilogue(p, ebuf, lane, ta * BMT + 32 * q, tb * BN, 0,
-                       p.epi == EPI_GEGLU ? 4 : c_last + 1, tb * 128, alpha, load, done);
+    rows_direct_epilogue(p, ta * BMT + 32 * q + lane, tb * BN, c_last + 1, tb * 128, alpha, load,
+                         done);
     return;
   }
   constexpr int TS = BMT + 4;
@@ -512,16 +611,9 @@ __host__ __device__ constexpr int t_tile_bytes() {
   return SWAP ? BN * (BMT + 4) * 4 : 0;
 }
 
-// normal orientation: the four epilogue warps' row staging buffers
-template <bool SWAP>
-__host__ __device__ constexpr int epi_stage_total() {
-  return SWAP ? 0 : 4 * kEpiStageBytes;
-}
-
 template <bool SWAP, int BMT, int BN, int STAGES>
 __host__ __device__ constexpr int smem_total() {
-  return STAGES * (BMT * BK + BN * BK) + t_tile_bytes<SWAP, BMT, BN>() + epi_stage_total<SWAP>() +
-         1024 + 512;
+  return STAGES * (BMT * BK + BN * BK) + t_tile_bytes<SWAP, BMT, BN>() + 1024 + 512;
 }
 
 // CLUSTER: the p.splits K-splits of a tile run as one thread-block cluster
@@ -550,8 +642,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
   float* T = reinterpret_cast<float*>(sB + STAGES * B_BYTES);
-  uint8_t* ebuf_base = sB + STAGES * B_BYTES + t_tile_bytes<SWAP, BMT, BN>();
-  uint64_t* full = reinterpret_cast<uint64_t*>(ebuf_base + epi_stage_total<SWAP>());
+  uint64_t* full =
+      reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES + t_tile_bytes<SWAP, BMT, BN>());
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -750,7 +842,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         tma_load_2d(sB + i * B_BYTES, &tmB, &full[i], (kb0 + i) * BK, tb * BN);
     }
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint8_t* ebuf = ebuf_base + (warp - 2) * kEpiStageBytes;  // normal orientation only
     const float alpha = __fmul_rn(__ldg(p.act_scale), __ldg(p.w_scale));
     const int row = acc_row<BMT>(q, lane);
     const bool valid = acc_row_valid<BMT>(lane);
@@ -809,7 +900,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       };
       if (p.splits == 1) {
         tile_epilogue<SWAP, BMT, BN>(
-            p, ta, tb, q, lane, alpha, T, ebuf,
+            p, ta, tb, q, lane, alpha, T,
             [&](int c, float (&v)[32]) { tmem_ld32(tbase + 32 * c, v); }, release_tmem);
       } else {
         // spill this split's fp32 partial, accumulator-row major
@@ -837,7 +928,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           __threadfence();
           const float* base = p.partials + long(tile) * p.splits * (BMT * BN) + long(row) * BN;
           tile_epilogue<SWAP, BMT, BN>(
-              p, ta, tb, q, lane, alpha, T, ebuf,
+              p, ta, tb, q, lane, alpha, T,
               [&](int c, float (&v)[32]) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = 0.0f;

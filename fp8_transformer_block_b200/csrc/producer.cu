@@ -75,9 +75,8 @@ __device__ __forceinline__ float row_sum(float v, int G, float* red) {
 __device__ __forceinline__ bool prefix_block(const ProducerArgs& a) {
   if (int(blockIdx.x) < a.row_blocks) return false;
   const long nb = long(gridDim.x) - a.row_blocks;
-  for (long u = (long(blockIdx.x) - a.row_blocks) * blockDim.x + threadIdx.x; u < a.pre.units;
-       u += nb * blockDim.x)
-    prefix_unit(a.pre, u);
+  prefix_units_strided(a.pre, (long(blockIdx.x) - a.row_blocks) * blockDim.x + threadIdx.x,
+                       nb * blockDim.x);
   return true;
 }
 

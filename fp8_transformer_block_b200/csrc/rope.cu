@@ -102,13 +102,12 @@ int launch_split(const SplitArgs& a, cudaStream_t s) {
                     dim3(kSplitThreads), 0, s, a);
 }
 
-// The prefix copy alone: 16-byte units over a grid sized to the SM count.
+// The prefix copy alone: 16-byte units over a grid sized to the SM count,
+// each thread's loads issued before its stores.
 __global__ void prefix_copy_kernel(PrefixArgs a) {
   pdl_trigger();
   pdl_wait();
-  for (long g = blockIdx.x * long(blockDim.x) + threadIdx.x; g < a.units;
-       g += long(gridDim.x) * blockDim.x)
-    prefix_unit(a, g);
+  prefix_units_strided(a, blockIdx.x * long(blockDim.x) + threadIdx.x, long(gridDim.x) * blockDim.x);
 }
 
 int launch_prefix(const PrefixArgs& a, cudaStream_t s) {
