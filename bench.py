@@ -64,11 +64,11 @@ KERNEL_SOURCES = {
     "style": ("style.cu", "frt_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("vla_action_expert", "gemm_rope_kv"): (5_428_309, "37cca62b76d214c9"),
-    ("video_dit", "gemm_rope_kv"): (156_936_192, "37cca62b76d214c9"),
-    ("gateup_mlp", "gemm_gateup_geglu"): (72_675_328, "37cca62b76d214c9"),
-    ("style_stack18", "style_project"): (58_491_392, "aefda1df19f33ba3"),
-    ("style_vla18", "style_project"): (935_920_640, "aefda1df19f33ba3"),
+    ("vla_action_expert", "gemm_rope_kv"): (5_428_224, "b5f3b77dce68174e"),
+    ("video_dit", "gemm_rope_kv"): (165_660_928, "b5f3b77dce68174e"),
+    ("gateup_mlp", "gemm_gateup_geglu"): (73_067_264, "b5f3b77dce68174e"),
+    ("style_stack18", "style_project"): (58_446_592 + 512, "164dc7c9f25cad55"),
+    ("style_vla18", "style_project"): (932_188_672 + 466_176, "164dc7c9f25cad55"),
 }
 
 
