@@ -232,42 +232,50 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// gelu_tanh(g) * u on two lanes at once, with gelu_tanh(x) = 0.5 x (1 +
-// tanh(sqrt(2/pi) (x + 0.044715 x^3))) (the tanh form of Hendrycks &
-// Gimpel's GELU).  Every multiply and add of that formula is an explicitly
-// rounded fp32 operation, issued as a paired instruction (each lane rounded
-// exactly as the scalar operation would be).
-// tanh comes from one exponential per lane: with E = exp(-2|y|) (the
-// hardware exponential, __expf), tanh(|y|) = 1 - w, w = 2E / (1 + E), and
-// the sign of y restored.  1 / (1 + E), an argument in [1, 2], is three
-// Newton steps r <- r + r (1 - d r) from the linear seed 24/17 - 8/17 d
-// (relative error at most 1/17, squared by each step: within about one ulp
-// after three), so the special-function unit does one operation per lane
-// instead of two.  Where |tanh| nears 1, w is small and carries only its
-// own relative error, so tanh is within about one ulp there -- which is
-// where 1 + tanh(y) cancels (y < 0) and every bit counts; near 0 the error
-// is a few ulps of 1 in absolute terms, which 1 + tanh absorbs; large |y|
-// gives exactly +-1 (E underflows to 0).
-__device__ __forceinline__ uint64_t gelu_tanh_mul2(uint64_t g, uint64_t u) {
-  const uint64_t k0 = f2_pack(0.7978845608028654f, 0.7978845608028654f);
-  const uint64_t k1 = f2_pack(0.044715f, 0.044715f);
-  const uint64_t one = f2_pack(1.0f, 1.0f), two = f2_pack(2.0f, 2.0f);
-  const uint64_t half = f2_pack(0.5f, 0.5f);
+// c * gelu_tanh(g) [* u] on two lanes at once, with gelu_tanh(x) = 0.5 x
+// (1 + tanh(y)), y = sqrt(2/pi) (x + 0.044715 x^3) (the tanh form of
+// Hendrycks & Gimpel's GELU), every step an explicitly rounded fp32
+// operation issued as a paired instruction.  half_c holds 0.5 c in both
+// lanes (c: the output scale's reciprocal, or 1).
+//   * -2 log2(e) y = g (A0 + A1 g^2), the constants folded (one fma, one
+//     multiply); the hardware base-2 exponential of 1 - 2 log2(e) |y| gives
+//     2E directly, E = exp(-2|y|) (ex2.approx.ftz: 0 once E underflows);
+//   * r = 1 / (1 + E), an argument d in [1, 2]: two Newton steps r <- r + r
+//     (1 - d r) from the minimax quadratic seed (70 - 48 d + 32 d^2 / 3) / 33
+//     (relative error at most 1/99, squared by each step: within one ulp
+//     after two, and exactly 1 at d = 1);
+//   * tanh|y| = 1 - 2E r, its sign that of y (= that of g), then 1 + tanh(y)
+//     formed as the fp32 formula 0.5 g (1 + tanh(y)) forms it -- cancelling
+//     where y << 0 just as that evaluation does (an accurate 2E / (1 + E)
+//     there moves e4m3 codes away from it);
+//   * gelu_one_plus_tanh2 returns 1 + tanh(y); gelu_tanh_scaled2 the result
+//     (0.5 c g) (1 + tanh y) [u]: exactly c g once tanh saturates (E = 0), a
+//     zero of g's sign at g = +-0.
+__device__ __forceinline__ uint64_t gelu_one_plus_tanh2(uint64_t g) {
+  constexpr float kA0 = -2.0f * 0.7978845608028654f * 1.4426950408889634f;
+  constexpr float kA1 = -2.0f * 0.7978845608028654f * 0.044715f * 1.4426950408889634f;
+  const uint64_t one = f2_pack(1.0f, 1.0f);
   constexpr uint64_t kSign = 0x8000000080000000ull;
-  const uint64_t g3 = mul2(mul2(g, g), g);
-  const uint64_t inner = mul2(k0, add2(g, mul2(k1, g3)));
-  // tanh(|inner|) = 1 - 2E / (1 + E), E = exp(-2|inner|)
-  const uint64_t x2 = mul2(two, inner | kSign);  // -2|y|
-  const uint64_t E = f2_pack(__expf(f2_lo(x2)), __expf(f2_hi(x2)));
-  const uint64_t d = add2(E, one);
-  uint64_t r = fma2(f2_pack(-8.0f / 17.0f, -8.0f / 17.0f), d,
-                    f2_pack(24.0f / 17.0f, 24.0f / 17.0f));
+  const uint64_t q = fma2(mul2(g, g), f2_pack(kA1, kA1), f2_pack(kA0, kA0));
+  const uint64_t x = add2(mul2(q, g) | kSign, one);  // 1 - 2 log2(e) |y|
+  float e_lo, e_hi;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e_lo) : "f"(f2_lo(x)));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e_hi) : "f"(f2_hi(x)));
+  const uint64_t e2 = f2_pack(e_lo, e_hi);  // 2E
+  const uint64_t d = fma2(e2, f2_pack(0.5f, 0.5f), one);
+  uint64_t r = fma2(fma2(d, f2_pack(32.0f / 99.0f, 32.0f / 99.0f),
+                         f2_pack(-48.0f / 33.0f, -48.0f / 33.0f)),
+                    d, f2_pack(70.0f / 33.0f, 70.0f / 33.0f));
 #pragma unroll
-  for (int i = 0; i < 3; ++i) r = fma2(r, fma2(d ^ kSign, r, one), r);
-  const uint64_t w = mul2(mul2(two, E), r);
-  const uint64_t t = sub2(one, w) | (inner & kSign);  // 1 - w >= +0 before the sign
-  const uint64_t gl = mul2(mul2(half, g), add2(one, t));
-  return mul2(gl, u);
+  for (int i = 0; i < 2; ++i) r = fma2(r, fma2(d ^ kSign, r, one), r);
+  const uint64_t t = sub2(one, mul2(e2, r)) | (g & kSign);  // tanh(y): y has g's sign
+  return add2(one, t);
+}
+template <bool GATED>
+__device__ __forceinline__ uint64_t gelu_tanh_scaled2(uint64_t g, uint64_t u, uint64_t half_c) {
+  const uint64_t v = mul2(mul2(g, half_c), gelu_one_plus_tanh2(g));
+  if constexpr (GATED) return mul2(v, u);
+  return v;
 }
 
 }  // namespace frt

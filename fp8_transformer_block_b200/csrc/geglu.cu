@@ -6,8 +6,9 @@
 // quantized with the down projection's static input scale) and the bind
 // check that the FFN activation is the tanh-approximate GELU.
 // gelu_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), the tanh
-// form of Hendrycks & Gimpel's GELU (frt::gelu_tanh_mul2, shared with the
-// fused GEMM epilogue so both forms give the same codes).
+// form of Hendrycks & Gimpel's GELU (frt::gelu_one_plus_tanh2, shared with
+// the fused GEMM epilogue, whose arithmetic these kernels repeat step for
+// step so both forms give the same codes).
 #include "frt_common.cuh"
 
 namespace frt {
@@ -20,7 +21,9 @@ __global__ void geglu_kernel(int M, int H, const uint16_t* gu, long ld, const fl
   const long total = long(M) * h8;
   pdl_trigger();
   pdl_wait();
-  const float inv_os = __frcp_rn(__ldg(out_scale));  // quantize: h * (1 / scale)
+  // quantize: h * (1 / scale), the reciprocal folded into the GELU's 0.5
+  const float inv_os = __frcp_rn(__ldg(out_scale));
+  const uint64_t half_c = f2_pack(0.5f * inv_os, 0.5f * inv_os), half = f2_pack(0.5f, 0.5f);
   float mx = 0.0f;
   for (long g = blockIdx.x * long(blockDim.x) + threadIdx.x; g < total;
        g += long(gridDim.x) * blockDim.x) {
@@ -31,10 +34,12 @@ __global__ void geglu_kernel(int M, int H, const uint16_t* gu, long ld, const fl
     unpack8(__ldg(reinterpret_cast<const uint4*>(gu + m * ld + H + 8 * c)), uv);
 #pragma unroll
     for (int j = 0; j < 8; j += 2) {
-      const uint64_t h = gelu_tanh_mul2(f2_pack(gv[j], gv[j + 1]), f2_pack(uv[j], uv[j + 1]));
-      mx = absmax2(mx, h);
-      q[j] = __fmul_rn(f2_lo(h), inv_os);
-      q[j + 1] = __fmul_rn(f2_hi(h), inv_os);
+      const uint64_t gp = f2_pack(gv[j], gv[j + 1]), up = f2_pack(uv[j], uv[j + 1]);
+      const uint64_t opt = gelu_one_plus_tanh2(gp);
+      const uint64_t h = mul2(mul2(mul2(gp, half_c), opt), up);
+      if (amax) mx = absmax2(mx, mul2(mul2(mul2(gp, half), opt), up));
+      q[j] = f2_lo(h);
+      q[j + 1] = f2_hi(h);
     }
     *reinterpret_cast<uint2*>(hid8 + m * H + 8 * c) = pack8_e4m3(q);
   }
@@ -54,6 +59,7 @@ __global__ void gelu_kernel(int M, int H, const uint16_t* u, long ld, const floa
   pdl_trigger();
   pdl_wait();
   const float inv_os = __frcp_rn(__ldg(out_scale));
+  const uint64_t half_c = f2_pack(0.5f * inv_os, 0.5f * inv_os), half = f2_pack(0.5f, 0.5f);
   float mx = 0.0f;
   for (long g = blockIdx.x * long(blockDim.x) + threadIdx.x; g < total;
        g += long(gridDim.x) * blockDim.x) {
@@ -63,10 +69,12 @@ __global__ void gelu_kernel(int M, int H, const uint16_t* u, long ld, const floa
     unpack8(__ldg(reinterpret_cast<const uint4*>(u + m * ld + 8 * c)), uv);
 #pragma unroll
     for (int j = 0; j < 8; j += 2) {
-      const uint64_t h = gelu_tanh_mul2(f2_pack(uv[j], uv[j + 1]), f2_pack(1.0f, 1.0f));
-      mx = absmax2(mx, h);
-      q[j] = __fmul_rn(f2_lo(h), inv_os);
-      q[j + 1] = __fmul_rn(f2_hi(h), inv_os);
+      const uint64_t x = f2_pack(uv[j], uv[j + 1]);
+      const uint64_t opt = gelu_one_plus_tanh2(x);
+      const uint64_t h = mul2(mul2(x, half_c), opt);
+      if (amax) mx = absmax2(mx, mul2(mul2(x, half), opt));
+      q[j] = f2_lo(h);
+      q[j + 1] = f2_hi(h);
     }
     *reinterpret_cast<uint2*>(hid8 + m * H + 8 * c) = pack8_e4m3(q);
   }
@@ -82,8 +90,8 @@ __global__ void gelu_selftest_kernel(const float* x, float* y, long n) {
   for (long i = blockIdx.x * long(blockDim.x) + threadIdx.x; i < pairs;
        i += long(gridDim.x) * blockDim.x) {
     const bool two = 2 * i + 1 < n;
-    const uint64_t h =
-        gelu_tanh_mul2(f2_pack(x[2 * i], two ? x[2 * i + 1] : 0.0f), f2_pack(1.0f, 1.0f));
+    const uint64_t h = gelu_tanh_scaled2<false>(f2_pack(x[2 * i], two ? x[2 * i + 1] : 0.0f), 0,
+                                                f2_pack(0.5f, 0.5f));
     y[2 * i] = f2_lo(h);
     if (two) y[2 * i + 1] = f2_hi(h);
   }

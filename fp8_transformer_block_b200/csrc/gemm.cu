@@ -279,17 +279,21 @@ __device__ __forceinline__ void load_bias32(const GemmParams& p, int n, uint4 (&
 }
 
 // v = bf16(acc * alpha [+ bias]) as a float, in place: the value the plain
-// epilogue stores and the gated epilogues and the rotation start from.
+// epilogue stores and the gated epilogues start from.  Paired fp32
+// instructions (each lane rounded as the scalar operation), one bf16x2
+// rounding per pair.
 __device__ __forceinline__ void scale_bias32(const GemmParams& p, float (&v)[32],
-                                             const uint4 (&b4)[4], float alpha) {
+                                             const uint4 (&b4)[4], uint64_t alpha2) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    float b[8];
-    unpack8(b4[k], b);
+    const uint32_t w[4] = {b4[k].x, b4[k].y, b4[k].z, b4[k].w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float a = __fmul_rn(v[8 * k + j], alpha);
-      v[8 * k + j] = bf2f(f2bf(p.bias ? __fadd_rn(a, b[j]) : a));
+    for (int i = 0; i < 4; ++i) {
+      uint64_t a = mul2(f2_pack(v[8 * k + 2 * i], v[8 * k + 2 * i + 1]), alpha2);
+      if (p.bias) a = add2(a, bf16x2_to_f2(w[i]));
+      const uint64_t y = bf16x2_to_f2(pack_bf16x2(f2_lo(a), f2_hi(a)));
+      v[8 * k + 2 * i] = f2_lo(y);
+      v[8 * k + 2 * i + 1] = f2_hi(y);
     }
   }
 }
@@ -331,6 +335,8 @@ __device__ __forceinline__ void warp_rows_epilogue(const GemmParams& p, uint8_t*
                                                    float alpha, Load load, Done done) {
   if (p.epi == EPI_GEGLU || p.epi == EPI_GELU) {
     const float inv_os = __frcp_rn(__ldg(p.out_scale));
+    const uint64_t half_c = f2_pack(0.5f * inv_os, 0.5f * inv_os);
+    const uint64_t alpha2 = f2_pack(alpha, alpha);
     const bool geglu = p.epi == EPI_GEGLU;
 #pragma unroll 1
     for (int c0 = cb; c0 < ce; c0 += 4) {
@@ -343,25 +349,23 @@ __device__ __forceinline__ void warp_rows_epilogue(const GemmParams& p, uint8_t*
         float q[32];
         load(c, q);
         if (!geglu && c == ce - 1) done();
-        scale_bias32(p, q, bg, alpha);
-        const uint64_t inv2 = f2_pack(inv_os, inv_os);
+        scale_bias32(p, q, bg, alpha2);
         if (geglu) {
           float z[32];
           load(c + 4, z);
           if (c == ce - 1) done();
-          scale_bias32(p, z, bu, alpha);
+          scale_bias32(p, z, bu, alpha2);
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const uint64_t h = mul2(gelu_tanh_mul2(f2_pack(q[j], q[j + 1]), f2_pack(z[j], z[j + 1])),
-                                    inv2);
+            const uint64_t h = gelu_tanh_scaled2<true>(f2_pack(q[j], q[j + 1]),
+                                                       f2_pack(z[j], z[j + 1]), half_c);
             q[j] = f2_lo(h);
             q[j + 1] = f2_hi(h);
           }
         } else {
-          const uint64_t one = f2_pack(1.0f, 1.0f);
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const uint64_t h = mul2(gelu_tanh_mul2(f2_pack(q[j], q[j + 1]), one), inv2);
+            const uint64_t h = gelu_tanh_scaled2<false>(f2_pack(q[j], q[j + 1]), 0, half_c);
             q[j] = f2_lo(h);
             q[j + 1] = f2_hi(h);
           }
@@ -421,7 +425,8 @@ __device__ __forceinline__ void rows_direct_epilogue(const GemmParams& p, int m,
   if (p.epi == EPI_GEGLU || p.epi == EPI_GELU) {
     const bool geglu = p.epi == EPI_GEGLU;
     const float inv_os = __frcp_rn(__ldg(p.out_scale));
-    const uint64_t inv2 = f2_pack(inv_os, inv_os);
+    const uint64_t half_c = f2_pack(0.5f * inv_os, 0.5f * inv_os);
+    const uint64_t alpha2 = f2_pack(alpha, alpha);
     const int nout = ce;
 #pragma unroll 1
     for (int c = cb; c < nout; ++c) {
@@ -431,24 +436,23 @@ __device__ __forceinline__ void rows_direct_epilogue(const GemmParams& p, int m,
       float q[32];
       load(c, q);
       if (!geglu && c == nout - 1) done();
-      scale_bias32(p, q, bg, alpha);
+      scale_bias32(p, q, bg, alpha2);
       if (geglu) {
         float z[32];
         load(c + 4, z);
         if (c == nout - 1) done();
-        scale_bias32(p, z, bu, alpha);
+        scale_bias32(p, z, bu, alpha2);
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const uint64_t h =
-              mul2(gelu_tanh_mul2(f2_pack(q[j], q[j + 1]), f2_pack(z[j], z[j + 1])), inv2);
+          const uint64_t h = gelu_tanh_scaled2<true>(f2_pack(q[j], q[j + 1]),
+                                                     f2_pack(z[j], z[j + 1]), half_c);
           q[j] = f2_lo(h);
           q[j + 1] = f2_hi(h);
         }
       } else {
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const uint64_t h = mul2(gelu_tanh_mul2(f2_pack(q[j], q[j + 1]), f2_pack(1.0f, 1.0f)),
-                                  inv2);
+          const uint64_t h = gelu_tanh_scaled2<false>(f2_pack(q[j], q[j + 1]), 0, half_c);
           q[j] = f2_lo(h);
           q[j + 1] = f2_hi(h);
         }

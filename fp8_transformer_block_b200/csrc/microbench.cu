@@ -3,7 +3,13 @@
 // GPU at hand:
 //   * a dense FP8 tensor-core loop: one CTA per SM issuing back-to-back
 //     tcgen05.mma.kind::f8f6f4 (M 128, N 256, K 32, e4m3 x e4m3 -> fp32)
-//     from operands resident in shared memory, no data movement;
+//     from operands resident in shared memory, no data movement.  The
+//     tensor pipe's rate depends on the operand values (its power draw sets
+//     the clock under the power limit), so the operands are chosen: the e4m3
+//     codes of Gaussian values scaled like statically quantised activations
+//     and weights (amax near 448: sigma 100, random signs, every mantissa
+//     bit in play), or low-toggle codes (non-negative, one exponent bit
+//     cleared), which draw less power and run faster;
 //   * a device-to-device copy over buffers far larger than L2.
 // The caller times the launches (CUDA events) and converts: the MMA loop does
 // 2 * 128 * 256 * 32 * 4 * iters flops per CTA; the copy moves 2 * bytes.
@@ -19,7 +25,8 @@ constexpr int kMbA = 128 * 128;  // 128 rows x 128 K-bytes
 constexpr int kMbB = 256 * 128;  // 256 rows x 128 K-bytes
 constexpr uint64_t kMbWaitNs = 4000000000ull;
 
-__global__ void __launch_bounds__(kMbThreads, 1) mma_peak_kernel(int iters, int* status) {
+__global__ void __launch_bounds__(kMbThreads, 1) mma_peak_kernel(int iters, int operands,
+                                                                 int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -34,7 +41,27 @@ __global__ void __launch_bounds__(kMbThreads, 1) mma_peak_kernel(int iters, int*
     h ^= h >> 15;
     h *= 2246822519u;
     h ^= h >> 13;
-    h &= 0x6F6F6F6Fu;  // clears bits 4 and 7 of every byte: never 0x7F/0xFF (NaN)
+    if (operands == FRT_PEAK_OPERANDS_GAUSSIAN) {
+      // four codes of N(0, 100^2) values: each the sum of four uniform
+      // bytes (Irwin-Hall, mean 510, sd 147.8) standardised and scaled,
+      // rounded to e4m3 with saturation at +-448 (never NaN)
+      float z[8];
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        uint32_t g = h * 0x9E3779B1u + uint32_t(b + 1) * 0x85EBCA77u;
+        g ^= g >> 15;
+        g *= 0x2C1B3C6Du;
+        g ^= g >> 12;
+        g *= 0x297A2D39u;
+        g ^= g >> 15;
+        const float u = float(g & 0xFFu) + float((g >> 8) & 0xFFu) + float((g >> 16) & 0xFFu) +
+                        float(g >> 24);
+        z[b] = (u - 510.0f) * (100.0f / 147.8f);
+      }
+      h = pack8_e4m3(z).x;
+    } else {
+      h &= 0x6F6F6F6Fu;  // clears bits 4 and 7 of every byte: never 0x7F/0xFF (NaN)
+    }
     reinterpret_cast<uint32_t*>(smem)[i] = h;
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -110,10 +137,12 @@ __global__ void __launch_bounds__(256) copy_peak_kernel(const uint4* __restrict_
 }  // namespace
 }  // namespace frt
 
-extern "C" int frt_peak_fp8_mma(int ctas, int iters, void* stream) {
+extern "C" int frt_peak_fp8_mma(int ctas, int iters, int operands, void* stream) {
   frt::clear_error();
   FRT_REQUIRE(ctas >= 1 && ctas <= 4096 && iters >= 1, FRT_EINVAL,
               "ctas must be in [1, 4096] and iters >= 1");
+  FRT_REQUIRE(operands == FRT_PEAK_OPERANDS_GAUSSIAN || operands == FRT_PEAK_OPERANDS_LOW_TOGGLE,
+              FRT_EINVAL, "operands must be FRT_PEAK_OPERANDS_GAUSSIAN or _LOW_TOGGLE");
   constexpr int smem = frt::kMbA + frt::kMbB + 1024 + 64;
   auto kern = frt::mma_peak_kernel;
   if (frt::first_use(reinterpret_cast<const void*>(kern)) &&
@@ -121,7 +150,7 @@ extern "C" int frt_peak_fp8_mma(int ctas, int iters, void* stream) {
           cudaSuccess)
     return frt::fail(FRT_ECUDA, "cudaFuncSetAttribute(mma_peak_kernel)");
   kern<<<ctas, frt::kMbThreads, smem, static_cast<cudaStream_t>(stream)>>>(
-      iters, frt::device_status_ptr());
+      iters, operands, frt::device_status_ptr());
   return frt::check_launch("mma_peak_kernel");
 }
 

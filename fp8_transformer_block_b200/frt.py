@@ -26,6 +26,7 @@ FRT_NORM_ADARMS, FRT_NORM_LAYERNORM_TABLE = 0, 1
 FRT_PACK_CONCAT, FRT_PACK_QK_INTERLEAVE, FRT_PACK_GATE_UP_BLOCKS = 0, 1, 2
 FRT_EPI_BF16, FRT_EPI_GEGLU_E4M3, FRT_EPI_GELU_E4M3 = 0, 1, 2
 FRT_CHAIN_FUSED_ROPE, FRT_CHAIN_UNFUSED = 0, 1
+FRT_PEAK_OPERANDS_GAUSSIAN, FRT_PEAK_OPERANDS_LOW_TOGGLE = 0, 1
 
 STATUS_NAMES = {0: "FRT_OK", -1: "FRT_EINVAL", -2: "FRT_ESHAPE",
                 -3: "FRT_EALIGN", -4: "FRT_ERANGE", -5: "FRT_ECUDA",
@@ -117,7 +118,7 @@ _SIGS = {
     "frt_ada_rms_tail": (_i, [_i, _i, _f, _p, _p, _p, _l, _p, _l, _p, _p]),
     "frt_style_project": (_i, [_i, _i, _i, _p, _l, _p, _l, _p, _p, _l, _p, _l, _i, _p]),
     "frt_gemm_plan_info": (_i, [_i, _i, _i, _i, _p, _i]),
-    "frt_peak_fp8_mma": (_i, [_i, _i, _p]),
+    "frt_peak_fp8_mma": (_i, [_i, _i, _i, _p]),
     "frt_peak_copy": (_i, [_p, _p, C.c_size_t, _p]),
 }
 
@@ -323,9 +324,11 @@ def frt_gemm_plan_info(M, N, K, epilogue=0) -> dict:
     return dict(zip(_PLAN_KEYS, list(buf)))
 
 
-def frt_peak_fp8_mma(ctas: int, iters: int, stream=None) -> None:
-    """Launch the dense FP8 tensor-core loop (the library's peak probe)."""
-    _check(_lib.frt_peak_fp8_mma(ctas, iters, _stream(stream)), "frt_peak_fp8_mma")
+def frt_peak_fp8_mma(ctas: int, iters: int,
+                     operands: int = FRT_PEAK_OPERANDS_GAUSSIAN, stream=None) -> None:
+    """Launch the dense FP8 tensor-core loop (the library's peak probe) on the
+    operand codes `operands` names."""
+    _check(_lib.frt_peak_fp8_mma(ctas, iters, operands, _stream(stream)), "frt_peak_fp8_mma")
 
 
 def frt_peak_copy(src, dst, nbytes: int, stream=None) -> None:

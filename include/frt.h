@@ -495,15 +495,25 @@ int frt_selftest_gelu(const float* x, float* y, long n, void* stream);
 /* The library's own peak probes (no counterpart on the pages).             */
 /* ----------------------------------------------------------------------- */
 
+/* Operand values of the FP8 probe (the tensor pipe's rate depends on them:
+ * its power draw sets the clock under the board's power limit). */
+enum {
+  FRT_PEAK_OPERANDS_GAUSSIAN = 0,  /* e4m3 codes of N(0, 100^2): random signs and
+                                      mantissas, amax near 448, like statically
+                                      quantised activations and weights */
+  FRT_PEAK_OPERANDS_LOW_TOGGLE = 1 /* non-negative codes with bit 4 cleared */
+};
+
 /*
  * Dense FP8 tensor-core loop: `ctas` CTAs (one per SM is the intended use)
  * each issue 4 * iters tcgen05.mma.kind::f8f6f4 (M 128, N 256, K 32,
  * e4m3 x e4m3 -> fp32 in TMEM) back to back from operands already in shared
- * memory: 2 * 128 * 256 * 128 * iters flops per CTA and no memory traffic.
- * The caller times the launch on `stream` (asynchronous).  FRT_EINVAL for
- * ctas outside [1, 4096] or iters < 1.
+ * memory, filled on the device with the codes `operands` names: 2 * 128 *
+ * 256 * 128 * iters flops per CTA and no memory traffic.  The caller times
+ * the launch on `stream` (asynchronous).  FRT_EINVAL for ctas outside
+ * [1, 4096], iters < 1 or an unknown `operands`.
  */
-int frt_peak_fp8_mma(int ctas, int iters, void* stream);
+int frt_peak_fp8_mma(int ctas, int iters, int operands, void* stream);
 
 /*
  * Device-to-device copy of `bytes` (16-byte aligned pointers, a multiple

@@ -217,5 +217,6 @@ def test_output_side_validation(frt):
     assert q(sp, 0, 64, 64, A16, 64, A16, 64, None, A16, 64, A16, 192, 0, None) == frt.FRT_OK
     # FFN half: no descriptor; the peak probe: no CTAs
     assert q("frt_ffn_layer", None, None) == frt.FRT_EINVAL
-    assert q("frt_peak_fp8_mma", 0, 10, None) == frt.FRT_EINVAL
+    assert q("frt_peak_fp8_mma", 0, 10, 0, None) == frt.FRT_EINVAL
+    assert q("frt_peak_fp8_mma", 1, 10, 2, None) == frt.FRT_EINVAL
     assert q("frt_peak_copy", A16 + 4, A16, 64, None) == frt.FRT_EALIGN

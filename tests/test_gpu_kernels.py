@@ -521,14 +521,15 @@ def test_peak_probes_run_and_are_plausible(rt):
     frt, runtime, torch = rt
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    frt.frt_peak_fp8_mma(sms, 200)
-    ev[0].record()
-    frt.frt_peak_fp8_mma(sms, 2000)
-    ev[1].record()
-    _sync(torch)
-    assert frt.frt_device_status(True) == frt.FRT_OK
-    tflops = 2.0 * 128 * 256 * 128 * 2000 * sms / (ev[0].elapsed_time(ev[1]) * 1e-3) / 1e12
-    assert 300 < tflops < 6000, tflops   # dense e4m3 on one B200: a few PFLOP/s
+    for operands in (frt.FRT_PEAK_OPERANDS_GAUSSIAN, frt.FRT_PEAK_OPERANDS_LOW_TOGGLE):
+        frt.frt_peak_fp8_mma(sms, 200, operands)
+        ev[0].record()
+        frt.frt_peak_fp8_mma(sms, 2000, operands)
+        ev[1].record()
+        _sync(torch)
+        assert frt.frt_device_status(True) == frt.FRT_OK
+        tflops = 2.0 * 128 * 256 * 128 * 2000 * sms / (ev[0].elapsed_time(ev[1]) * 1e-3) / 1e12
+        assert 300 < tflops < 6000, tflops   # dense e4m3 on one B200: a few PFLOP/s
     n = 64 << 20
     src = torch.randint(0, 255, (n,), dtype=torch.uint8, device="cuda")
     dst = torch.zeros_like(src)
