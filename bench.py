@@ -58,17 +58,17 @@ FP8_PER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 # counts only while the hash of the kernel's sources matches the one the
 # counters were taken on (else the line reports traffic null).
 KERNEL_SOURCES = {
-    "gemm": ("gemm.cu", "frt_sm100.cuh"),
+    "gemm": ("gemm.cu", "frt_sm100.cuh", "frt_common.cuh"),
     "producer": ("producer.cu", "frt_common.cuh", "frt_sm100.cuh", "frt_prefix.cuh"),
     "prefix_copy": ("rope.cu", "frt_prefix.cuh"),
     "style": ("style.cu", "frt_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("vla_action_expert", "gemm_rope_kv"): (5_428_224, "b5f3b77dce68174e"),
-    ("video_dit", "gemm_rope_kv"): (165_660_928, "b5f3b77dce68174e"),
-    ("gateup_mlp", "gemm_gateup_geglu"): (73_067_264, "b5f3b77dce68174e"),
-    ("style_stack18", "style_project"): (58_446_592 + 512, "164dc7c9f25cad55"),
-    ("style_vla18", "style_project"): (932_188_672 + 466_176, "164dc7c9f25cad55"),
+    ("vla_action_expert", "gemm_rope_kv"): (5_427_968, "47b626f9a992e5e7"),
+    ("video_dit", "gemm_rope_kv"): (58_575_616 + 110_788_352, "47b626f9a992e5e7"),
+    ("gateup_mlp", "gemm_gateup_geglu"): (69_275_648 + 4_848_128, "47b626f9a992e5e7"),
+    ("style_stack18", "style_project"): (58_446_336 + 5_888, "41d4aa014b38bc81"),
+    ("style_vla18", "style_project"): (932_082_432 + 1_793_024, "41d4aa014b38bc81"),
 }
 
 
