@@ -64,9 +64,9 @@ KERNEL_SOURCES = {
     "style": ("style.cu", "frt_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("vla_action_expert", "gemm_rope_kv"): (5_427_968, "47b626f9a992e5e7"),
-    ("video_dit", "gemm_rope_kv"): (58_575_616 + 110_788_352, "47b626f9a992e5e7"),
-    ("gateup_mlp", "gemm_gateup_geglu"): (69_275_648 + 4_848_128, "47b626f9a992e5e7"),
+    ("vla_action_expert", "gemm_rope_kv"): (5_427_968, "61e0f042b56e0b91"),
+    ("video_dit", "gemm_rope_kv"): (58_575_616 + 110_788_352, "61e0f042b56e0b91"),
+    ("gateup_mlp", "gemm_gateup_geglu"): (69_275_648 + 4_848_128, "61e0f042b56e0b91"),
     ("style_stack18", "style_project"): (58_446_336 + 5_888, "41d4aa014b38bc81"),
     ("style_vla18", "style_project"): (932_082_432 + 1_793_024, "41d4aa014b38bc81"),
 }

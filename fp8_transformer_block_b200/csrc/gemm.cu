@@ -2284,23 +2284,17 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name only stands in for the symbol; the address the kernels
-// need comes from cudaGetSymbolAddress, once per device, with that device
-// current (the first call on a device does this).
+// need comes from cudaGetSymbolAddress, looked up on every call (cheap, no
+// allocation), so no address outlives the context it belongs to (a device
+// reset or a new primary context gives the next call the new address).
 int noalloc_scratch(void** out) {
-  static std::mutex mu;
-  static void* addr[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-    return fail(FRT_ECUDA, "no current CUDA device for the static scratch");
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(FRT_ECUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
-    addr[dev] = p;
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p) {
+    cudaGetLastError();
+    return fail(FRT_ECUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
   }
-  *out = addr[dev];
+  *out = p;
   return FRT_OK;
 }
 

@@ -210,11 +210,11 @@ int frt_packed_fp8_gemm(int M, int N, int K, const frt_e4m3* x8,
  * need more are rejected with FRT_ERANGE (nothing is launched).  The call
  * allocates nothing.  Every argument is checked on the host first, exactly
  * as frt_packed_fp8_gemm checks them; a rejected call returns its code
- * without enqueueing anything.  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) and keeps it; make that
- * first call before any stream capture.  The kept address is valid while
- * the device's primary context lives: after cudaDeviceReset the entry
- * point must not be called again in the same process.  Every call shares
+ * without enqueueing anything.  Each call looks up the array's device
+ * address in the current context (cudaGetSymbolAddress: no allocation, no
+ * launch), so a call after cudaDeviceReset finds the array of the new
+ * context; make the first call on a device outside any stream capture (it
+ * may load the library's device code).  Every call shares
  * the one array and zeroes its split counters first (a stream-ordered
  * memset): calls that may overlap on the GPU (other streams, other
  * threads) race on it and must be serialised by the caller.
