@@ -492,6 +492,87 @@ def test_geglu_fused_epilogue(rt, M, H):
     assert_codes(runtime.u8_host(h1), ref_a, what="standalone GEGLU vs oracle")
 
 
+@pytest.mark.parametrize("scale_div", [8.0, 64.0])
+def test_gelu_requant_saturates(rt, scale_div):
+    """Output scales at amax / 448 / scale_div: a large share of the GEGLU and
+    GELU values lie beyond +-448 and must saturate to codes 0x7E / 0xFE (the
+    pages' clamp-then-round quantizer), never the NaN codes 0x7F / 0xFF; the
+    rest, down to e4m3's subnormal codes, at the code bar against the
+    oracle.  The standalone kernels and the fused GEGLU epilogue (the same
+    device GELU) on the same values."""
+    frt, runtime, torch = rt
+    rng = np.random.default_rng(41)
+    M, H = 128, 1024
+    gu = bf16_bits(np.concatenate([rng.standard_normal((M, H)) * 3,
+                                   rng.standard_normal((M, H)) * 2], 1))
+
+    def gelu64(x):  # values well past the clamp, where no rounding can matter
+        return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
+
+    def f64(bits):
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+    _, amax = oracle.geglu_quant(gu, 1.0)
+    a = amax / 448.0 / scale_div
+    ref, _ = oracle.geglu_quant(gu, a)
+    sat = np.abs(gelu64(f64(gu[:, :H])) * f64(gu[:, H:])) / a > 460.0
+    assert sat.mean() > 0.005, sat.mean()      # the case is exercised
+    assert ((ref[sat] & 0x7F) == 0x7E).all()
+    hid = runtime.empty_u8(M, H)
+    frt.frt_geglu_quant_fp8(M, H, runtime.bf16_dev(gu), 2 * H, runtime.scale_dev(a), hid)
+    _sync(torch)
+    got = runtime.u8_host(hid)
+    assert not ((got & 0x7F) == 0x7F).any(), "GEGLU produced NaN codes"
+    assert np.array_equal(got[sat], ref[sat])
+    assert_codes(got, ref, what="saturating GEGLU vs oracle")
+    # GELU alone on the gate half
+    u = np.ascontiguousarray(gu[:, :H])
+    _, amax_u = oracle.gelu_quant(u, 1.0)
+    au = amax_u / 448.0 / scale_div
+    ref_u, _ = oracle.gelu_quant(u, au)
+    sat_u = np.abs(gelu64(f64(u))) / au > 460.0
+    assert sat_u.mean() > 0.005, sat_u.mean()
+    assert ((ref_u[sat_u] & 0x7F) == 0x7E).all()
+    hu = runtime.empty_u8(M, H)
+    frt.frt_gelu_quant_fp8(M, H, runtime.bf16_dev(u), H, runtime.scale_dev(au), hu)
+    _sync(torch)
+    got_u = runtime.u8_host(hu)
+    assert not ((got_u & 0x7F) == 0x7F).any(), "GELU produced NaN codes"
+    assert np.array_equal(got_u[sat_u], ref_u[sat_u])
+    assert_codes(got_u, ref_u, what="saturating GELU vs oracle")
+    # the fused GEGLU epilogue at the same kind of scale, against the
+    # oracle's GEGLU on the bf16 gate/up values the same GEMM writes
+    D = 512
+    mw = synth.mlp_weights(D, H, 23)
+    x8 = runtime.u8_dev(_x8_codes(M, D, 79))
+    sc = runtime.scale_dev(0.02)
+    blk = runtime.pack([mw["gate"], mw["up"]], layout=frt.FRT_PACK_GATE_UP_BLOCKS)
+    order = gate_up_block_order(H)
+    g2 = runtime.empty_bf16(M, 2 * H)
+    wsb = frt.frt_gemm_workspace_size(M, 2 * H, D)
+    frt.frt_packed_fp8_gemm(M, 2 * H, D, x8, blk.w8, sc, blk.w_scale, None,
+                            frt.FRT_EPI_BF16, g2, 2 * H, None, runtime.workspace(wsb), wsb)
+    _sync(torch)
+    gu_cat = np.empty((M, 2 * H), np.uint16)
+    gu_cat[:, order] = runtime.bf16_host(g2)
+    _, amax2 = oracle.geglu_quant(gu_cat, 1.0)
+    a2 = amax2 / 448.0 / scale_div
+    ref2, _ = oracle.geglu_quant(gu_cat, a2)
+    h2 = torch.full((M, H), 0x7F, dtype=torch.uint8, device="cuda")
+    wsb2 = frt.frt_gemm_workspace_size(M, 2 * H, D, frt.FRT_EPI_GEGLU_E4M3)
+    frt.frt_packed_fp8_gemm(M, 2 * H, D, x8, blk.w8, sc, blk.w_scale, None,
+                            frt.FRT_EPI_GEGLU_E4M3, h2, H, runtime.scale_dev(a2),
+                            runtime.workspace(wsb2), wsb2)
+    _sync(torch)
+    assert frt.frt_device_status(True) == frt.FRT_OK
+    fused = runtime.u8_host(h2)
+    sat2 = np.abs(gelu64(f64(gu_cat[:, :H])) * f64(gu_cat[:, H:])) / a2 > 460.0
+    assert sat2.mean() > 0.005, sat2.mean()
+    assert not ((fused & 0x7F) == 0x7F).any(), "fused GEGLU produced NaN codes"
+    assert np.array_equal(fused[sat2], ref2[sat2])
+    assert_codes(fused, ref2, what="saturating fused GEGLU vs oracle")
+
+
 def test_device_gelu_error_bound(rt):
     """The device GELU (tanh from the exponential) against an fp64
     evaluation of the tanh-form GELU: within 5e-7 * max(1, |x|) plus four
