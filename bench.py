@@ -292,7 +292,12 @@ class ChainRunner:
                             ("res", "delta", "prev_gate", "style")}
         self.x8 = rt.empty_u8(rows, D)
         self.q = [rt.empty_bf16(B, M, w.hq, w.hd) for _ in range(2)]
-        self.ws_bytes = frt.frt_gemm_workspace_size(rows, N, D)
+        # the chain's own workspace size (its GEMM's split-K, or the counters
+        # of the producer-in-the-grid form at small M)
+        self.ws_bytes = frt.frt_chain_workspace_size(rt.chain_desc(
+            B=B, M=M, D=D, hq=w.hq, hkv=w.hkv, hd=w.hd,
+            norm_mode=(frt.FRT_NORM_LAYERNORM_TABLE if self.dit else frt.FRT_NORM_ADARMS),
+            flags=frt.FRT_CHAIN_FUSED_ROPE))
         self.ws = rt.workspace(self.ws_bytes)
         self.calibrate(synth)
         ks = []

@@ -93,7 +93,11 @@ class AdaRmsLayerStack:
             })
         self.layers_host = layers
         N = (w.hq + 2 * w.hkv) * w.hd
-        self.ws_bytes = max(frt.frt_gemm_workspace_size(rows, N, D),
+        self.ws_bytes = max(frt.frt_chain_workspace_size(rt.chain_desc(
+                                B=w.B, M=w.M, D=D, hq=w.hq, hkv=w.hkv, hd=w.hd,
+                                norm_mode=frt.FRT_NORM_ADARMS,
+                                flags=frt.FRT_CHAIN_FUSED_ROPE)),
+                            frt.frt_gemm_workspace_size(rows, N, D),
                             frt.frt_gemm_workspace_size(rows, D, D),
                             frt.frt_gemm_workspace_size(rows, 2 * H, D, frt.FRT_EPI_GEGLU_E4M3),
                             frt.frt_gemm_workspace_size(rows, 2 * H, D),

@@ -79,17 +79,23 @@ def test_chain_layer_adarms(rt, name, fused):
     kc = _sentinel_cache(torch, w.B, w.T, w.hkv, w.hd)
     vc = _sentinel_cache(torch, w.B, w.T, w.hkv, w.hd)
     qkv = runtime.empty_bf16(w.rows, w.N) if not fused else None
+    # the descriptor holds raw pointers: every tensor it names must outlive
+    # the call (a freed block may be handed to the workspace allocated below)
+    delta = runtime.bf16_dev(inp["delta"])
+    prev_gate = runtime.bf16_dev(inp["prev_gate"])
+    style = runtime.bf16_dev(inp["style"])
+    act = runtime.scale_dev(a)
+    pkd = None if prefix is None else runtime.bf16_dev(prefix[0])
+    pvd = None if prefix is None else runtime.bf16_dev(prefix[1])
     d = runtime.chain_desc(
         B=w.B, M=w.M, D=w.D, hq=w.hq, hkv=w.hkv, hd=w.hd, P=w.P, T=w.T,
         eps=w.eps, norm_mode=frt.FRT_NORM_ADARMS,
         flags=frt.FRT_CHAIN_FUSED_ROPE if fused else frt.FRT_CHAIN_UNFUSED,
-        res=res, delta=runtime.bf16_dev(inp["delta"]),
-        prev_gate=runtime.bf16_dev(inp["prev_gate"]), gate_row_stride=0,
-        style=runtime.bf16_dev(inp["style"]), style_row_stride=0,
-        gate_out=gate_out, act_scale=runtime.scale_dev(a), x8=x8, w8=pk.w8,
+        res=res, delta=delta, prev_gate=prev_gate, gate_row_stride=0,
+        style=style, style_row_stride=0,
+        gate_out=gate_out, act_scale=act, x8=x8, w8=pk.w8,
         w_scale=pk.w_scale, rope=rope, q_out=q, k_cache=kc, v_cache=vc,
-        prefix_k=None if prefix is None else runtime.bf16_dev(prefix[0]),
-        prefix_v=None if prefix is None else runtime.bf16_dev(prefix[1]),
+        prefix_k=pkd, prefix_v=pvd,
         prefix_T_src=0 if prefix is None else prefix[0].shape[2],
         prefix_interleave=1,
         qkv=qkv)
@@ -147,13 +153,15 @@ def test_chain_layer_video_dit_sampled(rt):
     q = runtime.empty_bf16(w.B, w.M, w.hq, w.hd)
     kc = _sentinel_cache(torch, w.B, w.T, w.hkv, w.hd)
     vc = _sentinel_cache(torch, w.B, w.T, w.hkv, w.hd)
+    # tensors the descriptor points at, alive through the call
+    xd, tembd = runtime.bf16_dev(inp["x"]), runtime.bf16_dev(inp["temb"])
+    table, act = runtime.f32_dev(inp["table"]), runtime.scale_dev(a)
     d = runtime.chain_desc(
         B=w.B, M=w.M, D=w.D, hq=w.hq, hkv=w.hkv, hd=w.hd, P=w.P, T=w.T,
         eps=w.eps, norm_mode=frt.FRT_NORM_LAYERNORM_TABLE,
-        flags=frt.FRT_CHAIN_FUSED_ROPE, x=runtime.bf16_dev(inp["x"]),
-        temb=runtime.bf16_dev(inp["temb"]), chunks=6,
-        table=runtime.f32_dev(inp["table"]), shift_idx=0, scale_idx=1,
-        act_scale=runtime.scale_dev(a), x8=x8, w8=pk.w8, w_scale=pk.w_scale,
+        flags=frt.FRT_CHAIN_FUSED_ROPE, x=xd, temb=tembd, chunks=6,
+        table=table, shift_idx=0, scale_idx=1,
+        act_scale=act, x8=x8, w8=pk.w8, w_scale=pk.w_scale,
         bias=pk.bias, rope=rope, q_out=q, k_cache=kc, v_cache=vc)
     wsb = frt.frt_chain_workspace_size(d)
     assert wsb == 0
